@@ -1,0 +1,280 @@
+"""Seeded synthetic workloads for paged decode attention.
+
+This module only draws inputs: random values, context lengths, a shuffled
+pool of physical blocks and the block tables that a simple allocator hands
+out.  It holds none of the attention arithmetic and imports neither the CUDA
+binding nor the oracle, so both sides can be fed the same arrays.
+
+The allocator here plays the Block Manager of the pages (page "Implementing
+teaching PagedAttention: reading the historical KV cache from the block
+table", opening section: free blocks are handed out for prefill and a slot
+is appended for each decode step).  It records where it put every token; the
+slot of a sequence's newest token is reported as the flat integer
+``physical_block_id * block_size + block_offset`` of the place it reserved.
+
+Workload recipes (all values N(0, 1); bf16 values are drawn in fp32 and
+rounded to nearest-even by torch's cast; every array is host memory):
+
+``tiny_fp32``
+    batch 3, 4 query / 4 KV heads, head_dim 64, block_size 4, 16 blocks,
+    context_lens [5, 9, 12]; sequence 0's table is fixed to [7, 2, 9], the
+    other tables are drawn without replacement from the remaining blocks.
+``gqa_bf16``
+    batch 32, 32 / 8 heads, head_dim 128, block_size 16, context lengths
+    uniform in [128, 2048], blocks a seeded permutation of a pool with 20 %
+    slack.
+``mixed_bf16``
+    batch 128, 32 / 8 heads, head_dim 128, block_size 16, lengths drawn from
+    {128: 50 %, 4096: 35 %, 16000: 15 %} plus uniform jitter in [0, 15],
+    scattered tables from a 20 %-slack pool.
+``long_bf16``
+    batch 4, context 131072 each, 32 / 8 heads, head_dim 128,
+    block_size 16, a seeded permutation of exactly the blocks needed,
+    512-token partitions.
+``mqa_prefix_bf16``
+    batch 256, 64 query heads / 1 KV head, head_dim 128, block_size 32;
+    every table starts with the same 64 shared prefix blocks (2048 tokens)
+    followed by a private suffix of uniform [1, 1024] tokens in scattered
+    blocks (20 % slack).
+
+In every workload but ``tiny_fp32`` the last token of each sequence is the
+token of the current decode step: its K/V rows are returned in
+``k_new``/``v_new`` with the slot reserved for it in ``slot_mapping``, and
+its place in the cache is filled with NaN until the cache write runs.  Slots
+of unreferenced blocks and slots past each context length are NaN too, so a
+kernel that reads outside the visible history produces NaN.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+
+DTYPE_F32 = "f32"
+DTYPE_BF16 = "bf16"
+
+WORKLOADS = ("tiny_fp32", "gqa_bf16", "mixed_bf16", "long_bf16", "mqa_prefix_bf16")
+
+_BF16_NAN = np.uint16(0x7FC0)
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    dtype: str  # "f32" (float32 arrays) or "bf16" (uint16 arrays of bf16 bits)
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    max_blocks: int
+    q: np.ndarray  # [B, Hq, D]
+    key_cache: np.ndarray  # [NB, bs, Hkv, D]
+    value_cache: np.ndarray  # [NB, bs, Hkv, D]
+    block_tables: np.ndarray  # [B, MB] int32, unused entries -1
+    context_lens: np.ndarray  # [B] int32
+    k_new: Optional[np.ndarray] = None  # [N, Hkv, D]
+    v_new: Optional[np.ndarray] = None
+    slot_mapping: Optional[np.ndarray] = None  # [N] int64
+    partition_tokens: Optional[int] = None
+    seed: int = 0
+    description: str = ""
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == DTYPE_F32 else 2
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+
+def to_storage(values_f32: np.ndarray, dtype: str) -> np.ndarray:
+    """fp32 values -> storage array: float32 as is, bf16 as uint16 bits (RNE)."""
+    if dtype == DTYPE_F32:
+        return np.ascontiguousarray(values_f32, dtype=np.float32)
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(values_f32, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.uint16).numpy().copy()
+
+
+def _nan_value(dtype: str):
+    return np.float32("nan") if dtype == DTYPE_F32 else _BF16_NAN
+
+
+def _normal_storage(rng: np.random.Generator, shape, dtype: str,
+                    chunk: int = 1 << 26) -> np.ndarray:
+    """N(0,1) draws in storage format, generated in chunks to bound memory."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32 if dtype == DTYPE_F32 else np.uint16)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        out[s:e] = to_storage(rng.standard_normal(e - s, dtype=np.float32), dtype)
+    return out.reshape(shape)
+
+
+def _pages(ctx: int, bs: int) -> int:
+    return (ctx + bs - 1) // bs
+
+
+def _finish(name, dtype, rng, B, Hq, Hkv, D, bs, NB, MB, ctx, tables,
+            new_tokens: bool, partition_tokens=None, seed=0, description=""):
+    """Draw q and cache contents, poison unused slots, peel off new tokens."""
+    q = _normal_storage(rng, (B, Hq, D), dtype)
+    kc = _normal_storage(rng, (NB, bs, Hkv, D), dtype)
+    vc = _normal_storage(rng, (NB, bs, Hkv, D), dtype)
+    nan = _nan_value(dtype)
+    # Slots that hold a visible token of some sequence.
+    live = np.zeros((NB, bs), dtype=bool)
+    for b in range(B):
+        for lb in range(_pages(int(ctx[b]), bs)):
+            n_valid = min(bs, int(ctx[b]) - lb * bs)
+            live[tables[b, lb], :n_valid] = True
+    kc[~live] = nan
+    vc[~live] = nan
+    k_new = v_new = slots = None
+    if new_tokens:
+        rows = [b for b in range(B) if ctx[b] > 0]
+        k_new = np.empty((len(rows), Hkv, D), dtype=kc.dtype)
+        v_new = np.empty_like(k_new)
+        slots = np.empty(len(rows), dtype=np.int64)
+        for i, b in enumerate(rows):
+            t = int(ctx[b]) - 1
+            pb, off = int(tables[b, t // bs]), t % bs  # where the allocator put it
+            k_new[i] = kc[pb, off]
+            v_new[i] = vc[pb, off]
+            kc[pb, off] = nan
+            vc[pb, off] = nan
+            slots[i] = pb * bs + off
+    return Workload(name=name, dtype=dtype, batch=B, num_q_heads=Hq,
+                    num_kv_heads=Hkv, head_dim=D, block_size=bs, num_blocks=NB,
+                    max_blocks=MB, q=q, key_cache=kc, value_cache=vc,
+                    block_tables=tables, context_lens=ctx.astype(np.int32),
+                    k_new=k_new, v_new=v_new, slot_mapping=slots,
+                    partition_tokens=partition_tokens, seed=seed,
+                    description=description)
+
+
+def _scattered_tables(rng, ctx, bs, MB, slack=0.2, prefix_blocks=0):
+    """Tables from a seeded permutation of a pool with `slack` spare blocks.
+
+    With prefix_blocks > 0 every table starts with the same prefix blocks
+    (the first ones of the permutation); suffix pages follow."""
+    B = len(ctx)
+    need = [_pages(int(c), bs) - prefix_blocks for c in ctx]
+    total = prefix_blocks + sum(need)
+    NB = int(math.ceil((1.0 + slack) * total))
+    perm = rng.permutation(NB).astype(np.int32)
+    tables = np.full((B, MB), -1, dtype=np.int32)
+    prefix = perm[:prefix_blocks]
+    pos = prefix_blocks
+    for b in range(B):
+        tables[b, :prefix_blocks] = prefix
+        tables[b, prefix_blocks:prefix_blocks + need[b]] = perm[pos:pos + need[b]]
+        pos += need[b]
+    return tables, NB
+
+
+def make_workload(name: str, seed: int = 0, batch: Optional[int] = None) -> Workload:
+    """Build one of the named workloads.  `batch` overrides the batch size
+    (used for reduced-size variants of the large workloads)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    if name == "tiny_fp32":
+        B, Hq, Hkv, D, bs, NB = 3, 4, 4, 64, 4, 16
+        ctx = np.array([5, 9, 12], dtype=np.int32)
+        MB = 3
+        tables = np.full((B, MB), -1, dtype=np.int32)
+        tables[0] = [7, 2, 9]
+        rest = np.array([x for x in range(NB) if x not in (7, 2, 9)], dtype=np.int32)
+        drawn = rng.choice(rest, size=_pages(9, bs) + _pages(12, bs), replace=False)
+        tables[1] = drawn[:3]
+        tables[2] = drawn[3:6]
+        return _finish(name, DTYPE_F32, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
+                       tables, new_tokens=False, seed=seed,
+                       description="B3 Hq4/Hkv4 D64 bs4 NB16 ctx[5,9,12] fp32")
+    if name == "gqa_bf16":
+        B = batch or 32
+        Hq, Hkv, D, bs = 32, 8, 128, 16
+        ctx = rng.integers(128, 2048, size=B, endpoint=True).astype(np.int32)
+        MB = _pages(2048, bs)
+        tables, NB = _scattered_tables(rng, ctx, bs, MB)
+        return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
+                       tables, new_tokens=True, seed=seed,
+                       description=f"B{B} Hq32/Hkv8 D128 bs16 ctx~U[128,2048] bf16")
+    if name == "mixed_bf16":
+        B = batch or 128
+        Hq, Hkv, D, bs = 32, 8, 128, 16
+        base = rng.choice(np.array([128, 4096, 16000]), size=B, p=[0.5, 0.35, 0.15])
+        jitter = rng.integers(0, 15, size=B, endpoint=True)
+        ctx = (base + jitter).astype(np.int32)
+        MB = _pages(16000 + 15, bs)
+        tables, NB = _scattered_tables(rng, ctx, bs, MB)
+        return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
+                       tables, new_tokens=True, seed=seed,
+                       description=f"B{B} Hq32/Hkv8 D128 bs16 ctx {{128,4096,16000}}+U[0,15] bf16")
+    if name == "long_bf16":
+        B = batch or 4
+        Hq, Hkv, D, bs, L = 32, 8, 128, 16, 131072
+        ctx = np.full(B, L, dtype=np.int32)
+        MB = _pages(L, bs)
+        tables, NB = _scattered_tables(rng, ctx, bs, MB, slack=0.0)
+        return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
+                       tables, new_tokens=True, partition_tokens=512, seed=seed,
+                       description=f"B{B} ctx131072 Hq32/Hkv8 D128 bs16 bf16, 512-token partitions")
+    if name == "mqa_prefix_bf16":
+        B = batch or 256
+        Hq, Hkv, D, bs, prefix = 64, 1, 128, 32, 2048
+        suffix = rng.integers(1, 1024, size=B, endpoint=True)
+        ctx = (prefix + suffix).astype(np.int32)
+        MB = _pages(prefix + 1024, bs)
+        tables, NB = _scattered_tables(rng, ctx, bs, MB, prefix_blocks=prefix // bs)
+        return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
+                       tables, new_tokens=True, seed=seed,
+                       description=f"B{B} Hq64/Hkv1 D128 bs32, 2048 shared prefix + U[1,1024] suffix, bf16")
+    raise ValueError(f"unknown workload {name!r}; known: {WORKLOADS}")
+
+
+def custom_workload(*, dtype: str, batch: int, num_q_heads: int, num_kv_heads: int,
+                    head_dim: int, block_size: int, context_lens, seed: int = 0,
+                    slack: float = 0.2, max_blocks: Optional[int] = None,
+                    new_tokens: bool = False) -> Workload:
+    """A workload with explicit context lengths (edge cases, sweeps)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    ctx = np.asarray(context_lens, dtype=np.int32)
+    need = max([_pages(int(c), block_size) for c in ctx] + [1])
+    MB = max_blocks if max_blocks is not None else need
+    tables, NB = _scattered_tables(rng, np.maximum(ctx, 0), block_size, MB, slack=slack)
+    NB = max(NB, 1)
+    return _finish("custom", dtype, rng, batch, num_q_heads, num_kv_heads, head_dim,
+                   block_size, NB, MB, ctx, tables,
+                   new_tokens=new_tokens, seed=seed,
+                   description=f"custom ctx={list(map(int, ctx))[:8]}...")
+
+
+def roofline_bytes(w: Workload, include_write: bool = True) -> int:
+    """Algorithmic HBM bytes of one decode step: unique K/V bytes of the
+    visible tokens (shared pages counted once), block tables, context
+    lengths, q and out, plus the new-token rows and slots when written."""
+    row = w.num_kv_heads * w.head_dim * w.elem_bytes
+    seen = set()
+    kv = 0
+    for b in range(w.batch):
+        ctx = int(w.context_lens[b])
+        for lb in range(_pages(ctx, w.block_size)):
+            pb = int(w.block_tables[b, lb])
+            n_valid = min(w.block_size, ctx - lb * w.block_size)
+            if pb in seen:
+                continue
+            seen.add(pb)
+            kv += 2 * n_valid * row
+    qo = 2 * w.batch * w.num_q_heads * w.head_dim * w.elem_bytes
+    meta = w.block_tables.size * 4 + w.context_lens.size * 4
+    extra = 0
+    if include_write and w.slot_mapping is not None:
+        # new rows read once and stored once, for K and for V
+        extra = 2 * (w.k_new.nbytes + w.v_new.nbytes) + w.slot_mapping.nbytes
+    return int(kv + qo + meta + extra)

@@ -1,0 +1,87 @@
+"""The seeded input generators: determinism and the structure each workload
+recipe promises (host only, no attention arithmetic involved)."""
+import numpy as np
+import pytest
+
+from paged_kv_cache_334_b200 import workloads as wl
+
+
+def test_tiny_recipe():
+    w = wl.make_workload("tiny_fp32", seed=0)
+    assert (w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks) == (3, 4, 4, 64, 4, 16)
+    assert list(w.context_lens) == [5, 9, 12]
+    assert list(w.block_tables[0]) == [7, 2, 9]
+    rest = np.concatenate([w.block_tables[1], w.block_tables[2]])
+    assert len(set(rest.tolist())) == 6 and not set(rest.tolist()) & {7, 2, 9}
+    assert w.q.dtype == np.float32 and w.key_cache.shape == (16, 4, 4, 64)
+    assert w.slot_mapping is None
+
+
+def test_determinism_and_seed_dependence():
+    a = wl.make_workload("gqa_bf16", seed=3, batch=4)
+    b = wl.make_workload("gqa_bf16", seed=3, batch=4)
+    c = wl.make_workload("gqa_bf16", seed=4, batch=4)
+    for f in ("q", "key_cache", "value_cache", "block_tables", "context_lens", "k_new", "slot_mapping"):
+        assert np.array_equal(getattr(a, f), getattr(b, f))
+    assert not np.array_equal(a.context_lens, c.context_lens)
+
+
+@pytest.mark.parametrize("name,batch", [("gqa_bf16", 8), ("mixed_bf16", 6), ("long_bf16", 1),
+                                        ("mqa_prefix_bf16", 8)])
+def test_structure(name, batch):
+    w = wl.make_workload(name, seed=0, batch=batch)
+    bs = w.block_size
+    assert w.dtype == wl.DTYPE_BF16 and w.q.dtype == np.uint16
+    pages = [(-(-int(c) // bs)) for c in w.context_lens]
+    assert max(pages) <= w.max_blocks
+    used = []
+    for b in range(w.batch):
+        row = w.block_tables[b]
+        assert np.all(row[:pages[b]] >= 0) and np.all(row[:pages[b]] < w.num_blocks)
+        assert np.all(row[pages[b]:] == -1)
+        used.extend(row[:pages[b]].tolist())
+    if name == "mqa_prefix_bf16":
+        prefix = w.block_tables[:, :64]
+        assert np.all(prefix == prefix[0])
+        assert np.all(w.context_lens >= 2049) and np.all(w.context_lens <= 3072)
+        suffix_blocks = [x for b in range(w.batch) for x in w.block_tables[b, 64:pages[b]]]
+        assert len(set(suffix_blocks)) == len(suffix_blocks)
+    else:
+        assert len(set(used)) == len(used)  # private pages
+    if name == "gqa_bf16":
+        assert np.all(w.context_lens >= 128) and np.all(w.context_lens <= 2048)
+    if name == "mixed_bf16":
+        assert all(any(0 <= c - x <= 15 for x in (128, 4096, 16000)) for c in w.context_lens)
+    if name == "long_bf16":
+        assert np.all(w.context_lens == 131072) and w.partition_tokens == 512
+    # the newest token's slot is reserved and poisoned until written
+    assert w.slot_mapping is not None and len(w.slot_mapping) == w.batch
+    nan_bits = 0x7FC0
+    for i, b in enumerate(range(w.batch)):
+        t = int(w.context_lens[b]) - 1
+        pb, off = int(w.block_tables[b, t // bs]), t % bs
+        assert w.slot_mapping[i] == pb * bs + off
+        assert np.all(w.key_cache[pb, off] == nan_bits)
+        assert not np.any(w.k_new[i] == nan_bits)
+
+
+def test_poison_marks_exactly_the_invisible_slots():
+    w = wl.make_workload("tiny_fp32", seed=0)
+    live = np.zeros((w.num_blocks, w.block_size), bool)
+    for b in range(w.batch):
+        for t in range(int(w.context_lens[b])):
+            live[w.block_tables[b, t // w.block_size], t % w.block_size] = True
+    nan_slot = np.isnan(w.key_cache).all(axis=(2, 3))
+    assert np.array_equal(nan_slot, ~live)
+    assert np.array_equal(np.isnan(w.value_cache).all(axis=(2, 3)), ~live)
+
+
+def test_roofline_bytes_counts_shared_prefix_once():
+    w = wl.make_workload("mqa_prefix_bf16", seed=0, batch=4)
+    row = w.num_kv_heads * w.head_dim * 2
+    kv_unique = 2 * row * (2048 + int(sum(w.context_lens - 2048)))
+    qo = 2 * w.batch * w.num_q_heads * w.head_dim * 2
+    meta = w.block_tables.size * 4 + w.batch * 4
+    write = 2 * (w.k_new.nbytes + w.v_new.nbytes) + w.slot_mapping.nbytes
+    assert wl.roofline_bytes(w) == kv_unique + qo + meta + write
+    assert wl.roofline_bytes(w, include_write=False) == kv_unique + qo + meta
