@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Benchmark of one paged decode-attention step on B200.
+
+A step is one pass of the hot path over one batch: the cache write of every
+sequence's newest token (pa_write_kv_cache via slot_mapping) followed by the
+fused paged decode (pa_decode), both through the C ABI.  The default workload
+is the bf16 GQA decode batch (batch 32, 32 query / 8 KV heads, head_dim 128,
+block_size 16, context lengths uniform in [128, 2048]); other workloads are
+selectable with --workload.
+
+Output: one JSON line on rank 0.  ``value`` is the achieved bandwidth on the
+algorithmic bytes of the step (unique K/V bytes of the visible tokens, block
+tables, context lengths, q, out and the new K/V rows) in GB/s, summed over
+ranks and divided by the slowest rank's time; each timed step is preceded by
+an L2 flush outside its CUDA-event pair.  ``e2e`` is the same metric with the
+per-step inputs copied from pinned host memory and the output read back
+inside the timed region.  ``roofline`` reports the decode kernel alone
+against the measured HBM copy bandwidth; ``cpu_baseline`` times the fp64 CPU
+oracle on the host cores (rank 0, one GPU only).
+
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own
+independent batch (seeded by rank); there is no data-path collective, only a
+barrier and max/sum reductions of the timings (weak scaling).
+
+``--impl reference`` times the fp64 CPU oracle itself as the reference arm
+(rank 0 only; other ranks exit at once).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from paged_kv_cache_334_b200 import workloads as wl  # noqa: E402
+
+METRIC = "decode-attention KV GB/s & fraction of B200 HBM peak; seq-tokens/s per step"
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCE = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc", "decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.md")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="gqa_bf16", choices=wl.WORKLOADS)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank decodes its own independent batch."""
+    return seed + 1000 * rank
+
+
+def init_dist(world: int, local: int, backend: str = "nccl"):
+    import torch
+    import torch.distributed as dist
+    if world <= 1:
+        return None
+    kw = {}
+    if backend == "nccl":
+        kw["device_id"] = torch.device("cuda", local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def reduce_scalar(x: float, op: str, dist=None, device=None) -> float:
+    """max / sum of a host scalar over ranks (identity with one rank)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        self.t0 = self.t1 = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.sel = str(device_index)
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "20", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            deadline = time.time() + 3.0
+            while time.time() < deadline and os.path.getsize(self.path) == 0:
+                time.sleep(0.01)
+        except Exception:
+            self.proc = None
+
+    def mark(self, which: str):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[1]), float(parts[2]), parts[3], parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.02 <= r[0] <= self.t1 + 0.02]
+        note = "samples inside the timed region"
+        if not inside:
+            after = [r for r in rows if self.t0 is not None and r[0] >= self.t0]
+            inside = after[:1] or rows[-1:]
+            note = "timed region shorter than the 20 ms sampling period: nearest sample"
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in inside for n, v in zip(names, r[4]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside), "note": note}
+
+
+# ---------------------------------------------------------------------------
+# measured peaks and ncu traffic
+# ---------------------------------------------------------------------------
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (of measured)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "6.65 TB/s fallback (of fallback)"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(os.path.dirname(DECODE_SOURCE))):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(os.path.dirname(DECODE_SOURCE), fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources for this workload; else None."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    want = decode_source_hash()
+    for line in text.splitlines():
+        parts = [p.strip() for p in line.strip().strip("|").split("|")]
+        if len(parts) >= 3 and parts[0] == workload and parts[1] == want:
+            try:
+                return float(parts[2])
+            except ValueError:
+                return None
+    return None
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def time_oracle(w, target_seconds: float, max_reps: int = 1000):
+    """Time the fp64 oracle's step (its own cache write + decode) on the host
+    cores, repeating the whole batch until about target_seconds elapsed, or
+    on a prefix of the batch when one pass is longer than that."""
+    import oracle
+    oracle.build()
+    sample = w
+    t_one = _oracle_step(w)
+    reps = 1
+    desc = f"full {w.name} batch ({w.batch} sequences)"
+    if t_one > target_seconds and w.batch > 1:
+        nb = max(1, int(w.batch * target_seconds / t_one))
+        sample = _prefix(w, nb)
+        t_one = _oracle_step(sample)
+        desc = f"first {nb} of {w.batch} sequences of {w.name}"
+    total = t_one
+    while total < target_seconds and reps < max_reps:
+        total += _oracle_step(sample)
+        reps += 1
+    per_step = total / reps
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return per_step, sample, cores, f"{desc}, {reps} repetition(s)"
+
+
+def _oracle_step(w) -> float:
+    import oracle
+    kc, vc = w.key_cache, w.value_cache
+    t0 = time.perf_counter()
+    if w.slot_mapping is not None:
+        oracle.write_kv_cache(kc, vc, w.k_new, w.v_new, w.slot_mapping)
+    oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, 1.0 / math.sqrt(w.head_dim))
+    return time.perf_counter() - t0
+
+
+def _prefix(w, nb):
+    import dataclasses
+    keep = w.slot_mapping is not None
+    return dataclasses.replace(
+        w, batch=nb, q=w.q[:nb].copy(), block_tables=w.block_tables[:nb].copy(),
+        context_lens=w.context_lens[:nb].copy(),
+        k_new=w.k_new[:nb].copy() if keep else None, v_new=w.v_new[:nb].copy() if keep else None,
+        slot_mapping=w.slot_mapping[:nb].copy() if keep else None)
+
+
+def workload_config(w, args):
+    return {
+        "workload": f"{w.name}: {w.description}",
+        "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+        "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
+        "context_tokens": int(w.context_lens.sum()), "seed": args.seed,
+        "step": "pa_write_kv_cache(newest token of every sequence) + pa_decode",
+        "l2": "flushed before every timed step (zero-fill of 2x L2, outside the events)",
+        "parallelism": f"replicas: one independent batch per GPU x{args.gpus}",
+    }
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    w = wl.make_workload(args.workload, seed=args.seed)
+    nbytes_full = wl.roofline_bytes(w)
+    budget = max(2.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    per_step, sample, cores, desc = time_oracle(w, budget, max_reps=1)
+    for _ in range(args.warmup):
+        _oracle_step(sample)
+    times = [_oracle_step(sample) for _ in range(args.steps)]
+    t = statistics.mean(times)
+    gbs = wl.roofline_bytes(sample) / t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args),
+        "seq_tokens_per_s": sample.batch / t,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": f"fp64 CPU oracle; full-batch step bytes {nbytes_full}",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    from paged_kv_cache_334_b200 import pa
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, local)
+    pa.load()
+
+    w = wl.make_workload(args.workload, seed=rank_seed(args.seed, rank))
+    tdt = torch.float32 if w.dtype == wl.DTYPE_F32 else torch.bfloat16
+
+    def dev_t(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).to(dev)
+
+    q, kc, vc = dev_t(w.q), dev_t(w.key_cache), dev_t(w.value_cache)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    cl = torch.from_numpy(w.context_lens).to(dev)
+    has_new = w.slot_mapping is not None
+    kn = dev_t(w.k_new) if has_new else None
+    vn = dev_t(w.v_new) if has_new else None
+    sm = torch.from_numpy(w.slot_mapping).to(dev) if has_new else None
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = pa.decode_workspace(kc, w.batch, w.num_q_heads, w.max_blocks)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    stream = torch.cuda.current_stream(dev)
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    launches_per_step = 2 if has_new else 1
+
+    def write():
+        if has_new:
+            pa.pa_write_kv_cache(kc, vc, kn, vn, sm, err_word=err, stream=stream)
+
+    def decode():
+        pa.pa_decode(out, q, kc, vc, bt, cl, scale=scale, workspace=ws, err_word=err,
+                     stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush_buf.zero_()
+        write()
+        decode()
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())} during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark("t0")
+    for k in range(K):
+        flush_buf.zero_()
+        ev[k][0].record(stream)
+        write()
+        ev[k][1].record(stream)
+        decode()
+        ev[k][2].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark("t1")
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    t_step = statistics.mean(step_ms)
+    t_dec = statistics.mean(dec_ms)
+
+    # end to end: inputs of the step from pinned host memory, output back
+    e2e = None
+    if not args.no_e2e:
+        host = {"q": q.cpu().pin_memory(), "bt": bt.cpu().pin_memory(),
+                "cl": cl.cpu().pin_memory()}
+        if has_new:
+            host.update(kn=kn.cpu().pin_memory(), vn=vn.cpu().pin_memory(),
+                        sm=sm.cpu().pin_memory())
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+        pairs = [(q, host["q"]), (bt, host["bt"]), (cl, host["cl"])]
+        if has_new:
+            pairs += [(kn, host["kn"]), (vn, host["vn"]), (sm, host["sm"])]
+        Ke = max(3, min(K, 500))
+        eve = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+        for k in range(Ke + 3):
+            flush_buf.zero_()
+            if k >= 3:
+                eve[k - 3][0].record(stream)
+            for dst, src in pairs:
+                dst.copy_(src, non_blocking=True)
+            write()
+            decode()
+            out_host.copy_(out, non_blocking=True)
+            if k >= 3:
+                eve[k - 3][1].record(stream)
+        torch.cuda.synchronize(dev)
+        t_e2e = statistics.mean(e[0].elapsed_time(e[1]) for e in eve)
+        e2e = (t_e2e, h2d, d2h)
+
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+
+    step_bytes = wl.roofline_bytes(w)
+    dec_bytes = wl.roofline_bytes(w, include_write=False)
+    t_step_max = reduce_scalar(t_step, "max", dist, dev)
+    bytes_all = reduce_scalar(step_bytes, "sum", dist, dev)
+    seqs_all = reduce_scalar(w.batch, "sum", dist, dev)
+    ctx_all = reduce_scalar(float(w.context_lens.sum()), "sum", dist, dev)
+    e2e_line = None
+    if e2e is not None:
+        t_e2e_max = reduce_scalar(e2e[0], "max", dist, dev)
+        e2e_line = {"value": bytes_all / (t_e2e_max * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": int(e2e[1]), "d2h_bytes_per_step": int(e2e[2]),
+                    "ms_per_step": t_e2e_max}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_step, sample, cores, desc = time_oracle(w, args.cpu_seconds)
+        cpu = {"value": wl.roofline_bytes(sample) / per_step / 1e9, "unit": "GB/s",
+               "cores": cores, "kind": "oracle", "sample": desc,
+               "ms_per_step": per_step * 1e3}
+
+    peak, peak_src = hbm_peak()
+    achieved = dec_bytes / (t_dec * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": bytes_all / (t_step_max * 1e-3) / 1e9,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": t_step_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic",
+        "config": workload_config(w, args),
+        "seq_tokens_per_s": seqs_all / (t_step_max * 1e-3),
+        "context_tokens_per_s": ctx_all / (t_step_max * 1e-3),
+        "hbm_frac_step": (bytes_all / (t_step_max * 1e-3) / 1e9) / (peak * world),
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+            "kernel": "pa_decode", "algorithmic_bytes_per_launch": dec_bytes,
+            "launch_us": t_dec * 1e3, "peak_source": peak_src,
+        },
+        "e2e": e2e_line,
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,208 @@
+/*
+ * pa.h -- C ABI of libpa: single-query decode attention over a paged KV
+ * cache on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three public pages:
+ *   [route]    "From correct to faster: the PagedAttention optimisation
+ *              route" (yjxyzxyz.cn, article oHue8hrF);
+ *   [teaching] "Implementing teaching PagedAttention: reading the historical
+ *              KV cache from the block table" (yjxyzxyz.cn, article wVdUWYLj);
+ *   [serving]  "Operators and compilers: inference attention and KV kernels"
+ *              (charles2530.github.io, 2025-09-30).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer argument except `cache` is a DEVICE pointer on the current
+ *   CUDA device, owned by the caller; the library keeps no reference after
+ *   the call returns, allocates no memory and never synchronises.  Work is
+ *   enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *   and runs asynchronously: outputs are valid once the stream reaches the
+ *   call.
+ * - Arrays are dense, row-major, exactly as written:
+ *     key_cache, value_cache  [num_blocks, block_size, num_kv_heads, head_dim]
+ *     q, out                  [batch, num_q_heads, head_dim]
+ *     k_new, v_new            [num_tokens, num_kv_heads, head_dim]
+ *     block_tables            [batch, max_blocks_per_seq] int32
+ *     context_lens            [batch] int32
+ *     slot_mapping            [num_tokens] int64
+ *   Caches, q, out, k_new, v_new and partial outputs must be 16-byte
+ *   aligned.  Elements are fp32 or bf16 (cache->dtype); q, k_new, v_new and
+ *   out have the cache's dtype; partials are always fp32.
+ * - Query head hq reads KV head hq / (num_q_heads / num_kv_heads)
+ *   (contiguous GQA / MQA groups; [serving] section 7 "Why MQA / GQA change
+ *   serving performance").
+ * - Synchronous errors are returned: PA_ERR_INVALID_ARG for bad sizes,
+ *   null or misaligned pointers; PA_ERR_UNSUPPORTED for a shape with no
+ *   compiled kernel (head_dim not 64/128, block_size not a power of two
+ *   in [1, 256], more than 512 query heads per KV head); PA_ERR_CUDA when
+ *   a launch fails.  pa_last_error_message() gives the detail.
+ * - Errors that depend on device data are not returned: a block id outside
+ *   [0, num_blocks) among a sequence's visible pages, a context length
+ *   outside [0, max_blocks_per_seq * block_size], or a slot at or past
+ *   num_blocks * block_size set a PA_DEVERR_* bit in *err_word (an int32
+ *   in device memory, may be NULL) with an atomic OR; the affected
+ *   sequence's output is written as zeros (a bad slot is skipped).  The
+ *   caller reads the word after its own synchronisation.  No kernel traps.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *pa_stream_t; /* a cudaStream_t */
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,
+  PA_ERR_UNSUPPORTED = 2,
+  PA_ERR_CUDA = 3
+} pa_status;
+
+typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+
+/* Bits OR'd into *err_word by kernels that meet bad device data. */
+#define PA_DEVERR_BLOCK_ID 1
+#define PA_DEVERR_CONTEXT_LEN 2
+#define PA_DEVERR_SLOT 4
+
+/* Shape of the physical KV cache pool ([teaching] section "First define a
+ * simple KV cache layout": [num_blocks, block_size, num_heads, head_dim],
+ * with num_heads = the number of KV heads). */
+typedef struct pa_cache_desc {
+  int32_t num_blocks;
+  int32_t block_size;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t dtype; /* pa_dtype */
+} pa_cache_desc;
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+int32_t pa_version(void);
+
+/* Static text for a status code. */
+const char *pa_status_string(int32_t status);
+
+/* Detail of the last non-OK status returned on the calling host thread. */
+const char *pa_last_error_message(void);
+
+/*
+ * pa_write_kv_cache -- store the current tokens' K/V rows in their slots.
+ *
+ * [teaching] section "Writing slots and reading the block table must
+ * agree": the Block Manager reserves a slot (physical_block_id,
+ * block_offset) for the current token and its K/V are written there before
+ * attention reads it as history.  Slot encoding: slot_mapping[i] =
+ * physical_block_id * block_size + block_offset; a negative slot means
+ * "no token" and is skipped.  For each i with 0 <= slot < num_blocks *
+ * block_size, key_cache[slot / block_size, slot % block_size, :, :] =
+ * k_new[i] and the same for value_cache / v_new, as a byte copy.  A slot
+ * past the pool sets PA_DEVERR_SLOT and is skipped.  num_tokens == 0 is a
+ * no-op.  Two tokens with the same slot race (last writer undefined).
+ */
+pa_status pa_write_kv_cache(const pa_cache_desc *cache, void *key_cache,
+                            void *value_cache, const void *k_new,
+                            const void *v_new, const int64_t *slot_mapping,
+                            int32_t num_tokens, int32_t *err_word,
+                            pa_stream_t stream);
+
+/*
+ * pa_decode_workspace_bytes -- size of the scratch memory pa_decode needs
+ * for these sizes (0 on invalid arguments).
+ */
+size_t pa_decode_workspace_bytes(const pa_cache_desc *cache, int32_t batch,
+                                 int32_t num_q_heads,
+                                 int32_t max_blocks_per_seq);
+
+/*
+ * pa_decode -- fused paged decode attention.
+ *
+ * For every sequence b and query head hq, with h = hq / (Hq / Hkv):
+ * for t in [0, context_lens[b]): logical_block_id = t / block_size,
+ * block_offset = t % block_size, physical_block_id =
+ * block_tables[b, logical_block_id] ([teaching] section "From logical
+ * token to physical block"); s_t = scale * dot(q[b, hq], K_t[h]); out[b,
+ * hq] = sum_t softmax(s)_t * V_t[h] ([route] section "What the attention
+ * kernel really does").  One pass over the history with an online softmax
+ * (running max and normaliser), the block-table lookup done inside the
+ * kernel, no gathered K/V and no stored score vector ([route] sections
+ * "The core idea of high-performance PagedAttention" and "What the
+ * attention kernel really does").  The decode query attends to exactly the
+ * given history, so there is no mask argument ([teaching] section "Where
+ * is the attention mask").  context_lens[b] == 0 gives a zero output.
+ * Table entries past ceil(context_lens[b] / block_size) are never read.
+ *
+ * scale is usually 1 / sqrt(head_dim).  workspace: device memory of at
+ * least pa_decode_workspace_bytes(...) bytes, 256-byte aligned, ZERO-FILLED
+ * before its first use; every call leaves it zero-filled again on return,
+ * so one buffer serves any number of stream-ordered calls.  Calls that
+ * overlap on the GPU must not share a workspace.
+ */
+pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
+                    const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, const int32_t *context_lens,
+                    int32_t batch, int32_t num_q_heads,
+                    int32_t max_blocks_per_seq, float scale, void *workspace,
+                    size_t workspace_bytes, int32_t *err_word,
+                    pa_stream_t stream);
+
+/*
+ * pa_decode_splitk -- per-partition partial results for long contexts.
+ *
+ * Partition p of sequence b covers tokens [p * partition_tokens,
+ * min((p + 1) * partition_tokens, context_lens[b])).  For every
+ * non-empty partition and query head, with s_t as in pa_decode:
+ *   part_max[b, hq, p] = max_t s_t
+ *   part_sum[b, hq, p] = sum_t exp(s_t - part_max)
+ *   part_out[b, hq, p, :] = sum_t exp(s_t - part_max) V_t[h] / part_sum
+ * i.e. the running maximum and normaliser of the online softmax of [route]
+ * section "What the attention kernel really does", kept per partition.
+ * Partitions p in [ceil(context_lens[b] / partition_tokens),
+ * max_partitions) get part_max = -inf, part_sum = 0, part_out = 0.  A
+ * partition that meets a bad block id gets part_sum = -1 (and sets
+ * PA_DEVERR_BLOCK_ID); a sequence with a bad context length gets empty
+ * partials everywhere (and sets PA_DEVERR_CONTEXT_LEN).
+ * Shapes: part_max, part_sum [batch, num_q_heads, max_partitions];
+ * part_out [batch, num_q_heads, max_partitions, head_dim]; all fp32.
+ * partition_tokens must be a positive multiple of block_size;
+ * max_partitions must be >= ceil(max_blocks_per_seq * block_size /
+ * partition_tokens).
+ */
+pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
+                           const void *key_cache, const void *value_cache,
+                           const int32_t *block_tables,
+                           const int32_t *context_lens, int32_t batch,
+                           int32_t num_q_heads, int32_t max_blocks_per_seq,
+                           float scale, int32_t partition_tokens,
+                           int32_t max_partitions, float *part_max,
+                           float *part_sum, float *part_out, int32_t *err_word,
+                           pa_stream_t stream);
+
+/*
+ * pa_reduce -- merge per-partition partials into the output.
+ *
+ * For each (b, hq), over partitions p < min(ceil(context_lens[b] /
+ * partition_tokens), max_partitions) with part_sum > 0:
+ * M = max_p part_max, w_p = part_sum * exp(part_max - M),
+ * out[b, hq, :] = sum_p w_p part_out[p] / sum_p w_p -- the rescaling rule
+ * of the online softmax applied across partitions.  Zero output when no
+ * partition is non-empty or when any of them has part_sum < 0 (a bad
+ * block id upstream).  A context length < 0 or past max_partitions *
+ * partition_tokens sets PA_DEVERR_CONTEXT_LEN and gives zeros.  out has
+ * dtype `out_dtype`.
+ */
+pa_status pa_reduce(void *out, const float *part_max, const float *part_sum,
+                    const float *part_out, const int32_t *context_lens,
+                    int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                    int32_t partition_tokens, int32_t max_partitions,
+                    int32_t out_dtype, int32_t *err_word, pa_stream_t stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* PA_H_ */

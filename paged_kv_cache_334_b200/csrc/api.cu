@@ -1,0 +1,305 @@
+// api.cu -- the extern "C" entry points of libpa (declared in include/pa.h).
+//
+// This layer validates arguments on the host, lays out the decode workspace
+// and enqueues kernels on the caller's stream.  It never allocates, never
+// synchronises and has no CPU fallback: every step of the computation runs in
+// the kernels of write_kv.cu, decode.cu and reduce.cu.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/pa.h"
+#include "pa_launch.h"
+
+namespace {
+
+constexpr int32_t kDecodePartitionTokens = 256;
+constexpr int32_t kMaxPartitionPages = 1024;  // block-table slice held in smem
+constexpr size_t kAlign = 256;
+
+thread_local char g_msg[512] = "";
+
+pa_status fail(pa_status s, const char *fmt, const char *detail = nullptr,
+               long long v = 0) {
+  snprintf(g_msg, sizeof g_msg, fmt, detail ? detail : "", v);
+  return s;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool is_pow2(int32_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int32_t elem_bytes(int32_t dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
+
+pa_status check_cache(const pa_cache_desc *c) {
+  if (c == nullptr) return fail(PA_ERR_INVALID_ARG, "cache descriptor is NULL%s");
+  if (c->dtype != PA_DTYPE_F32 && c->dtype != PA_DTYPE_BF16)
+    return fail(PA_ERR_INVALID_ARG, "dtype %s%lld is neither F32 nor BF16", "", c->dtype);
+  if (c->num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "num_blocks must be > 0%s (got %lld)", "", c->num_blocks);
+  if (c->num_kv_heads <= 0)
+    return fail(PA_ERR_INVALID_ARG, "num_kv_heads must be > 0%s (got %lld)", "", c->num_kv_heads);
+  if (!is_pow2(c->block_size) || c->block_size > 256)
+    return fail(PA_ERR_UNSUPPORTED, "block_size must be a power of two in [1, 256]%s (got %lld)",
+                "", c->block_size);
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim must be 64 or 128%s (got %lld)", "", c->head_dim);
+  return PA_OK;
+}
+
+pa_status check_ptr(const void *p, const char *name) {
+  if (p == nullptr) return fail(PA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(PA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return PA_OK;
+}
+
+// Checks shared by pa_decode and pa_decode_splitk.
+pa_status check_decode_common(const pa_cache_desc *cache, const void *q,
+                              const void *key_cache, const void *value_cache,
+                              const int32_t *block_tables,
+                              const int32_t *context_lens, int32_t batch,
+                              int32_t num_q_heads, int32_t max_blocks,
+                              float scale) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (batch < 0 || batch > 65535)
+    return fail(PA_ERR_INVALID_ARG, "batch must be in [0, 65535]%s (got %lld)", "", batch);
+  if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "num_q_heads must be a positive multiple of num_kv_heads%s (got %lld)", "",
+                num_q_heads);
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  if (group > 512)
+    return fail(PA_ERR_UNSUPPORTED, "more than 512 query heads per KV head%s (%lld)", "", group);
+  const int32_t gt = pa::decode_head_tile(group);
+  if ((int64_t)cache->num_kv_heads * ((group + gt - 1) / gt) > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "too many KV heads x head tiles%s (%lld)", "",
+                (long long)cache->num_kv_heads * ((group + gt - 1) / gt));
+  if (max_blocks < 0 || (int64_t)max_blocks * cache->block_size > 0x7fffffffLL)
+    return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq * block_size must fit int32%s (%lld)", "",
+                max_blocks);
+  if (!isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite%s");
+  if (batch == 0) return PA_OK;
+  if ((s = check_ptr(q, "q")) != PA_OK) return s;
+  if ((s = check_ptr(key_cache, "key_cache")) != PA_OK) return s;
+  if ((s = check_ptr(value_cache, "value_cache")) != PA_OK) return s;
+  if (context_lens == nullptr) return fail(PA_ERR_INVALID_ARG, "context_lens is NULL%s");
+  if (max_blocks > 0 && block_tables == nullptr)
+    return fail(PA_ERR_INVALID_ARG, "block_tables is NULL%s");
+  return PA_OK;
+}
+
+struct WorkspaceLayout {
+  size_t part_max, part_sum, part_out, counters, total;
+  int32_t max_parts;
+};
+
+WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
+                              int32_t num_q_heads, int32_t max_blocks) {
+  WorkspaceLayout w{};
+  const int64_t tokens = (int64_t)max_blocks * c->block_size;
+  w.max_parts = (int32_t)((tokens + kDecodePartitionTokens - 1) / kDecodePartitionTokens);
+  const size_t n = (size_t)batch * num_q_heads * w.max_parts;
+  const int32_t group = num_q_heads / c->num_kv_heads;
+  const int32_t gt = pa::decode_head_tile(group);
+  const size_t ncnt = (size_t)batch * c->num_kv_heads * ((group + gt - 1) / gt);
+  w.part_max = 0;
+  w.part_sum = round_up(w.part_max + n * sizeof(float));
+  w.part_out = round_up(w.part_sum + n * sizeof(float));
+  w.counters = round_up(w.part_out + n * c->head_dim * sizeof(float));
+  w.total = round_up(w.counters + ncnt * sizeof(int32_t));
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_version(void) { return 100; }
+
+const char *pa_status_string(int32_t status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    default: return "PA_UNKNOWN_STATUS";
+  }
+}
+
+const char *pa_last_error_message(void) { return g_msg; }
+
+pa_status pa_write_kv_cache(const pa_cache_desc *cache, void *key_cache,
+                            void *value_cache, const void *k_new,
+                            const void *v_new, const int64_t *slot_mapping,
+                            int32_t num_tokens, int32_t *err_word,
+                            pa_stream_t stream) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (num_tokens < 0)
+    return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0%s (got %lld)", "", num_tokens);
+  if (num_tokens == 0) return PA_OK;
+  if ((s = check_ptr(key_cache, "key_cache")) != PA_OK) return s;
+  if ((s = check_ptr(value_cache, "value_cache")) != PA_OK) return s;
+  if ((s = check_ptr(k_new, "k_new")) != PA_OK) return s;
+  if ((s = check_ptr(v_new, "v_new")) != PA_OK) return s;
+  if (slot_mapping == nullptr) return fail(PA_ERR_INVALID_ARG, "slot_mapping is NULL%s");
+  const int64_t row_bytes =
+      (int64_t)cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype);
+  cudaError_t e = pa::launch_write_kv(cache->dtype, cache->block_size,
+                                      cache->num_blocks, row_bytes, key_cache,
+                                      value_cache, k_new, v_new, slot_mapping,
+                                      num_tokens, err_word,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "write_kv launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+size_t pa_decode_workspace_bytes(const pa_cache_desc *cache, int32_t batch,
+                                 int32_t num_q_heads, int32_t max_blocks_per_seq) {
+  if (check_cache(cache) != PA_OK || batch < 0 || num_q_heads <= 0 ||
+      num_q_heads % cache->num_kv_heads != 0 || max_blocks_per_seq < 0)
+    return 0;
+  return decode_layout(cache, batch, num_q_heads, max_blocks_per_seq).total;
+}
+
+pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
+                    const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, const int32_t *context_lens,
+                    int32_t batch, int32_t num_q_heads,
+                    int32_t max_blocks_per_seq, float scale, void *workspace,
+                    size_t workspace_bytes, int32_t *err_word,
+                    pa_stream_t stream) {
+  pa_status s = check_decode_common(cache, q, key_cache, value_cache, block_tables,
+                                    context_lens, batch, num_q_heads,
+                                    max_blocks_per_seq, scale);
+  if (s != PA_OK) return s;
+  if (batch == 0) return PA_OK;
+  if ((s = check_ptr(out, "out")) != PA_OK) return s;
+  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+  if (workspace_bytes < w.total)
+    return fail(PA_ERR_INVALID_ARG, "workspace too small%s: need %lld bytes", "",
+                (long long)w.total);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
+  char *ws = static_cast<char *>(workspace);
+  pa::DecodeArgs a{};
+  a.q = q;
+  a.out = out;
+  a.key_cache = key_cache;
+  a.value_cache = value_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.part_max = reinterpret_cast<float *>(ws + w.part_max);
+  a.part_sum = reinterpret_cast<float *>(ws + w.part_sum);
+  a.part_out = reinterpret_cast<float *>(ws + w.part_out);
+  a.counters = reinterpret_cast<int32_t *>(ws + w.counters);
+  a.err_word = err_word;
+  a.dtype = cache->dtype;
+  a.num_blocks = cache->num_blocks;
+  a.block_size = cache->block_size;
+  a.num_kv_heads = cache->num_kv_heads;
+  a.head_dim = cache->head_dim;
+  a.batch = batch;
+  a.num_q_heads = num_q_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.part_tokens = kDecodePartitionTokens;
+  a.max_parts = w.max_parts;
+  a.scale = scale;
+  a.merge = true;
+  cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
+                           const void *key_cache, const void *value_cache,
+                           const int32_t *block_tables,
+                           const int32_t *context_lens, int32_t batch,
+                           int32_t num_q_heads, int32_t max_blocks_per_seq,
+                           float scale, int32_t partition_tokens,
+                           int32_t max_partitions, float *part_max,
+                           float *part_sum, float *part_out, int32_t *err_word,
+                           pa_stream_t stream) {
+  pa_status s = check_decode_common(cache, q, key_cache, value_cache, block_tables,
+                                    context_lens, batch, num_q_heads,
+                                    max_blocks_per_seq, scale);
+  if (s != PA_OK) return s;
+  if (partition_tokens <= 0 || partition_tokens % cache->block_size != 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "partition_tokens must be a positive multiple of block_size%s (got %lld)", "",
+                partition_tokens);
+  if (partition_tokens / cache->block_size > kMaxPartitionPages)
+    return fail(PA_ERR_UNSUPPORTED, "more than 1024 blocks per partition%s (%lld)", "",
+                partition_tokens / cache->block_size);
+  const int64_t need =
+      ((int64_t)max_blocks_per_seq * cache->block_size + partition_tokens - 1) / partition_tokens;
+  if (max_partitions < need || max_partitions <= 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "max_partitions must be >= ceil(max_blocks_per_seq*block_size/partition_tokens)%s"
+                " = %lld",
+                "", need);
+  if (batch == 0) return PA_OK;
+  if ((s = check_ptr(part_max, "part_max")) != PA_OK) return s;
+  if ((s = check_ptr(part_sum, "part_sum")) != PA_OK) return s;
+  if ((s = check_ptr(part_out, "part_out")) != PA_OK) return s;
+  pa::DecodeArgs a{};
+  a.q = q;
+  a.out = nullptr;
+  a.key_cache = key_cache;
+  a.value_cache = value_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.part_max = part_max;
+  a.part_sum = part_sum;
+  a.part_out = part_out;
+  a.counters = nullptr;
+  a.err_word = err_word;
+  a.dtype = cache->dtype;
+  a.num_blocks = cache->num_blocks;
+  a.block_size = cache->block_size;
+  a.num_kv_heads = cache->num_kv_heads;
+  a.head_dim = cache->head_dim;
+  a.batch = batch;
+  a.num_q_heads = num_q_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.part_tokens = partition_tokens;
+  a.max_parts = max_partitions;
+  a.scale = scale;
+  a.merge = false;
+  cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return fail(PA_ERR_CUDA, "decode_splitk launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+pa_status pa_reduce(void *out, const float *part_max, const float *part_sum,
+                    const float *part_out, const int32_t *context_lens,
+                    int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                    int32_t partition_tokens, int32_t max_partitions,
+                    int32_t out_dtype, int32_t *err_word, pa_stream_t stream) {
+  if (out_dtype != PA_DTYPE_F32 && out_dtype != PA_DTYPE_BF16)
+    return fail(PA_ERR_INVALID_ARG, "out_dtype %s%lld is neither F32 nor BF16", "", out_dtype);
+  if (batch < 0 || num_q_heads <= 0 || head_dim <= 0 || partition_tokens <= 0 ||
+      max_partitions <= 0)
+    return fail(PA_ERR_INVALID_ARG, "sizes must be positive%s");
+  if ((int64_t)batch * num_q_heads > 0x7fffffffLL)
+    return fail(PA_ERR_UNSUPPORTED, "batch * num_q_heads too large%s");
+  if (head_dim % 4 != 0) return fail(PA_ERR_INVALID_ARG, "head_dim must be a multiple of 4%s");
+  if (batch == 0) return PA_OK;
+  pa_status s;
+  if ((s = check_ptr(out, "out")) != PA_OK) return s;
+  if ((s = check_ptr(part_max, "part_max")) != PA_OK) return s;
+  if ((s = check_ptr(part_sum, "part_sum")) != PA_OK) return s;
+  if ((s = check_ptr(part_out, "part_out")) != PA_OK) return s;
+  if (context_lens == nullptr) return fail(PA_ERR_INVALID_ARG, "context_lens is NULL%s");
+  cudaError_t e = pa::launch_reduce(out, part_max, part_sum, part_out, context_lens, batch,
+                                    num_q_heads, head_dim, partition_tokens, max_partitions,
+                                    out_dtype, err_word, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reduce launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,118 @@
+// pa_common.cuh -- device helpers shared by the libpa kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---------------------------------------------------------------------------
+// Element types.  Cache rows are moved as 16-byte vectors; each vector holds
+// kPerVec elements and is widened to fp32 in registers.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+  static constexpr int kBytes = 4;
+  static constexpr int kPerVec = 4;
+  __device__ __forceinline__ static void widen(const uint4 &v, float (&f)[4]) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+  __device__ __forceinline__ static float load1(const void *p, int64_t i) {
+    return static_cast<const float *>(p)[i];
+  }
+  __device__ __forceinline__ static void store1(void *p, int64_t i, float x) {
+    static_cast<float *>(p)[i] = x;
+  }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static constexpr int kPerVec = 8;
+  // bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 bits.
+  __device__ __forceinline__ static void widen(const uint4 &v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ __forceinline__ static float load1(const void *p, int64_t i) {
+    return __uint_as_float(
+        static_cast<uint32_t>(static_cast<const uint16_t *>(p)[i]) << 16);
+  }
+  __device__ __forceinline__ static void store1(void *p, int64_t i, float x) {
+    static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+  }
+};
+
+// Streaming 16-byte read of data that no kernel writes while it runs.
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void set_error(int32_t *err_word, int32_t bit) {
+  if (err_word != nullptr) atomicOr(err_word, bit);
+}
+
+// ---------------------------------------------------------------------------
+// Transposed butterfly reduction across the L lanes of an aligned lane group.
+//
+// Every lane holds N partial sums v[0..N).  After the call, with j the lane's
+// index inside its group:
+//   N >= L : v[0 .. N/L) hold the group-wide sums of indices
+//            j*(N/L) .. j*(N/L) + N/L - 1;
+//   N <  L : v[0] holds the group-wide sum of index j >> log2(L/N) (lanes
+//            that differ only in their low log2(L/N) bits hold the same sum).
+// Each stage halves the number of live values, so the whole reduction costs
+// N - 1 shuffles per lane when N >= L instead of N * log2(L).
+// ---------------------------------------------------------------------------
+template <int N, int MASK>
+struct Butterfly {
+  __device__ __forceinline__ static void run(float *v, int lane) {
+    if constexpr (MASK > 0) {
+      if constexpr (N >= 2) {
+        constexpr int H = N / 2;
+        const bool upper = (lane & MASK) != 0;
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+          const float send = upper ? v[i] : v[i + H];
+          const float keep = upper ? v[i + H] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, MASK);
+        }
+        Butterfly<H, MASK / 2>::run(v, lane);
+      } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], MASK);
+        Butterfly<1, MASK / 2>::run(v, lane);
+      }
+    }
+  }
+};
+
+template <int X>
+struct Log2 {
+  static constexpr int value = 1 + Log2<X / 2>::value;
+};
+template <>
+struct Log2<1> {
+  static constexpr int value = 0;
+};
+
+}  // namespace pa

@@ -1,0 +1,61 @@
+// write_kv.cu -- cache write by slot mapping.
+//
+// Page "Implementing teaching PagedAttention: reading the historical KV cache
+// from the block table", section "Writing slots and reading the block table
+// must agree": the current token's K/V rows go to the slot the Block Manager
+// reserved for it, (physical_block_id, block_offset), encoded here as
+// slot = physical_block_id * block_size + block_offset.
+//
+// One CTA per (new token, row slice); each thread moves 16-byte vectors, so a
+// row (num_kv_heads * head_dim elements) is copied with coalesced loads and
+// stores.  Bit-exact: the bytes are moved, never converted.
+#include "pa_common.cuh"
+#include "pa_launch.h"
+
+namespace pa {
+namespace {
+
+__global__ void __launch_bounds__(128)
+write_kv_kernel(uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache,
+                const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                const int64_t *__restrict__ slot_mapping, int64_t num_slots,
+                int64_t row_vecs, int32_t *err_word) {
+  const int64_t token = blockIdx.x;
+  const int64_t slot = slot_mapping[token];
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (blockIdx.y == 0 && threadIdx.x == 0) set_error(err_word, PA_DEVERR_SLOT);
+    return;
+  }
+  const int64_t src = token * row_vecs;
+  const int64_t dst = slot * row_vecs;
+  for (int64_t i = blockIdx.y * (int64_t)blockDim.x + threadIdx.x; i < row_vecs;
+       i += (int64_t)gridDim.y * blockDim.x) {
+    key_cache[dst + i] = k_new[src + i];
+    value_cache[dst + i] = v_new[src + i];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_write_kv(int32_t dtype, int32_t block_size,
+                            int32_t num_blocks, int64_t row_bytes,
+                            void *key_cache, void *value_cache,
+                            const void *k_new, const void *v_new,
+                            const int64_t *slot_mapping, int32_t num_tokens,
+                            int32_t *err_word, cudaStream_t stream) {
+  (void)dtype;
+  if (num_tokens == 0) return cudaSuccess;
+  const int64_t row_vecs = row_bytes / 16;
+  const int threads = 128;
+  int64_t gy = (row_vecs + threads - 1) / threads;
+  if (gy > 64) gy = 64;
+  dim3 grid((unsigned)num_tokens, (unsigned)gy);
+  write_kv_kernel<<<grid, threads, 0, stream>>>(
+      static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache),
+      static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
+      slot_mapping, (int64_t)num_blocks * block_size, row_vecs, err_word);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

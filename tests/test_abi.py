@@ -1,0 +1,129 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every
+symbol include/pa.h declares, and its host-side argument checks return the
+documented statuses before any device work (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_334_b200 import pa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        names |= set(re.findall(r"\b(pa_\w+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_334_b200 import build
+    build.build()
+    return pa.load()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("pa_write_kv_cache", "pa_decode", "pa_decode_splitk", "pa_reduce"):
+        assert required in names
+    assert set(pa.EXPORTED_SYMBOLS) <= set(names)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_version_and_status_strings(lib):
+    assert pa.pa_version() >= 100
+    assert lib.pa_status_string(0) == b"PA_OK"
+    assert lib.pa_status_string(1) == b"PA_ERR_INVALID_ARG"
+    assert lib.pa_status_string(2) == b"PA_ERR_UNSUPPORTED"
+    assert lib.pa_status_string(3) == b"PA_ERR_CUDA"
+
+
+def _desc(nb=16, bs=16, hkv=8, d=128, dtype=1):
+    return pa.CacheDesc(nb, bs, hkv, d, dtype)
+
+
+FAKE = ctypes.c_void_p(0x10000)       # aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def _decode(lib, desc, *, out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, B=2, Hq=32,
+            MB=4, scale=0.1, ws=FAKE, wsb=1 << 30):
+    return lib.pa_decode(ctypes.byref(desc) if desc is not None else None, out, q, kc, vc, bt,
+                         cl, B, Hq, MB, scale, ws, wsb, None, None)
+
+
+def test_decode_argument_checks(lib):
+    assert _decode(lib, None) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(d=96)) == pa.PA_ERR_UNSUPPORTED
+    assert _decode(lib, _desc(bs=12)) == pa.PA_ERR_UNSUPPORTED
+    assert _decode(lib, _desc(bs=512)) == pa.PA_ERR_UNSUPPORTED
+    assert _decode(lib, _desc(dtype=7)) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(), Hq=30) == pa.PA_ERR_INVALID_ARG       # not a multiple of Hkv
+    assert _decode(lib, _desc(), B=-1) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(), q=MISALIGNED) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(), kc=None) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(), cl=None) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(), scale=float("inf")) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(), wsb=16) == pa.PA_ERR_INVALID_ARG       # workspace too small
+    assert _decode(lib, _desc(), ws=ctypes.c_void_p(0x10010)) == pa.PA_ERR_INVALID_ARG
+    assert _decode(lib, _desc(hkv=1), Hq=1024) == pa.PA_ERR_UNSUPPORTED  # group > 512
+    assert b"head_dim" in _msg(lib, _decode(lib, _desc(d=96)))
+    # an empty batch is a valid no-op (no device work)
+    assert _decode(lib, _desc(), B=0) == pa.PA_OK
+
+
+def _msg(lib, _status):
+    return lib.pa_last_error_message()
+
+
+def test_splitk_and_reduce_argument_checks(lib):
+    d = _desc()
+    f = lib.pa_decode_splitk
+    # partition not a multiple of the block size
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4, 0.1, 24, 8, FAKE, FAKE,
+             FAKE, None, None) == pa.PA_ERR_INVALID_ARG
+    # too few partitions for max_blocks * block_size tokens
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 64, 0.1, 256, 3, FAKE, FAKE,
+             FAKE, None, None) == pa.PA_ERR_INVALID_ARG
+    # more than 1024 blocks in one partition
+    assert f(ctypes.byref(_desc(bs=1)), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4096, 0.1, 2048, 2,
+             FAKE, FAKE, FAKE, None, None) == pa.PA_ERR_UNSUPPORTED
+    r = lib.pa_reduce
+    assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 128, 512, 4, 9, None, None) == pa.PA_ERR_INVALID_ARG
+    assert r(MISALIGNED, FAKE, FAKE, FAKE, FAKE, 2, 32, 128, 512, 4, 1, None, None) == \
+        pa.PA_ERR_INVALID_ARG
+    assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 32, 128, 512, 4, 1, None, None) == pa.PA_OK
+
+
+def test_write_argument_checks(lib):
+    d = _desc()
+    w = lib.pa_write_kv_cache
+    assert w(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, -1, None, None) == pa.PA_ERR_INVALID_ARG
+    assert w(ctypes.byref(d), FAKE, FAKE, MISALIGNED, FAKE, FAKE, 3, None, None) == \
+        pa.PA_ERR_INVALID_ARG
+    assert w(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, None, 3, None, None) == pa.PA_ERR_INVALID_ARG
+    assert w(ctypes.byref(d), None, None, None, None, None, 0, None, None) == pa.PA_OK
+
+
+def test_workspace_size(lib):
+    d = _desc(nb=100, bs=16, hkv=8, d=128)
+    n = lib.pa_decode_workspace_bytes(ctypes.byref(d), 32, 32, 128)
+    assert n > 0 and n % 256 == 0
+    # partial max, sum and output per (sequence, query head, 256-token partition)
+    parts = (128 * 16 + 255) // 256
+    assert n >= 32 * 32 * parts * (2 + 128) * 4
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(d), 32, 30, 128) == 0
+    assert lib.pa_decode_workspace_bytes(None, 32, 32, 128) == 0
