@@ -50,6 +50,7 @@ from paged_kv_cache_334_b200 import workloads as wl  # noqa: E402
 METRIC = "decode-attention KV GB/s & fraction of B200 HBM peak; seq-tokens/s per step"
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCE = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc", "decode.cu")
+DECODE_HELPERS = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc", "pa_common.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.md")
 
 
@@ -193,11 +194,11 @@ def hbm_peak():
 
 
 def decode_source_hash() -> str:
+    """Hash of the decode kernel's own sources (kernel file + device helpers)."""
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(os.path.dirname(DECODE_SOURCE))):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(os.path.dirname(DECODE_SOURCE), fn), "rb") as f:
-                h.update(fn.encode() + f.read())
+    for path in (DECODE_SOURCE, DECODE_HELPERS):
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + f.read())
     return h.hexdigest()[:16]
 
 
