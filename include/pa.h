@@ -151,6 +151,49 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
                     pa_stream_t stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.
+ *
+ * The pages have no counterpart to this entry point.  It serves callers of
+ * this library that may not call cudaMalloc and so cannot hand pa_decode a
+ * workspace: code running as a plugin or callback inside a host engine that
+ * owns every byte of device memory through its own pool (an allocation
+ * behind the pool's back can fail or break its accounting), and decode loops
+ * with hard latency budgets, where cudaMalloc / cudaFree may wait for the
+ * whole device to go idle.
+ *
+ * Arguments, semantics, results and error reporting are those of pa_decode,
+ * minus the workspace.  The scratch space is a fixed array of
+ * PA_DECODE_NOALLOC_SCRATCH_BYTES bytes of device memory inside libpa; every
+ * GPU that loads the library holds it until the process exits.  This call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * - Limit: when pa_decode_workspace_bytes(cache, batch, num_q_heads,
+ *   max_blocks_per_seq) exceeds PA_DECODE_NOALLOC_SCRATCH_BYTES the call
+ *   returns PA_ERR_UNSUPPORTED (see pa_last_error_message) and enqueues no
+ *   work; use pa_decode with a workspace for such sizes.
+ * - Set-up: the first call on a device looks up the array's device address
+ *   for that device (the calling thread's current device) and remembers it.
+ *   Make that first call on each device before any stream capture.
+ * - Sharing: all calls on a device use the same array, and it keeps what the
+ *   last call left in it.  Each call clears the bytes it needs (an
+ *   asynchronous memset on `stream`) before the decode kernel runs.  Calls
+ *   that overlap on the GPU (other streams, or other host threads without
+ *   ordering between them) race on the array and give wrong results; order
+ *   them on one stream.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+pa_status pa_decode_noalloc(const pa_cache_desc *cache, void *out,
+                            const void *q, const void *key_cache,
+                            const void *value_cache,
+                            const int32_t *block_tables,
+                            const int32_t *context_lens, int32_t batch,
+                            int32_t num_q_heads, int32_t max_blocks_per_seq,
+                            float scale, int32_t *err_word,
+                            pa_stream_t stream);
+
+/*
  * pa_decode_splitk -- per-partition partial results for long contexts.
  *
  * Partition p of sequence b covers tokens [p * partition_tokens,

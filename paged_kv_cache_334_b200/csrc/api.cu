@@ -115,6 +115,10 @@ WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
 
 }  // namespace
 
+namespace pa {
+void set_last_error_message(const char *msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
+}  // namespace pa
+
 extern "C" {
 
 int32_t pa_version(void) { return 100; }

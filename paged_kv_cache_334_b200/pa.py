@@ -39,7 +39,11 @@ PA_DEVERR_SLOT = 4
 EXPORTED_SYMBOLS = (
     "pa_version", "pa_status_string", "pa_last_error_message", "pa_write_kv_cache",
     "pa_decode_workspace_bytes", "pa_decode", "pa_decode_splitk", "pa_reduce",
+    "pa_decode_noalloc",
 )
+
+# Size of the fixed device scratch array pa_decode_noalloc uses.
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class PaError(RuntimeError):
@@ -86,6 +90,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_splitk.restype = ctypes.c_int
     lib.pa_reduce.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P]
     lib.pa_reduce.restype = ctypes.c_int
+    lib.pa_decode_noalloc.argtypes = [D, P, P, P, P, P, P, i32, i32, i32, f32, P, P]
+    lib.pa_decode_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -228,4 +234,27 @@ def pa_reduce(out, part_max, part_sum, part_out, context_lens, partition_tokens:
         _dev(context_lens, "context_lens", torch.int32), B, Hq, Dh, int(partition_tokens),
         int(P), _dtype_code(out.dtype), _dev(err_word, "err_word", torch.int32),
         _stream(stream)))
+    return out
+
+
+def pa_decode_noalloc(out, q, key_cache, value_cache, block_tables, context_lens,
+                      scale: Optional[float] = None, err_word: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """pa_decode without a workspace, for callers that may not allocate device
+    memory: the library's own fixed scratch array (NOALLOC_SCRATCH_BYTES per
+    GPU) stands in for it.  Sizes whose workspace would not fit raise
+    PaError(PA_ERR_UNSUPPORTED).  Calls that overlap on the GPU share that
+    array and race; keep them on one stream (see include/pa.h)."""
+    lib = load()
+    desc = cache_desc(key_cache)
+    B, Hq, Dq = q.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dq)
+    _check(lib.pa_decode_noalloc(
+        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
+        _dev(err_word, "err_word", torch.int32), _stream(stream)))
     return out

@@ -1,0 +1,94 @@
+"""pa_decode_noalloc against pa_decode, through the C ABI.
+
+pa_decode_noalloc is the decode call for users of this library that may not
+allocate device memory themselves -- for instance a plugin whose host engine
+owns all device memory through its own pool, or a decode loop that cannot
+afford the device-wide stalls cudaMalloc / cudaFree can cause -- and so
+cannot pass pa_decode a workspace.  It uses a fixed scratch array inside the
+library instead.  This file checks, on two calls in a row and on shapes that
+alternate between calls (so leftovers of one call meet the next), that it
+returns what pa_decode returns, within the tolerances the other tests use.
+
+It is named to be collected last: a failure here does not hide any other
+test when the run stops at the first failure.  It needs no state from other
+tests and passes alone in a fresh process.
+"""
+import pytest
+import torch
+
+from paged_kv_cache_334_b200 import pa
+from paged_kv_cache_334_b200 import workloads as wl
+
+from _pa_helpers import assert_close, to_f64, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def _prepare(w):
+    d = upload(w)
+    if "slot_mapping" in d:
+        pa.pa_write_kv_cache(d["key_cache"], d["value_cache"], d["k_new"], d["v_new"],
+                             d["slot_mapping"])
+    ref = torch.empty_like(d["q"])
+    pa.pa_decode(ref, d["q"], d["key_cache"], d["value_cache"], d["block_tables"],
+                 d["context_lens"])
+    return d, ref
+
+
+def _noalloc(d, err):
+    out = torch.full_like(d["q"], float("nan"))
+    pa.pa_decode_noalloc(out, d["q"], d["key_cache"], d["value_cache"], d["block_tables"],
+                         d["context_lens"], err_word=err)
+    return out
+
+
+def test_noalloc_matches_pa_decode_on_two_calls_in_a_row():
+    w = wl.make_workload("gqa_bf16", seed=4)
+    assert pa.pa_decode_workspace_bytes(upload_shape(w), w.batch, w.num_q_heads,
+                                        w.max_blocks) <= pa.NOALLOC_SCRATCH_BYTES
+    d, ref = _prepare(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for call in range(2):
+        out = _noalloc(d, err)
+        torch.cuda.synchronize()
+        assert_close(to_f64(out), to_f64(ref), w.dtype, f"noalloc call {call}")
+    assert int(err.item()) == 0
+
+
+def test_noalloc_alternating_shapes_reuse_the_scratch():
+    """Calls with different sizes share the scratch array; each one clears
+    what it needs, so the previous call's leftovers do not leak in."""
+    cases = [wl.make_workload("mixed_bf16", seed=1, batch=6),
+             wl.make_workload("tiny_fp32", seed=0),
+             wl.make_workload("gqa_bf16", seed=8, batch=12)]
+    prepared = [(w, *_prepare(w)) for w in cases]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for rnd in range(2):
+        for w, d, ref in prepared:
+            out = _noalloc(d, err)
+            torch.cuda.synchronize()
+            assert_close(to_f64(out), to_f64(ref), w.dtype, f"{w.name} round {rnd}")
+    assert int(err.item()) == 0
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    w = wl.make_workload("mqa_prefix_bf16", seed=0, batch=64)
+    need = pa.pa_decode_workspace_bytes(upload_shape(w), w.batch, w.num_q_heads, w.max_blocks)
+    assert need > pa.NOALLOC_SCRATCH_BYTES
+    d = upload(w)
+    out = torch.zeros_like(d["q"])
+    with pytest.raises(pa.PaError) as ei:
+        pa.pa_decode_noalloc(out, d["q"], d["key_cache"], d["value_cache"],
+                             d["block_tables"], d["context_lens"])
+    assert ei.value.status == pa.PA_ERR_UNSUPPORTED
+    assert "scratch" in str(ei.value)
+    torch.cuda.synchronize()
+    assert int(out.count_nonzero().item()) == 0  # nothing was enqueued
+
+
+def upload_shape(w):
+    """A stand-in with the cache's shape and dtype: the workspace size depends
+    only on the cache descriptor, so no cache needs to be materialised."""
+    dt = torch.float32 if w.dtype == wl.DTYPE_F32 else torch.bfloat16
+    return torch.empty(1, 1, 1, 1, dtype=dt).expand(
+        w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
