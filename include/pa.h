@@ -69,6 +69,9 @@ typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_BLOCK_ID 1
 #define PA_DEVERR_CONTEXT_LEN 2
 #define PA_DEVERR_SLOT 4
+/* A pipeline wait inside a kernel gave up (never expected; the outputs of
+ * that call are incomplete and its workspace must be zero-filled again). */
+#define PA_DEVERR_TIMEOUT 8
 
 /* Shape of the physical KV cache pool ([teaching] section "First define a
  * simple KV cache layout": [num_blocks, block_size, num_heads, head_dim],

@@ -91,14 +91,83 @@ pa_status check_decode_common(const pa_cache_desc *cache, const void *q,
   return PA_OK;
 }
 
+// Shape plan of the persistent decode kernel; ok == false means the shape is
+// served by the partition kernel of decode.cu instead.
+struct StreamPlan {
+  bool ok;
+  int32_t vbs, log2_vbs, log2_vpp, row_bytes, vpage_bytes, q_bytes, pps, stages, stage_bytes;
+  size_t smem;
+};
+
+int32_t ilog2(int32_t x) {
+  int32_t l = 0;
+  while ((1 << l) < x) ++l;
+  return l;
+}
+
+StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads) {
+  namespace st = pa::stream;
+  StreamPlan s{};
+  s.ok = false;
+  const int32_t hkv = c->num_kv_heads;
+  const int32_t group = num_q_heads / hkv;
+  if (hkv != 4 && hkv != 8) return s;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return s;
+  const int32_t elt = elem_bytes(c->dtype);
+  s.row_bytes = hkv * c->head_dim * elt;
+  if (s.row_bytes > st::kVPageBytes) return s;
+  const int32_t rows = st::kVPageBytes / s.row_bytes;
+  s.vbs = c->block_size < rows ? c->block_size : rows;
+  s.log2_vbs = ilog2(s.vbs);
+  s.log2_vpp = ilog2(c->block_size / s.vbs);
+  s.vpage_bytes = s.vbs * s.row_bytes;
+  s.pps = st::kVPageBytes / s.vpage_bytes;
+  if (s.pps > st::kMaxPPS) s.pps = st::kMaxPPS;
+  if (s.pps < 1) s.pps = 1;
+  s.q_bytes = num_q_heads * c->head_dim * elt;
+  s.stage_bytes = (int32_t)(((size_t)2 * s.pps * s.vpage_bytes + (size_t)s.pps * s.q_bytes + 127) /
+                            128 * 128);
+  s.stages = (st::kSmemLimit - st::kHdrBytes) / s.stage_bytes;
+  if (s.stages > st::kMaxStages) s.stages = st::kMaxStages;
+  if (s.stages < 2) return s;
+  s.smem = (size_t)st::kHdrBytes + (size_t)s.stages * s.stage_bytes;
+  s.ok = true;
+  return s;
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 struct WorkspaceLayout {
   size_t part_max, part_sum, part_out, counters, total;
   int32_t max_parts;
+  bool stream;
 };
 
 WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
                               int32_t num_q_heads, int32_t max_blocks) {
   WorkspaceLayout w{};
+  if (plan_stream(c, num_q_heads).ok) {
+    // persistent kernel: (max, sum) and output per (CTA, head/tail slot, query head)
+    const size_t slots = (size_t)pa::stream::kMaxGrid * 2 * num_q_heads;
+    w.stream = true;
+    w.max_parts = 0;
+    w.part_max = 0;  // (max, sum) pairs
+    w.part_sum = 0;
+    w.part_out = round_up(slots * 2 * sizeof(float));
+    w.counters = round_up(w.part_out + slots * c->head_dim * sizeof(float));
+    w.total = round_up(w.counters + (size_t)batch * c->num_kv_heads * sizeof(int32_t));
+    return w;
+  }
   const int64_t tokens = (int64_t)max_blocks * c->block_size;
   w.max_parts = (int32_t)((tokens + kDecodePartitionTokens - 1) / kDecodePartitionTokens);
   const size_t n = (size_t)batch * num_q_heads * w.max_parts;
@@ -110,6 +179,7 @@ WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
   w.part_out = round_up(w.part_sum + n * sizeof(float));
   w.counters = round_up(w.part_out + n * c->head_dim * sizeof(float));
   w.total = round_up(w.counters + ncnt * sizeof(int32_t));
+  w.stream = false;
   return w;
 }
 
@@ -189,6 +259,48 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
     return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
   char *ws = static_cast<char *>(workspace);
+  if (w.stream) {
+    const StreamPlan sp = plan_stream(cache, num_q_heads);
+    const int sms = device_sm_count();
+    if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
+    pa::stream::Params p{};
+    p.q = q;
+    p.out = out;
+    p.key_cache = key_cache;
+    p.value_cache = value_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.part_ml = reinterpret_cast<float *>(ws + w.part_max);
+    p.part_o = reinterpret_cast<float *>(ws + w.part_out);
+    p.counters = reinterpret_cast<int32_t *>(ws + w.counters);
+    p.err_word = err_word;
+    p.num_blocks = cache->num_blocks;
+    p.block_size = cache->block_size;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.num_q_heads = num_q_heads;
+    p.max_blocks = max_blocks_per_seq;
+    p.batch = batch;
+    p.vbs = sp.vbs;
+    p.log2_vbs = sp.log2_vbs;
+    p.log2_vpp = sp.log2_vpp;
+    p.row_bytes = sp.row_bytes;
+    p.vpage_bytes = sp.vpage_bytes;
+    p.q_bytes = sp.q_bytes;
+    p.pps = sp.pps;
+    p.stages = sp.stages;
+    p.stage_bytes = sp.stage_bytes;
+    p.hdr_bytes = pa::stream::kHdrBytes;
+    p.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int group = num_q_heads / cache->num_kv_heads;
+    cudaError_t e = (cache->dtype == PA_DTYPE_BF16)
+                        ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
+                                                  sp.smem, static_cast<cudaStream_t>(stream))
+                        : pa::stream::launch_f32(p, cache->head_dim, group, cache->num_kv_heads,
+                                                 sp.smem, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+  }
   pa::DecodeArgs a{};
   a.q = q;
   a.out = out;

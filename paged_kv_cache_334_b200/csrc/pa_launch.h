@@ -27,6 +27,44 @@ struct DecodeArgs {
   bool merge;  // true: pa_decode (single-partition output + last-CTA merge)
 };
 
+namespace stream {
+
+constexpr int kMaxStages = 4;
+constexpr int kMaxPPS = 8;              // virtual pages per stage
+constexpr int kVPageBytes = 32 * 1024;  // largest virtual page (whole token rows)
+constexpr int kMaxGrid = 192;           // CTAs (one per SM); sizes the workspace
+constexpr int kHdrBytes = 8192;         // barriers, descriptors, score exchange
+constexpr int kSmemLimit = 232448;      // opt-in shared memory per CTA on sm_100
+
+// Arguments of the persistent decode kernel (decode_stream.cuh).
+struct Params {
+  const void *q;
+  void *out;
+  const void *key_cache;
+  const void *value_cache;
+  const int32_t *block_tables;
+  const int32_t *context_lens;
+  float *part_ml;     // [kMaxGrid * 2][Hq][2]: (max in log2 units, normaliser)
+  float *part_o;      // [kMaxGrid * 2][Hq][D]: normalised partial output
+  int32_t *counters;  // [batch * Hkv]
+  int32_t *err_word;
+  int32_t num_blocks, block_size, num_kv_heads, num_q_heads, max_blocks, batch;
+  int32_t vbs, log2_vbs, log2_vpp;  // virtual page tokens; log2 of pages per block
+  int32_t row_bytes;                // one token row, all KV heads
+  int32_t vpage_bytes;              // vbs * row_bytes
+  int32_t q_bytes;                  // Hq * D * elt
+  int32_t pps, stages, stage_bytes, hdr_bytes;
+  int32_t grid;
+  float scale_log2;
+};
+
+cudaError_t launch_bf16(const Params &p, int head_dim, int group, int hkv, size_t smem,
+                        cudaStream_t stream);
+cudaError_t launch_f32(const Params &p, int head_dim, int group, int hkv, size_t smem,
+                       cudaStream_t stream);
+
+}  // namespace stream
+
 // Query heads handled together by one CTA for a GQA group of `group` heads.
 int decode_head_tile(int group);
 

@@ -345,3 +345,91 @@ def test_negative_context_len_is_flagged():
     torch.cuda.synchronize()
     assert int(err.item()) == pa.PA_DEVERR_CONTEXT_LEN
     assert torch.all(out[0] == 0) and torch.all(torch.isfinite(out[1]))
+
+
+# ---------------------------------------------------------------------------
+# The persistent page-stream kernel (KV heads 4 or 8, group 1/2/4/8): shapes,
+# many sequences with empties, fewer pages than CTAs, long splits.
+# ---------------------------------------------------------------------------
+
+STREAM_SHAPES = [
+    # dtype, Hq, Hkv, D, bs
+    (wl.DTYPE_BF16, 8, 8, 128, 16),
+    (wl.DTYPE_BF16, 16, 8, 128, 16),
+    (wl.DTYPE_BF16, 64, 8, 128, 16),
+    (wl.DTYPE_F32, 32, 8, 128, 16),
+    (wl.DTYPE_BF16, 32, 8, 64, 32),
+    (wl.DTYPE_F32, 16, 4, 64, 8),
+    (wl.DTYPE_BF16, 32, 4, 128, 64),
+    (wl.DTYPE_BF16, 8, 8, 128, 1),
+    (wl.DTYPE_BF16, 32, 8, 128, 256),
+    (wl.DTYPE_F32, 4, 4, 128, 4),
+]
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", STREAM_SHAPES)
+def test_stream_kernel_shapes(dtype, Hq, Hkv, D, bs):
+    lens = [1, 15, 16, 17, 300, 1000, 2049, 4097]
+    w = wl.custom_workload(dtype=dtype, batch=len(lens), num_q_heads=Hq, num_kv_heads=Hkv,
+                           head_dim=D, block_size=bs, context_lens=lens, seed=Hq * 3 + bs,
+                           new_tokens=True)
+    d = upload(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gpu_write_and_decode(w, d, err)
+    torch.cuda.synchronize()
+    ref, _, _, _ = oracle_after_write(w)
+    assert int(err.item()) == 0
+    assert_close(to_f64(out), ref, dtype, f"stream {dtype} {Hq}/{Hkv} D{D} bs{bs}")
+
+
+def test_stream_many_sequences_with_empty_ones():
+    """700 sequences (more than one block of threads scans them), a third of
+    them empty, in runs longer than a 32-wide window."""
+    rng = np.random.default_rng(21)
+    lens = rng.integers(1, 600, size=700)
+    lens[rng.random(700) < 0.33] = 0
+    lens[100:170] = 0  # a run of 70 empty sequences
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=700, num_q_heads=32, num_kv_heads=8,
+                           head_dim=128, block_size=16, context_lens=lens.tolist(), seed=21,
+                           new_tokens=True)
+    d = upload(w)
+    out = torch.full_like(d["q"], float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_write_kv_cache(d["key_cache"], d["value_cache"], d["k_new"], d["v_new"],
+                         d["slot_mapping"], err_word=err)
+    pa.pa_decode(out, d["q"], d["key_cache"], d["value_cache"], d["block_tables"],
+                 d["context_lens"], err_word=err)
+    torch.cuda.synchronize()
+    ref, _, _, _ = oracle_after_write(w)
+    got = to_f64(out)
+    assert int(err.item()) == 0
+    assert np.all(got[lens == 0] == 0)
+    assert_close(got, ref, w.dtype, "700 sequences")
+
+
+@pytest.mark.parametrize("lens", [[100], [3, 5000], [1], [16, 16, 16]])
+def test_stream_fewer_pages_than_ctas(lens):
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=len(lens), num_q_heads=32,
+                           num_kv_heads=8, head_dim=128, block_size=16, context_lens=lens,
+                           seed=len(lens), new_tokens=True)
+    d = upload(w)
+    out = gpu_write_and_decode(w, d)
+    torch.cuda.synchronize()
+    ref, _, _, _ = oracle_after_write(w)
+    assert_close(to_f64(out), ref, w.dtype, f"lens {lens}")
+
+
+def test_stream_repeated_calls_keep_workspace_clean():
+    """Sequences split over many CTAs, decoded 5 times with the same
+    workspace: identical bits every time (counters reset by the merging
+    warp)."""
+    w = wl.make_workload("long_bf16", seed=3, batch=2)
+    d = upload(w)
+    outs = []
+    for _ in range(5):
+        outs.append(gpu_write_and_decode(w, d).clone())
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.uint16), outs[0].view(torch.uint16))
+    ref, _, _, _ = oracle_after_write(w)
+    assert_close(to_f64(outs[0]), ref, w.dtype, "long split")
