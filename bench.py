@@ -275,7 +275,7 @@ def workload_config(w, args):
         "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
         "context_tokens": int(w.context_lens.sum()), "seed": args.seed,
         "step": "pa_write_kv_cache(newest token of every sequence) + pa_decode",
-        "l2": "flushed before every timed step (zero-fill of 2x L2, outside the events)",
+        "l2": "flushed before every timed step (zero-fill then read of 2x L2, outside the events)",
         "parallelism": f"replicas: one independent batch per GPU x{args.gpus}",
     }
 
@@ -345,7 +345,16 @@ def run_ours(args):
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    flush_f32 = flush_buf.view(torch.float32)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
     launches_per_step = 2 if has_new else 1
+
+    def flush_l2():
+        # Write a buffer twice the L2 size, then read it back: the step's
+        # inputs are evicted and L2 is left holding clean lines, so the timed
+        # step pays no write-back of the flush itself.
+        flush_buf.zero_()
+        torch.amax(flush_f32, out=flush_sink)
 
     def write():
         if has_new:
@@ -356,7 +365,7 @@ def run_ours(args):
                      stream=stream)
 
     for _ in range(max(args.warmup, 3)):
-        flush_buf.zero_()
+        flush_l2()
         write()
         decode()
     torch.cuda.synchronize(dev)
@@ -372,7 +381,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     clocks.mark("t0")
     for k in range(K):
-        flush_buf.zero_()
+        flush_l2()
         ev[k][0].record(stream)
         write()
         ev[k][1].record(stream)
@@ -405,7 +414,7 @@ def run_ours(args):
         Ke = max(3, min(K, 500))
         eve = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
         for k in range(Ke + 3):
-            flush_buf.zero_()
+            flush_l2()
             if k >= 3:
                 eve[k - 3][0].record(stream)
             for dst, src in pairs:

@@ -95,7 +95,9 @@ pa_status check_decode_common(const pa_cache_desc *cache, const void *q,
 // served by the partition kernel of decode.cu instead.
 struct StreamPlan {
   bool ok;
-  int32_t vbs, log2_vbs, log2_vpp, row_bytes, vpage_bytes, q_bytes, pps, stages, stage_bytes;
+  int32_t vbs, log2_vbs, log2_vpp, row_bytes, row_pitch, vpage_stride, q_bytes, pps, stages,
+      stage_bytes;
+  int32_t heads_per_warp, warps_per_kv;
   size_t smem;
 };
 
@@ -111,24 +113,45 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads) {
   s.ok = false;
   const int32_t hkv = c->num_kv_heads;
   const int32_t group = num_q_heads / hkv;
-  if (hkv != 4 && hkv != 8) return s;
-  if (group != 1 && group != 2 && group != 4 && group != 8) return s;
+  const bool bf16 = c->dtype == PA_DTYPE_BF16;
+  if (bf16) {
+    // tensor-core consumers: one warp per (KV head, 8 query heads)
+    if (group > 8 && group % 8 != 0) return s;
+    s.heads_per_warp = group < 8 ? group : 8;
+    s.warps_per_kv = group > 8 ? group / 8 : 1;
+    const int32_t ncw = hkv * s.warps_per_kv;
+    if (ncw != 4 && ncw != 8 && ncw != 16) return s;
+  } else {
+    // CUDA-core consumers: one warp per KV head
+    if (hkv != 4 && hkv != 8) return s;
+    if (group != 1 && group != 2 && group != 4 && group != 8) return s;
+    s.heads_per_warp = group;
+    s.warps_per_kv = 1;
+  }
   const int32_t elt = elem_bytes(c->dtype);
   s.row_bytes = hkv * c->head_dim * elt;
-  if (s.row_bytes > st::kVPageBytes) return s;
-  const int32_t rows = st::kVPageBytes / s.row_bytes;
+  // tensor-core tiles read 8 token rows at one column: pad rows by 16 bytes so
+  // those rows fall in 8 different shared-memory bank groups
+  s.row_pitch = bf16 ? s.row_bytes + 16 : s.row_bytes;
+  if (s.row_pitch > st::kVPageBytes) return s;
+  const int32_t rows = st::kVPageBytes / s.row_bytes;  // power of two
   s.vbs = c->block_size < rows ? c->block_size : rows;
   s.log2_vbs = ilog2(s.vbs);
   s.log2_vpp = ilog2(c->block_size / s.vbs);
-  s.vpage_bytes = s.vbs * s.row_bytes;
-  s.pps = st::kVPageBytes / s.vpage_bytes;
+  // tensor-core tiles span 16 token rows: give every page slot at least 16
+  s.vpage_stride = (bf16 && s.vbs < 16 ? 16 : s.vbs) * s.row_pitch;
+  s.q_bytes = num_q_heads * c->head_dim * elt;
+  s.pps = st::kVPageBytes / s.vpage_stride;
   if (s.pps > st::kMaxPPS) s.pps = st::kMaxPPS;
   if (s.pps < 1) s.pps = 1;
-  s.q_bytes = num_q_heads * c->head_dim * elt;
-  s.stage_bytes = (int32_t)(((size_t)2 * s.pps * s.vpage_bytes + (size_t)s.pps * s.q_bytes + 127) /
-                            128 * 128);
-  s.stages = (st::kSmemLimit - st::kHdrBytes) / s.stage_bytes;
-  if (s.stages > st::kMaxStages) s.stages = st::kMaxStages;
+  for (;;) {
+    s.stage_bytes = (int32_t)(((size_t)2 * s.pps * s.vpage_stride + (size_t)s.pps * s.q_bytes +
+                               127) / 128 * 128);
+    s.stages = (st::kSmemLimit - st::kHdrBytes) / s.stage_bytes;
+    if (s.stages > st::kMaxStages) s.stages = st::kMaxStages;
+    if (s.stages >= 3 || s.pps == 1) break;
+    --s.pps;
+  }
   if (s.stages < 2) return s;
   s.smem = (size_t)st::kHdrBytes + (size_t)s.stages * s.stage_bytes;
   s.ok = true;
@@ -156,16 +179,19 @@ struct WorkspaceLayout {
 WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
                               int32_t num_q_heads, int32_t max_blocks) {
   WorkspaceLayout w{};
-  if (plan_stream(c, num_q_heads).ok) {
-    // persistent kernel: (max, sum) and output per (CTA, head/tail slot, query head)
+  const StreamPlan sp = plan_stream(c, num_q_heads);
+  if (sp.ok) {
+    // persistent kernel: (max, sum) and output per (CTA, head/tail slot, query
+    // head); one arrival counter per (sequence, query-head slice of a warp)
     const size_t slots = (size_t)pa::stream::kMaxGrid * 2 * num_q_heads;
+    const size_t slices = (size_t)num_q_heads / sp.heads_per_warp;
     w.stream = true;
     w.max_parts = 0;
     w.part_max = 0;  // (max, sum) pairs
     w.part_sum = 0;
     w.part_out = round_up(slots * 2 * sizeof(float));
     w.counters = round_up(w.part_out + slots * c->head_dim * sizeof(float));
-    w.total = round_up(w.counters + (size_t)batch * c->num_kv_heads * sizeof(int32_t));
+    w.total = round_up(w.counters + (size_t)batch * slices * sizeof(int32_t));
     return w;
   }
   const int64_t tokens = (int64_t)max_blocks * c->block_size;
@@ -284,7 +310,8 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
     p.log2_vbs = sp.log2_vbs;
     p.log2_vpp = sp.log2_vpp;
     p.row_bytes = sp.row_bytes;
-    p.vpage_bytes = sp.vpage_bytes;
+    p.row_pitch = sp.row_pitch;
+    p.vpage_stride = sp.vpage_stride;
     p.q_bytes = sp.q_bytes;
     p.pps = sp.pps;
     p.stages = sp.stages;
@@ -293,6 +320,9 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
     p.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
     p.scale_log2 = scale * 1.4426950408889634f;
     const int group = num_q_heads / cache->num_kv_heads;
+    p.group = group;
+    p.heads_per_warp = sp.heads_per_warp;
+    p.warps_per_kv = sp.warps_per_kv;
     cudaError_t e = (cache->dtype == PA_DTYPE_BF16)
                         ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
                                                   sp.smem, static_cast<cudaStream_t>(stream))

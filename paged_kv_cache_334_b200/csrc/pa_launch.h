@@ -50,11 +50,15 @@ struct Params {
   int32_t *err_word;
   int32_t num_blocks, block_size, num_kv_heads, num_q_heads, max_blocks, batch;
   int32_t vbs, log2_vbs, log2_vpp;  // virtual page tokens; log2 of pages per block
-  int32_t row_bytes;                // one token row, all KV heads
-  int32_t vpage_bytes;              // vbs * row_bytes
+  int32_t row_bytes;                // one token row, all KV heads (global layout)
+  int32_t row_pitch;                // bytes between token rows in a shared-memory stage
+  int32_t vpage_stride;             // vbs * row_pitch
   int32_t q_bytes;                  // Hq * D * elt
   int32_t pps, stages, stage_bytes, hdr_bytes;
   int32_t grid;
+  int32_t group;                    // query heads per KV head
+  int32_t heads_per_warp;           // query heads one consumer warp serves (<= 8)
+  int32_t warps_per_kv;             // consumer warps per KV head
   float scale_log2;
 };
 

@@ -133,11 +133,11 @@ def test_noalloc_size_limit_and_argument_checks(lib):
     """pa_decode_noalloc refuses sizes whose workspace exceeds its fixed
     scratch before any device work, and passes other argument errors
     through from pa_decode."""
-    d = _desc(nb=100000, bs=16, hkv=1, d=128)
-    need = lib.pa_decode_workspace_bytes(ctypes.byref(d), 4096, 64, 1024)
+    d = _desc(nb=100000, bs=16, hkv=2, d=128)
+    need = lib.pa_decode_workspace_bytes(ctypes.byref(d), 4096, 2, 1024)
     assert need > pa.NOALLOC_SCRATCH_BYTES
     f = lib.pa_decode_noalloc
-    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, 64, 1024, 0.1, None,
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, 2, 1024, 0.1, None,
              None) == pa.PA_ERR_UNSUPPORTED
     assert b"scratch" in lib.pa_last_error_message()
     assert f(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4, 0.1, None, None) == \

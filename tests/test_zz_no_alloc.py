@@ -72,7 +72,11 @@ def test_noalloc_alternating_shapes_reuse_the_scratch():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    w = wl.make_workload("mqa_prefix_bf16", seed=0, batch=64)
+    # a table long enough for 65536 tokens per sequence: the workspace would
+    # exceed the fixed scratch even though the actual contexts are short
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=64, num_q_heads=2, num_kv_heads=2,
+                           head_dim=128, block_size=16, context_lens=[10] * 64, seed=2,
+                           max_blocks=4096)
     need = pa.pa_decode_workspace_bytes(upload_shape(w), w.batch, w.num_q_heads, w.max_blocks)
     assert need > pa.NOALLOC_SCRATCH_BYTES
     d = upload(w)
