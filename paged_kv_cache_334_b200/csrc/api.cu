@@ -4,6 +4,7 @@
 // and enqueues kernels on the caller's stream.  It never allocates, never
 // synchronises and has no CPU fallback: every step of the computation runs in
 // the kernels of write_kv.cu, decode.cu and reduce.cu.
+#include <cudaTypedefs.h>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -95,8 +96,9 @@ pa_status check_decode_common(const pa_cache_desc *cache, const void *q,
 // served by the partition kernel of decode.cu instead.
 struct StreamPlan {
   bool ok;
+  bool tile;  // bf16 pages of >= 16 tokens: tensor copies of swizzled boxes
   int32_t vbs, log2_vbs, log2_vpp, row_bytes, row_pitch, vpage_stride, q_bytes, pps, stages,
-      stage_bytes;
+      stage_bytes, box_bytes, n_dhalf;
   int32_t heads_per_warp, warps_per_kv;
   size_t smem;
 };
@@ -107,7 +109,7 @@ int32_t ilog2(int32_t x) {
   return l;
 }
 
-StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads) {
+StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_tile = true) {
   namespace st = pa::stream;
   StreamPlan s{};
   s.ok = false;
@@ -130,32 +132,78 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads) {
   }
   const int32_t elt = elem_bytes(c->dtype);
   s.row_bytes = hkv * c->head_dim * elt;
-  // tensor-core tiles read 8 token rows at one column: pad rows by 16 bytes so
-  // those rows fall in 8 different shared-memory bank groups
-  s.row_pitch = bf16 ? s.row_bytes + 16 : s.row_bytes;
-  if (s.row_pitch > st::kVPageBytes) return s;
+  if (s.row_bytes + 16 > st::kVPageBytes) return s;
   const int32_t rows = st::kVPageBytes / s.row_bytes;  // power of two
   s.vbs = c->block_size < rows ? c->block_size : rows;
   s.log2_vbs = ilog2(s.vbs);
   s.log2_vpp = ilog2(c->block_size / s.vbs);
-  // tensor-core tiles span 16 token rows: give every page slot at least 16
-  s.vpage_stride = (bf16 && s.vbs < 16 ? 16 : s.vbs) * s.row_pitch;
+  s.tile = allow_tile && bf16 && s.vbs >= 16 && hkv <= 256;
+  s.n_dhalf = c->head_dim / 64;
+  s.box_bytes = 128 * s.vbs * hkv;
+  if (s.tile) {
+    // boxes land back to back: no padding, the swizzle keeps ldmatrix conflict-free
+    s.row_pitch = s.row_bytes;
+    s.vpage_stride = s.vbs * s.row_bytes;
+  } else if (bf16) {
+    // row copies at a 16-byte padded pitch; tiles span 16 rows, so slots get >= 16
+    s.row_pitch = s.row_bytes + 16;
+    s.vpage_stride = (s.vbs < 16 ? 16 : s.vbs) * s.row_pitch;
+  } else {
+    s.row_pitch = s.row_bytes;
+    s.vpage_stride = s.vbs * s.row_bytes;
+  }
   s.q_bytes = num_q_heads * c->head_dim * elt;
   s.pps = st::kVPageBytes / s.vpage_stride;
   if (s.pps > st::kMaxPPS) s.pps = st::kMaxPPS;
   if (s.pps < 1) s.pps = 1;
+  const int32_t avail = st::kSmemLimit - st::kHdrBytes - 1024;  // 1 KB alignment slack
   for (;;) {
     s.stage_bytes = (int32_t)(((size_t)2 * s.pps * s.vpage_stride + (size_t)s.pps * s.q_bytes +
-                               127) / 128 * 128);
-    s.stages = (st::kSmemLimit - st::kHdrBytes) / s.stage_bytes;
+                               1023) / 1024 * 1024);
+    s.stages = avail / s.stage_bytes;
     if (s.stages > st::kMaxStages) s.stages = st::kMaxStages;
     if (s.stages >= 3 || s.pps == 1) break;
     --s.pps;
   }
   if (s.stages < 2) return s;
-  s.smem = (size_t)st::kHdrBytes + (size_t)s.stages * s.stage_bytes;
+  s.smem = (size_t)st::kHdrBytes + 1024 + (size_t)s.stages * s.stage_bytes;
   s.ok = true;
   return s;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    tried = true;
+  }
+  return fn;
+}
+
+// 3-D view (head_dim, token row of the pool, KV head) of a bf16 cache with
+// boxes of 64 x vbs x Hkv and 128-byte swizzle.
+bool encode_cache_map(CUtensorMap *map, const void *base, const pa_cache_desc *c, int32_t vbs) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)c->head_dim,
+                              (cuuint64_t)c->num_blocks * (cuuint64_t)c->block_size,
+                              (cuuint64_t)c->num_kv_heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)c->num_kv_heads * c->head_dim * 2,
+                                 (cuuint64_t)c->head_dim * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)vbs, (cuuint32_t)c->num_kv_heads};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 int device_sm_count() {
@@ -286,10 +334,13 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
     return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
   char *ws = static_cast<char *>(workspace);
   if (w.stream) {
-    const StreamPlan sp = plan_stream(cache, num_q_heads);
+    StreamPlan sp = plan_stream(cache, num_q_heads);
     const int sms = device_sm_count();
     if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
     pa::stream::Params p{};
+    if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, sp.vbs) &&
+                     encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs)))
+      sp = plan_stream(cache, num_q_heads, /*allow_tile=*/false);
     p.q = q;
     p.out = out;
     p.key_cache = key_cache;
@@ -323,6 +374,9 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
     p.group = group;
     p.heads_per_warp = sp.heads_per_warp;
     p.warps_per_kv = sp.warps_per_kv;
+    p.tile = sp.tile ? 1 : 0;
+    p.box_bytes = sp.box_bytes;
+    p.n_dhalf = sp.n_dhalf;
     cudaError_t e = (cache->dtype == PA_DTYPE_BF16)
                         ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
                                                   sp.smem, static_cast<cudaStream_t>(stream))

@@ -110,6 +110,15 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gsrc, uint3
       "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Tiled tensor copy of one box (coordinates innermost first), no multicast.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, int x, int y,
+                                            int z, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -211,6 +220,7 @@ struct MmaConsumer {
   uint32_t qb[KS][2];                // Q^T as B operand (d x head), one pair per k step
   float o[KS][4];                    // O^T accumulators
   float m0, m1, l0, l1;              // running max / partial normaliser, heads 2t, 2t+1
+  float scale_log2_;
   bool seg_bad;
 
   __device__ __forceinline__ void reset() {
@@ -238,28 +248,35 @@ struct MmaConsumer {
     }
   }
 
-  // One staged virtual page of `ntok` tokens, rows `pitch` bytes apart; the
-  // head's slice starts `col_bytes` into each row.
+  // One staged virtual page of `ntok` tokens.  Layouts:
+  //  tile  : per 64-wide d half a box of [KV head][vbs tokens][128 B] rows with
+  //          the 16-byte chunk index XORed with (row % 8) (128-byte swizzle);
+  //  padded: token rows `pitch` bytes apart, this head's slice at col_bytes.
+  // Either way eight consecutive tokens at one chunk hit eight bank groups.
   __device__ __forceinline__ void page(const unsigned char *kp, const unsigned char *vp,
-                                       int ntok, int pitch, int col_bytes, float scale_log2,
+                                       int ntok, const Params &p, int h, int col_bytes,
                                        int lane) {
-    const int g = lane >> 2;
+    const int g = lane >> 2, t = lane & 3;
+    const bool tile = p.tile != 0;
     for (int m0t = 0; m0t < ntok; m0t += 16) {
       // S^T (16 tokens x 8 heads) = K (16 x D) Q^T (D x 8)
       float s[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t kaddr = smem_u32(kp + (size_t)(m0t + (lane & 15)) * pitch + col_bytes +
-                                      (lane >> 4) * 16);
+      const int tk = m0t + (lane & 15), hk = lane >> 4;
+      const int rowk = tile ? (h * p.vbs + tk) * 128 : tk * p.row_pitch + col_bytes;
 #pragma unroll
       for (int k = 0; k < KS; ++k) {
+        const int cg = k * 2 + hk;  // 16-byte chunk of the row (8 elements)
+        const int off = tile ? (cg >> 3) * p.box_bytes + rowk + (((cg & 7) ^ (tk & 7)) << 4)
+                             : rowk + cg * 16;
         uint32_t a[4];
-        ldsm_x4(a, kaddr + k * 32);
+        ldsm_x4(a, smem_u32(kp + off));
         mma_16816(s, a, qb[k][0], qb[k][1]);
       }
       const bool v0 = m0t + g < ntok, v1 = m0t + g + 8 < ntok;
-      s[0] = v0 ? s[0] * scale_log2 : -INFINITY;
-      s[1] = v0 ? s[1] * scale_log2 : -INFINITY;
-      s[2] = v1 ? s[2] * scale_log2 : -INFINITY;
-      s[3] = v1 ? s[3] * scale_log2 : -INFINITY;
+      s[0] = v0 ? s[0] * scale_log2_ : -INFINITY;
+      s[1] = v0 ? s[1] * scale_log2_ : -INFINITY;
+      s[2] = v1 ? s[2] * scale_log2_ : -INFINITY;
+      s[3] = v1 ? s[3] * scale_log2_ : -INFINITY;
       float x0 = fmaxf(s[0], s[2]), x1 = fmaxf(s[1], s[3]);
 #pragma unroll
       for (int mask = 4; mask < 32; mask <<= 1) {
@@ -286,15 +303,30 @@ struct MmaConsumer {
       // P^T (16 tokens x 8 heads) as the B operand: transpose the two 8x8 tiles.
       const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
       const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
-      // Rows past ntok hold stale (finite) data of earlier pages or zeros;
-      // their P is 0, so they add nothing.
+      // V rows past ntok may hold anything (other tokens, never-written
+      // shared memory): their P is 0, and their V elements are zeroed below
+      // so that 0 * NaN cannot occur.
+      const bool partial = m0t + 16 > ntok;
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (partial) {
+        mlo = (m0t + 2 * t < ntok ? 0x0000ffffu : 0u) | (m0t + 2 * t + 1 < ntok ? 0xffff0000u : 0u);
+        mhi = (m0t + 2 * t + 8 < ntok ? 0x0000ffffu : 0u) |
+              (m0t + 2 * t + 9 < ntok ? 0xffff0000u : 0u);
+      }
       const int mi = lane >> 3, rr = lane & 7;
-      const uint32_t vaddr = smem_u32(vp + (size_t)(m0t + rr + ((mi >> 1) << 3)) * pitch +
-                                      col_bytes + (mi & 1) * 16);
+      const int tv = m0t + rr + ((mi >> 1) << 3), hv = mi & 1;
+      const int rowv = tile ? (h * p.vbs + tv) * 128 : tv * p.row_pitch + col_bytes;
 #pragma unroll
       for (int k = 0; k < KS; ++k) {
+        const int cg = k * 2 + hv;
+        const int off = tile ? (cg >> 3) * p.box_bytes + rowv + (((cg & 7) ^ (tv & 7)) << 4)
+                             : rowv + cg * 16;
         uint32_t a[4];
-        ldsm_x4_trans(a, vaddr + k * 32);
+        ldsm_x4_trans(a, smem_u32(vp + off));
+        a[0] &= mlo;
+        a[1] &= mlo;
+        a[2] &= mhi;
+        a[3] &= mhi;
         mma_16816(o[k], a, b0, b1);
       }
     }
@@ -671,7 +703,8 @@ struct FmaConsumer {
 // for the fp32 consumer (unused, 0, for bf16); NCW = consumer warps.
 // ===========================================================================
 template <typename T, int D, int G, int NCW>
-__global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_stream_kernel(const Params p) {
+__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+    decode_stream_kernel(const __grid_constant__ Params p) {
   constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
   constexpr int kScoreFloats = kMma ? 1 : FmaConsumer<T, D, (G > 0 ? G : 1)>::E;
   static_assert(sizeof(Shared) + sizeof(PageDesc) * kMaxStages * kMaxPPS +
@@ -686,7 +719,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_stream_kernel(const 
   PageDesc *descs = reinterpret_cast<PageDesc *>(smem_raw + sizeof(Shared));
   float *s_scores = reinterpret_cast<float *>(smem_raw + sizeof(Shared) +
                                               sizeof(PageDesc) * kMaxStages * kMaxPPS);
-  unsigned char *stages = smem_raw + p.hdr_bytes;
+  // stages start 1024-byte aligned (the 128-byte swizzle repeats every 1 KB)
+  unsigned char *stages =
+      smem_raw + (((smem_u32(smem_raw) + p.hdr_bytes + 1023u) & ~1023u) - smem_u32(smem_raw));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
@@ -699,19 +734,6 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_stream_kernel(const 
     sh.abort_flag = 0;
     // make the initialised barriers visible to the bulk-copy (async) proxy
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if constexpr (kMma) {
-    // Tensor-core tiles also read the rows past a page's valid tokens (their
-    // P is 0).  Start every V area at zero so those rows are finite; rows
-    // written later by copies hold finite cache data.
-    for (int sl = 0; sl < p.stages; ++sl) {
-      uint4 *v = reinterpret_cast<uint4 *>(stages + (size_t)sl * p.stage_bytes +
-                                           (size_t)p.pps * p.vpage_stride);
-      const int n = p.pps * p.vpage_stride / 16;
-      for (int x = tid; x < n; x += blockDim.x) v[x] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    // order these generic-proxy stores before the bulk copies (async proxy)
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
 
   // ---- Prologue: total virtual pages T, this CTA's range and first page.
@@ -805,7 +827,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_stream_kernel(const 
             }
             descs[slot * kMaxPPS + k] = d;
           }
-          if (!bad) bytes += 2u * (uint32_t)ntok * (uint32_t)p.row_bytes;
+          if (!bad)
+            bytes += p.tile ? 2u * (uint32_t)p.n_dhalf * (uint32_t)p.box_bytes
+                            : 2u * (uint32_t)ntok * (uint32_t)p.row_bytes;
           if (first) bytes += (uint32_t)p.q_bytes;
           // advance the cursor
           ++cursor;
@@ -844,7 +868,16 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_stream_kernel(const 
         unsigned char *qst = st + (size_t)2 * p.pps * p.vpage_stride;
         for (int k = 0; k < npg; ++k) {
           const PageDesc d = descs[slot * kMaxPPS + k];
-          if (!(d.flags & kBad)) {
+          if (!(d.flags & kBad) && p.tile) {
+            // one box per (tensor, 64-wide d half), one lane each
+            if (lane < 2 * p.n_dhalf) {
+              const int dh = lane % p.n_dhalf;
+              const bool isv = lane >= p.n_dhalf;
+              tma_load_3d((isv ? vst : kst) + (size_t)k * p.vpage_stride + (size_t)dh * p.box_bytes,
+                          isv ? &p.tmap_v : &p.tmap_k, dh * 64, d.pb * p.block_size + d.toff, 0,
+                          &sh.full[slot]);
+            }
+          } else if (!(d.flags & kBad)) {
             const int64_t off = ((int64_t)d.pb * p.block_size + d.toff) * (int64_t)p.row_bytes;
             const unsigned char *ksrc = static_cast<const unsigned char *>(p.key_cache) + off;
             const unsigned char *vsrc = static_cast<const unsigned char *>(p.value_cache) + off;
@@ -889,6 +922,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_stream_kernel(const 
       const int col_bytes = h * D * (int)sizeof(T);
       Cons cs;
       cs.reset();
+      if constexpr (kMma) cs.scale_log2_ = p.scale_log2;
       float *sc_buf = s_scores + (size_t)cw_idx * kScoreFloats;
       int64_t cursor = start;
       for (int i = 0; i < n_stages; ++i) {
@@ -924,7 +958,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_stream_kernel(const 
             const unsigned char *kp = kst + (size_t)k * p.vpage_stride;
             const unsigned char *vp = vst + (size_t)k * p.vpage_stride;
             if constexpr (kMma) {
-              cs.page(kp, vp, d.ntok, p.row_pitch, col_bytes, p.scale_log2, lane);
+              cs.page(kp, vp, d.ntok, p, h, col_bytes, lane);
             } else {
               cs.page(kp, vp, d.ntok, p.row_pitch, col_bytes, sc_buf, lane);
             }

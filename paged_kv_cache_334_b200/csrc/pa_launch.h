@@ -1,6 +1,7 @@
 // pa_launch.h -- internal launchers behind the C ABI (host side).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -38,6 +39,11 @@ constexpr int kSmemLimit = 232448;      // opt-in shared memory per CTA on sm_10
 
 // Arguments of the persistent decode kernel (decode_stream.cuh).
 struct Params {
+  // 3-D tiled views (head_dim, token row of the pool, KV head) of the caches,
+  // boxes of 64 elements x vbs tokens x all KV heads, 128-byte swizzle; used
+  // when `tile` is set (bf16, vbs >= 16).
+  CUtensorMap tmap_k;
+  CUtensorMap tmap_v;
   const void *q;
   void *out;
   const void *key_cache;
@@ -59,6 +65,9 @@ struct Params {
   int32_t group;                    // query heads per KV head
   int32_t heads_per_warp;           // query heads one consumer warp serves (<= 8)
   int32_t warps_per_kv;             // consumer warps per KV head
+  int32_t tile;                     // 1: tensor copies of swizzled boxes, else row copies
+  int32_t box_bytes;                // bytes of one box (64 x vbs x Hkv bf16)
+  int32_t n_dhalf;                  // boxes per page per tensor (head_dim / 64)
   float scale_log2;
 };
 
