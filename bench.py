@@ -49,8 +49,10 @@ from paged_kv_cache_334_b200 import workloads as wl  # noqa: E402
 
 METRIC = "decode-attention KV GB/s & fraction of B200 HBM peak; seq-tokens/s per step"
 FALLBACK_HBM_GBS = 6650.0
-DECODE_SOURCE = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc", "decode.cu")
-DECODE_HELPERS = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc", "pa_common.cuh")
+CSRC = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc")
+# sources that define the decode kernel's code and launch shape
+DECODE_SOURCES = ("decode_stream.cuh", "decode_stream_bf16.cu", "decode_stream_f32.cu",
+                  "pa_common.cuh", "pa_launch.h", "api.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.md")
 
 
@@ -193,12 +195,37 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "6.65 TB/s fallback (of fallback)"
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and blank-line or indentation
+    differences, so that editing a comment keeps the recorded counters."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] in "\"'":
+            q, j = text[i], i + 1
+            while j < n and text[j] != q:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    lines = (ln.strip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def decode_source_hash() -> str:
-    """Hash of the decode kernel's own sources (kernel file + device helpers)."""
+    """Hash of the decode kernel's code (kernel, device helpers, launch plan),
+    comments excluded."""
     h = hashlib.sha256()
-    for path in (DECODE_SOURCE, DECODE_HELPERS):
-        with open(path, "rb") as f:
-            h.update(os.path.basename(path).encode() + f.read())
+    for name in DECODE_SOURCES:
+        with open(os.path.join(CSRC, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -141,9 +141,11 @@ size_t pa_decode_workspace_bytes(const pa_cache_desc *cache, int32_t batch,
  *
  * scale is usually 1 / sqrt(head_dim).  workspace: device memory of at
  * least pa_decode_workspace_bytes(...) bytes, 256-byte aligned, ZERO-FILLED
- * before its first use; every call leaves it zero-filled again on return,
- * so one buffer serves any number of stream-ordered calls.  Calls that
- * overlap on the GPU must not share a workspace.
+ * before its first use; every call leaves it ready for the next one, so one
+ * buffer serves any number of stream-ordered calls.  Calls that overlap on
+ * the GPU must not share a workspace.  A call may run as more than one
+ * kernel; the later ones are launched with programmatic stream
+ * serialisation and wait for the earlier ones.
  */
 pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
                     const void *key_cache, const void *value_cache,

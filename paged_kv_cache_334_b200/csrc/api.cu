@@ -3,7 +3,9 @@
 // This layer validates arguments on the host, lays out the decode workspace
 // and enqueues kernels on the caller's stream.  It never allocates, never
 // synchronises and has no CPU fallback: every step of the computation runs in
-// the kernels of write_kv.cu, decode.cu and reduce.cu.
+// the kernels of write_kv.cu, decode_stream.cuh (persistent page-stream decode
+// and its merge kernel), decode.cu (partition decode for split-K and the
+// shapes the stream kernel does not cover) and reduce.cu.
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <stdio.h>
@@ -230,16 +232,15 @@ WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
   const StreamPlan sp = plan_stream(c, num_q_heads);
   if (sp.ok) {
     // persistent kernel: (max, sum) and output per (CTA, head/tail slot, query
-    // head); one arrival counter per (sequence, query-head slice of a warp)
+    // head); one merge record (4 x int32) per sequence
     const size_t slots = (size_t)pa::stream::kMaxGrid * 2 * num_q_heads;
-    const size_t slices = (size_t)num_q_heads / sp.heads_per_warp;
     w.stream = true;
     w.max_parts = 0;
     w.part_max = 0;  // (max, sum) pairs
     w.part_sum = 0;
     w.part_out = round_up(slots * 2 * sizeof(float));
     w.counters = round_up(w.part_out + slots * c->head_dim * sizeof(float));
-    w.total = round_up(w.counters + (size_t)batch * slices * sizeof(int32_t));
+    w.total = round_up(w.counters + (size_t)batch * 4 * sizeof(int32_t));
     return w;
   }
   const int64_t tokens = (int64_t)max_blocks * c->block_size;
@@ -349,7 +350,7 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
     p.context_lens = context_lens;
     p.part_ml = reinterpret_cast<float *>(ws + w.part_max);
     p.part_o = reinterpret_cast<float *>(ws + w.part_out);
-    p.counters = reinterpret_cast<int32_t *>(ws + w.counters);
+    p.seq_merge = reinterpret_cast<int32_t *>(ws + w.counters);
     p.err_word = err_word;
     p.num_blocks = cache->num_blocks;
     p.block_size = cache->block_size;
@@ -383,6 +384,10 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
                         : pa::stream::launch_f32(p, cache->head_dim, group, cache->num_kv_heads,
                                                  sp.smem, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    e = (cache->dtype == PA_DTYPE_BF16)
+            ? pa::stream::launch_merge_bf16(p, cache->head_dim, static_cast<cudaStream_t>(stream))
+            : pa::stream::launch_merge_f32(p, cache->head_dim, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
     return PA_OK;
   }
   pa::DecodeArgs a{};

@@ -16,12 +16,17 @@
 //   whatever the mix of context lengths.
 // * Producer warp: walks its range (block-table entries fetched 32 at a time
 //   into registers, context lengths likewise), validates each physical block
-//   id, and issues 1-D bulk copies (cp.async.bulk, no multicast) of the valid
-//   token rows of K and V -- plus the sequence's query rows when a sequence
-//   segment starts -- into a ring of shared-memory stages guarded by mbarriers.
-//   For the tensor-core consumers each token row lands at a pitch of
-//   row_bytes + 16 so that eight consecutive tokens fall in eight different
-//   shared-memory bank groups (conflict-free ldmatrix).
+//   id, and fills a ring of shared-memory stages guarded by mbarriers (no
+//   multicast anywhere):
+//     - bf16 with >= 16 tokens per virtual page: tiled tensor copies
+//       (cp.async.bulk.tensor.3d) of boxes [64 d][vbs tokens][Hkv heads] of
+//       K and V with the 128-byte swizzle, one box per 64-wide half of D, so
+//       a whole virtual page takes 2 * D/64 copies and ldmatrix reads it
+//       without bank conflicts;
+//     - otherwise: 1-D bulk copies (cp.async.bulk) of the valid token rows,
+//       landing at a pitch of row_bytes + 16 for the tensor-core consumers
+//       (eight consecutive tokens in eight different bank groups);
+//   plus the sequence's query rows when a sequence segment starts.
 // * Consumer warps keep the online-softmax state (running max, normaliser,
 //   fp32 accumulator) of up to 8 query heads of one KV head for the current
 //   sequence segment.
@@ -31,9 +36,10 @@
 //       bf16 and turned into the B operand with movmatrix.
 //     - fp32: CUDA-core FMAs, per-(token, head) dot products reduced with a
 //       transposed butterfly (the 1e-5 tolerance rules out bf16/tf32 MMA).
-// * A sequence split across CTAs leaves one partial per CTA in the workspace;
-//   the last warp to finish (per sequence and query-head slice, found with an
-//   atomic counter -- nobody waits) merges them and resets the counter.
+// * A sequence split across CTAs leaves one partial per CTA in the workspace,
+//   and the CTA that owns its last page records where they are; a small merge
+//   kernel (launched right behind, programmatically) folds them together with
+//   the running-max rescaling once the stream of pages is done.
 //
 // Every mbarrier wait is bounded; on expiry the kernel sets PA_DEVERR_TIMEOUT,
 // drains its own copies (bounded) and returns.
@@ -144,6 +150,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// 2^x with the hardware approximation (inputs here are <= 0: softmax
+// weights; results below the normal range flush to zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -219,7 +232,7 @@ struct MmaConsumer {
   static constexpr int KS = D / 16;  // k steps of QK, d tiles of PV
   uint32_t qb[KS][2];                // Q^T as B operand (d x head), one pair per k step
   float o[KS][4];                    // O^T accumulators
-  float m0, m1, l0, l1;              // running max / partial normaliser, heads 2t, 2t+1
+  float m0_, m1_, l0, l1;            // running max / partial normaliser, heads 2t, 2t+1
   float scale_log2_;
   bool seg_bad;
 
@@ -228,7 +241,7 @@ struct MmaConsumer {
     for (int k = 0; k < KS; ++k)
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[k][e] = 0.f;
-    m0 = m1 = -INFINITY;
+    m0_ = m1_ = -INFINITY;
     l0 = l1 = 0.f;
     seg_bad = false;
   }
@@ -249,93 +262,147 @@ struct MmaConsumer {
   }
 
   // One staged virtual page of `ntok` tokens.  Layouts:
-  //  tile  : per 64-wide d half a box of [KV head][vbs tokens][128 B] rows with
-  //          the 16-byte chunk index XORed with (row % 8) (128-byte swizzle);
+  //  TL (tile): per 64-wide d half a box of [KV head][vbs tokens][128 B] rows
+  //          with the 16-byte chunk index XORed with (row % 8) (128-byte
+  //          swizzle); a tile's first row is a multiple of 16, so a lane's
+  //          XOR term depends only on its own lane bits;
   //  padded: token rows `pitch` bytes apart, this head's slice at col_bytes.
   // Either way eight consecutive tokens at one chunk hit eight bank groups.
-  __device__ __forceinline__ void page(const unsigned char *kp, const unsigned char *vp,
-                                       int ntok, const Params &p, int h, int col_bytes,
-                                       int lane) {
+  // Tokens go in groups of NT (1 or 2) 16-token tiles that share one max
+  // reduction and one rescale; each tile's QK runs as two independent MMA
+  // chains, so the dependent-latency path per token is short.
+  template <int NT, bool TL>
+  __device__ __forceinline__ void tiles(const unsigned char *kp, const unsigned char *vp, int m0,
+                                        int ntok, const Params &p, int h, int col_bytes,
+                                        int lane) {
     const int g = lane >> 2, t = lane & 3;
-    const bool tile = p.tile != 0;
-    for (int m0t = 0; m0t < ntok; m0t += 16) {
-      // S^T (16 tokens x 8 heads) = K (16 x D) Q^T (D x 8)
-      float s[4] = {0.f, 0.f, 0.f, 0.f};
-      const int tk = m0t + (lane & 15), hk = lane >> 4;
-      const int rowk = tile ? (h * p.vbs + tk) * 128 : tk * p.row_pitch + col_bytes;
+    // K operand rows: token m0 + 16u + (lane & 15), chunk 2k + (lane >> 4)
+    const int xk = ((lane >> 4) ^ (lane & 7)) << 4;   // TL: XOR term of chunk 2k
+    const int ck = (lane >> 4) << 4;                  // padded: chunk offset
+    // V operand rows (transposed load): token base + (lane & 7) + 8 * (lane >> 4),
+    // chunk 2k + ((lane >> 3) & 1)
+    const int mi = lane >> 3;
+    const int xv = ((mi & 1) ^ (lane & 7)) << 4;
+    const int cv = (mi & 1) << 4;
+    float s[NT][4];
 #pragma unroll
-      for (int k = 0; k < KS; ++k) {
-        const int cg = k * 2 + hk;  // 16-byte chunk of the row (8 elements)
-        const int off = tile ? (cg >> 3) * p.box_bytes + rowk + (((cg & 7) ^ (tk & 7)) << 4)
-                             : rowk + cg * 16;
-        uint32_t a[4];
-        ldsm_x4(a, smem_u32(kp + off));
-        mma_16816(s, a, qb[k][0], qb[k][1]);
-      }
-      const bool v0 = m0t + g < ntok, v1 = m0t + g + 8 < ntok;
-      s[0] = v0 ? s[0] * scale_log2_ : -INFINITY;
-      s[1] = v0 ? s[1] * scale_log2_ : -INFINITY;
-      s[2] = v1 ? s[2] * scale_log2_ : -INFINITY;
-      s[3] = v1 ? s[3] * scale_log2_ : -INFINITY;
-      float x0 = fmaxf(s[0], s[2]), x1 = fmaxf(s[1], s[3]);
+    for (int u = 0; u < NT; ++u) {
+      const int tk = m0 + 16 * u + (lane & 15);
+      const unsigned char *kr =
+          TL ? kp + (h * p.vbs + tk) * 128 : kp + tk * p.row_pitch + col_bytes + ck;
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int mask = 4; mask < 32; mask <<= 1) {
-        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, mask));
-        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, mask));
-      }
-      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-      const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
-      m0 = n0;
-      m1 = n1;
-      const float p0 = exp2f(s[0] - n0), p1 = exp2f(s[1] - n1);
-      const float p2 = exp2f(s[2] - n0), p3 = exp2f(s[3] - n1);
-      l0 = l0 * a0 + p0 + p2;
-      l1 = l1 * a1 + p1 + p3;
-      if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
-#pragma unroll
-        for (int k = 0; k < KS; ++k) {
-          o[k][0] *= a0;
-          o[k][1] *= a1;
-          o[k][2] *= a0;
-          o[k][3] *= a1;
+      for (int k = 0; k < KS; k += 2) {
+        uint32_t a[4], b[4];
+        if (TL) {
+          ldsm_x4(a, smem_u32(kr + (k >> 2) * p.box_bytes + ((((2 * k) & 7) << 4) ^ xk)));
+          ldsm_x4(b, smem_u32(kr + ((k + 1) >> 2) * p.box_bytes +
+                              ((((2 * k + 2) & 7) << 4) ^ xk)));
+        } else {
+          ldsm_x4(a, smem_u32(kr + k * 32));
+          ldsm_x4(b, smem_u32(kr + (k + 1) * 32));
         }
+        mma_16816(sa, a, qb[k][0], qb[k][1]);
+        mma_16816(sb, b, qb[k + 1][0], qb[k + 1][1]);
       }
-      // P^T (16 tokens x 8 heads) as the B operand: transpose the two 8x8 tiles.
-      const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
-      const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
-      // V rows past ntok may hold anything (other tokens, never-written
-      // shared memory): their P is 0, and their V elements are zeroed below
-      // so that 0 * NaN cannot occur.
-      const bool partial = m0t + 16 > ntok;
-      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-      if (partial) {
-        mlo = (m0t + 2 * t < ntok ? 0x0000ffffu : 0u) | (m0t + 2 * t + 1 < ntok ? 0xffff0000u : 0u);
-        mhi = (m0t + 2 * t + 8 < ntok ? 0x0000ffffu : 0u) |
-              (m0t + 2 * t + 9 < ntok ? 0xffff0000u : 0u);
-      }
-      const int mi = lane >> 3, rr = lane & 7;
-      const int tv = m0t + rr + ((mi >> 1) << 3), hv = mi & 1;
-      const int rowv = tile ? (h * p.vbs + tv) * 128 : tv * p.row_pitch + col_bytes;
+      const int r0 = m0 + 16 * u + g;
+      const bool v0 = r0 < ntok, v1 = r0 + 8 < ntok;
+      s[u][0] = v0 ? (sa[0] + sb[0]) * scale_log2_ : -INFINITY;
+      s[u][1] = v0 ? (sa[1] + sb[1]) * scale_log2_ : -INFINITY;
+      s[u][2] = v1 ? (sa[2] + sb[2]) * scale_log2_ : -INFINITY;
+      s[u][3] = v1 ? (sa[3] + sb[3]) * scale_log2_ : -INFINITY;
+    }
+    float x0 = -INFINITY, x1 = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      x0 = fmaxf(x0, fmaxf(s[u][0], s[u][2]));
+      x1 = fmaxf(x1, fmaxf(s[u][1], s[u][3]));
+    }
+#pragma unroll
+    for (int mask = 4; mask < 32; mask <<= 1) {
+      x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, mask));
+      x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, mask));
+    }
+    const float n0 = fmaxf(m0_, x0), n1 = fmaxf(m1_, x1);
+    const float a0 = ex2(m0_ - n0), a1 = ex2(m1_ - n1);
+    m0_ = n0;
+    m1_ = n1;
+    uint32_t pb[NT][2];
+    float add0 = 0.f, add1 = 0.f;
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      const float p0 = ex2(s[u][0] - n0), p1 = ex2(s[u][1] - n1);
+      const float p2 = ex2(s[u][2] - n0), p3 = ex2(s[u][3] - n1);
+      add0 += p0 + p2;
+      add1 += p1 + p3;
+      // P^T (16 tokens x 8 heads) as the B operand: transpose the two 8x8 tiles
+      pb[u][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+      pb[u][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+    }
+    l0 = l0 * a0 + add0;
+    l1 = l1 * a1 + add1;
+    if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
 #pragma unroll
       for (int k = 0; k < KS; ++k) {
-        const int cg = k * 2 + hv;
-        const int off = tile ? (cg >> 3) * p.box_bytes + rowv + (((cg & 7) ^ (tv & 7)) << 4)
-                             : rowv + cg * 16;
+        o[k][0] *= a0;
+        o[k][1] *= a1;
+        o[k][2] *= a0;
+        o[k][3] *= a1;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      // V rows past ntok may hold anything (other tokens, never-written
+      // shared memory): their P is 0 and their V elements are zeroed here so
+      // that 0 * NaN cannot occur.
+      const int base = m0 + 16 * u;
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (base + 16 > ntok) {
+        mlo = (base + 2 * t < ntok ? 0x0000ffffu : 0u) | (base + 2 * t + 1 < ntok ? 0xffff0000u : 0u);
+        mhi = (base + 2 * t + 8 < ntok ? 0x0000ffffu : 0u) |
+              (base + 2 * t + 9 < ntok ? 0xffff0000u : 0u);
+      }
+      const int tv = base + (lane & 7) + ((mi >> 1) << 3);
+      const unsigned char *vr =
+          TL ? vp + (h * p.vbs + tv) * 128 : vp + tv * p.row_pitch + col_bytes + cv;
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
         uint32_t a[4];
-        ldsm_x4_trans(a, smem_u32(vp + off));
+        if (TL)
+          ldsm_x4_trans(a, smem_u32(vr + (k >> 2) * p.box_bytes + ((((2 * k) & 7) << 4) ^ xv)));
+        else
+          ldsm_x4_trans(a, smem_u32(vr + k * 32));
         a[0] &= mlo;
         a[1] &= mlo;
         a[2] &= mhi;
         a[3] &= mhi;
-        mma_16816(o[k], a, b0, b1);
+        mma_16816(o[k], a, pb[u][0], pb[u][1]);
       }
     }
+  }
+
+  template <bool TL>
+  __device__ __forceinline__ void page_t(const unsigned char *kp, const unsigned char *vp,
+                                         int ntok, const Params &p, int h, int col_bytes,
+                                         int lane) {
+    int m0 = 0;
+    for (; m0 + 16 < ntok; m0 += 32) tiles<2, TL>(kp, vp, m0, ntok, p, h, col_bytes, lane);
+    if (m0 < ntok) tiles<1, TL>(kp, vp, m0, ntok, p, h, col_bytes, lane);
+  }
+
+  __device__ __forceinline__ void page(const unsigned char *kp, const unsigned char *vp,
+                                       int ntok, const Params &p, int h, int col_bytes,
+                                       int lane) {
+    if (p.tile)
+      page_t<true>(kp, vp, ntok, p, h, col_bytes, lane);
+    else
+      page_t<false>(kp, vp, ntok, p, h, col_bytes, lane);
   }
 
   // End of a segment: write out[...] directly or a partial + merge.
   template <typename Tout>
   __device__ __forceinline__ void flush(const Params &p, const PageDesc &d, int hq0, int nh,
-                                        int c, int lane, int32_t *counter) {
+                                        int c, int lane) {
     const int g = lane >> 2, t = lane & 3;
     float L0 = l0, L1 = l1;
 #pragma unroll
@@ -364,11 +431,11 @@ struct MmaConsumer {
     const int64_t prow = ((int64_t)c * 2 + (d.slot_bits & 1)) * p.num_q_heads + hq0;
     if (g == 0) {
       if (h0 < nh) {
-        p.part_ml[(prow + h0) * 2 + 0] = m0;
+        p.part_ml[(prow + h0) * 2 + 0] = m0_;
         p.part_ml[(prow + h0) * 2 + 1] = seg_bad ? -1.f : L0;
       }
       if (h1 < nh) {
-        p.part_ml[(prow + h1) * 2 + 0] = m1;
+        p.part_ml[(prow + h1) * 2 + 0] = m1_;
         p.part_ml[(prow + h1) * 2 + 1] = seg_bad ? -1.f : L1;
       }
     }
@@ -387,73 +454,7 @@ struct MmaConsumer {
         }
       }
     }
-    __threadfence();
-    __syncwarp();
-    int32_t old = 0;
-    if (lane == 0) old = atomicAdd(counter, 1);
-    old = __shfl_sync(0xffffffffu, old, 0);
-    if (old != d.n_contrib - 1) return;
-    // Last contributor: merge every CTA's partial of this sequence / slice.
-    __threadfence();
-    const int first_slot = (d.slot_bits >> 1) & 1;
-    float M0 = -INFINITY, M1 = -INFINITY, W0 = 0.f, W1 = 0.f;
-    bool any_bad = false;
-    for (int x = 0; x < d.n_contrib; ++x) {
-      const int64_t r =
-          ((int64_t)(d.c_first + x) * 2 + (x == 0 ? first_slot : 0)) * p.num_q_heads + hq0;
-      if (h0 < nh) {
-        any_bad |= __ldcg(p.part_ml + (r + h0) * 2 + 1) < 0.f;
-        M0 = fmaxf(M0, __ldcg(p.part_ml + (r + h0) * 2 + 0));
-      }
-      if (h1 < nh) {
-        any_bad |= __ldcg(p.part_ml + (r + h1) * 2 + 1) < 0.f;
-        M1 = fmaxf(M1, __ldcg(p.part_ml + (r + h1) * 2 + 0));
-      }
-    }
-    float acc[KS][4];
-#pragma unroll
-    for (int k = 0; k < KS; ++k)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
-    for (int x = 0; x < d.n_contrib; ++x) {
-      const int64_t r =
-          ((int64_t)(d.c_first + x) * 2 + (x == 0 ? first_slot : 0)) * p.num_q_heads + hq0;
-      float w0 = 0.f, w1 = 0.f;
-      if (h0 < nh)
-        w0 = __ldcg(p.part_ml + (r + h0) * 2 + 1) *
-             exp2f(__ldcg(p.part_ml + (r + h0) * 2 + 0) - M0);
-      if (h1 < nh)
-        w1 = __ldcg(p.part_ml + (r + h1) * 2 + 1) *
-             exp2f(__ldcg(p.part_ml + (r + h1) * 2 + 0) - M1);
-      W0 += w0;
-      W1 += w1;
-#pragma unroll
-      for (int k = 0; k < KS; ++k) {
-        const int dd = k * 16 + g;
-        if (h0 < nh) {
-          acc[k][0] += w0 * __ldcg(p.part_o + (r + h0) * D + dd);
-          acc[k][2] += w0 * __ldcg(p.part_o + (r + h0) * D + dd + 8);
-        }
-        if (h1 < nh) {
-          acc[k][1] += w1 * __ldcg(p.part_o + (r + h1) * D + dd);
-          acc[k][3] += w1 * __ldcg(p.part_o + (r + h1) * D + dd + 8);
-        }
-      }
-    }
-    const float i0 = 1.f / W0, i1 = 1.f / W1;
-#pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      const int dd = k * 16 + g;
-      if (h0 < nh) {
-        Elem<Tout>::store1(p.out, (orow + h0) * D + dd, any_bad ? 0.f : acc[k][0] * i0);
-        Elem<Tout>::store1(p.out, (orow + h0) * D + dd + 8, any_bad ? 0.f : acc[k][2] * i0);
-      }
-      if (h1 < nh) {
-        Elem<Tout>::store1(p.out, (orow + h1) * D + dd, any_bad ? 0.f : acc[k][1] * i1);
-        Elem<Tout>::store1(p.out, (orow + h1) * D + dd + 8, any_bad ? 0.f : acc[k][3] * i1);
-      }
-    }
-    if (lane == 0) atomicExch(counter, 0);
+    // merged later by the merge kernel
   }
 };
 
@@ -601,7 +602,7 @@ struct FmaConsumer {
   }
 
   __device__ __forceinline__ void flush(const Params &p, const PageDesc &d, int hq0, int c,
-                                        int lane, int32_t *counter) {
+                                        int lane) {
     const int tg = lane / LPT, j = lane % LPT;
     float ac[G][EPV];
 #pragma unroll
@@ -643,58 +644,76 @@ struct FmaConsumer {
         for (int e = 0; e < EPV; ++e)
           p.part_o[(prow + g) * D + j * EPV + e] = seg_bad ? 0.f : ac[g][e] / lg[g];
     }
-    __threadfence();
-    __syncwarp();
-    int32_t old = 0;
-    if (lane == 0) old = atomicAdd(counter, 1);
-    old = __shfl_sync(0xffffffffu, old, 0);
-    if (old != d.n_contrib - 1) return;
-    __threadfence();
-    const int first_slot = (d.slot_bits >> 1) & 1;
-    float M[G], W[G];
-    bool any_bad = false;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      M[g] = -INFINITY;
-      W[g] = 0.f;
+    // merged later by the merge kernel
+  }
+};
+
+// ===========================================================================
+// Walk over a CTA's virtual pages in stream order (all lanes of the producer
+// warp in lock step).  Context lengths and block-table entries are fetched 32
+// at a time into lane registers; the current page's values are shuffled out.
+// ===========================================================================
+struct PageWalker {
+  int32_t s, vlb, ctx_s, pages_s;
+  int32_t cw, cw_ctx;             // context-length window: lane l holds sequence cw + l
+  int32_t tw_seq, tw_lb, tw_val;  // table window: lane l holds entry tw_lb + l of tw_seq
+  int64_t P_s, cursor;
+
+  __device__ __forceinline__ void init(const Params &p, int32_t s0, int32_t vlb0, int64_t P0,
+                                       int64_t cur0, int lane) {
+    s = s0;
+    vlb = vlb0;
+    P_s = P0;
+    cursor = cur0;
+    cw = s0;
+    cw_ctx = (cw + lane < p.batch) ? p.context_lens[cw + lane] : 0;
+    ctx_s = __shfl_sync(0xffffffffu, cw_ctx, 0);
+    pages_s = vpages_of(ctx_s, p);
+    tw_seq = -1;
+    tw_lb = 0;
+    tw_val = -1;
+  }
+  // Physical block of the current page.
+  __device__ __forceinline__ int32_t block(const Params &p, int lane) {
+    const int32_t lb = vlb >> p.log2_vpp;
+    if (s != tw_seq || lb >= tw_lb + 32) {
+      tw_seq = s;
+      tw_lb = lb;
+      const int32_t e = lb + lane;
+      tw_val = (e < p.max_blocks) ? p.block_tables[(int64_t)s * p.max_blocks + e] : -1;
     }
-    for (int x = 0; x < d.n_contrib; ++x) {
-      const int64_t r =
-          ((int64_t)(d.c_first + x) * 2 + (x == 0 ? first_slot : 0)) * p.num_q_heads + hq0;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        any_bad |= __ldcg(p.part_ml + (r + g) * 2 + 1) < 0.f;
-        M[g] = fmaxf(M[g], __ldcg(p.part_ml + (r + g) * 2 + 0));
-      }
-    }
-    float O[G][EPV];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < EPV; ++e) O[g][e] = 0.f;
-    for (int x = 0; x < d.n_contrib; ++x) {
-      const int64_t r =
-          ((int64_t)(d.c_first + x) * 2 + (x == 0 ? first_slot : 0)) * p.num_q_heads + hq0;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float w = __ldcg(p.part_ml + (r + g) * 2 + 1) *
-                        exp2f(__ldcg(p.part_ml + (r + g) * 2 + 0) - M[g]);
-        W[g] += w;
-        if (tg == 0) {
-#pragma unroll
-          for (int e = 0; e < EPV; ++e)
-            O[g][e] += w * __ldcg(p.part_o + (r + g) * D + j * EPV + e);
+    return __shfl_sync(0xffffffffu, tw_val, lb - tw_lb);
+  }
+  __device__ __forceinline__ int32_t ntok(const Params &p) const {
+    return min(p.vbs, ctx_s - vlb * p.vbs);
+  }
+  // Next page of the stream (skips sequences without pages).
+  __device__ __forceinline__ void advance(const Params &p, int64_t end, int lane) {
+    ++cursor;
+    ++vlb;
+    if (vlb == pages_s && cursor < end) {
+      int32_t nxt = s + 1;
+      for (;;) {
+        if (nxt >= cw + 32) {
+          cw = nxt;
+          cw_ctx = (cw + lane < p.batch) ? p.context_lens[cw + lane] : 0;
         }
+        const bool has =
+            (cw + lane >= nxt) && (cw + lane < p.batch) && vpages_of(cw_ctx, p) > 0;
+        const uint32_t m = __ballot_sync(0xffffffffu, has);
+        if (m) {
+          const int l = __ffs(m) - 1;
+          nxt = cw + l;
+          ctx_s = __shfl_sync(0xffffffffu, cw_ctx, l);
+          break;
+        }
+        nxt = cw + 32;
       }
+      P_s += pages_s;
+      s = nxt;
+      vlb = 0;
+      pages_s = vpages_of(ctx_s, p);
     }
-    if (tg == 0) {
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < EPV; ++e)
-          Elem<T>::store1(p.out, (orow + g) * D + j * EPV + e, any_bad ? 0.f : O[g][e] / W[g]);
-    }
-    if (lane == 0) atomicExch(counter, 0);
   }
 };
 
@@ -725,6 +744,12 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
+  // Launched with programmatic stream serialisation: this CTA may start
+  // while the previous kernel of the stream still runs.  Nothing it reads or
+  // writes is touched before that kernel has finished and flushed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the merge kernel that follows may be scheduled now; it waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;");
 
   if (tid == 0) {
     for (int i = 0; i < p.stages; ++i) {
@@ -772,17 +797,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     const int n_stages = (int)((end - start + p.pps - 1) / p.pps);
     if (warp == 0) {
       // ===================== producer =====================
-      int32_t s = sh.s_begin;
-      int32_t vlb = sh.vlb_begin;
-      int64_t P_s = sh.P_begin;
-      // context-length window: lane l holds sequence cw + l
-      int32_t cw = s;
-      int32_t cw_ctx = (cw + lane < p.batch) ? p.context_lens[cw + lane] : 0;
-      int32_t ctx_s = __shfl_sync(0xffffffffu, cw_ctx, 0);
-      int32_t pages_s = vpages_of(ctx_s, p);
-      // block-table window: lane l holds entry tw_lb + l of sequence tw_seq
-      int32_t tw_seq = -1, tw_lb = 0, tw_val = -1;
-      int64_t cursor = start;
+      PageWalker wk;
+      wk.init(p, sh.s_begin, sh.vlb_begin, sh.P_begin, start, lane);
       bool ok = true;
       int issued = 0;
       for (int i = 0; i < n_stages && ok; ++i) {
@@ -792,38 +808,37 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                           mbar_wait(&sh.empty[slot], ((i / p.stages) - 1) & 1, &sh.abort_flag));
           if (!ok) break;
         }
-        const int npg = (int)min((int64_t)p.pps, end - cursor);
+        const int npg = (int)min((int64_t)p.pps, end - wk.cursor);
         uint32_t bytes = 0;
         for (int k = 0; k < npg; ++k) {
-          const int32_t lb = vlb >> p.log2_vpp;
-          if (s != tw_seq || lb >= tw_lb + 32) {
-            tw_seq = s;
-            tw_lb = lb;
-            const int32_t e = lb + lane;
-            tw_val = (e < p.max_blocks) ? p.block_tables[(int64_t)s * p.max_blocks + e] : -1;
-          }
-          const int32_t pb = __shfl_sync(0xffffffffu, tw_val, lb - tw_lb);
-          const int32_t ntok = min(p.vbs, ctx_s - vlb * p.vbs);
-          const bool first = (vlb == 0) || (cursor == start);
-          const bool last = (vlb == pages_s - 1) || (cursor == end - 1);
+          const int32_t pb = wk.block(p, lane);
+          const int32_t ntok = wk.ntok(p);
+          const bool first = (wk.vlb == 0) || (wk.cursor == start);
+          const bool last = (wk.vlb == wk.pages_s - 1) || (wk.cursor == end - 1);
           const bool bad = pb < 0 || pb >= p.num_blocks;
           if (lane == 0) {
             PageDesc d;
-            d.seq = s;
+            d.seq = wk.s;
             d.ntok = ntok;
             d.flags = (first ? kFirst : 0) | (last ? kLast : 0) | (bad ? kBad : 0);
             d.pb = pb;
-            d.toff = (vlb & ((1 << p.log2_vpp) - 1)) * p.vbs;
+            d.toff = (wk.vlb & ((1 << p.log2_vpp) - 1)) * p.vbs;
             d.n_contrib = 1;
             d.c_first = c;
             d.slot_bits = 0;
             if (last) {
-              const int32_t c_first = owner_of(P_s, Tp, g_eff);
-              const int32_t c_last = owner_of(P_s + pages_s - 1, Tp, g_eff);
+              const int32_t c_first = owner_of(wk.P_s, Tp, g_eff);
+              const int32_t c_last = owner_of(wk.P_s + wk.pages_s - 1, Tp, g_eff);
               d.n_contrib = c_last - c_first + 1;
               d.c_first = c_first;
               const int64_t st_first = (int64_t)c_first * Tp / g_eff;
-              d.slot_bits = ((start < P_s) ? 1 : 0) | ((st_first < P_s) ? 2 : 0);
+              d.slot_bits = ((start < wk.P_s) ? 1 : 0) | ((st_first < wk.P_s) ? 2 : 0);
+              if (c == c_last) {
+                // the owner of the sequence's last page tells the merge kernel
+                // where the partials are (or that there is nothing to merge)
+                reinterpret_cast<int4 *>(p.seq_merge)[wk.s] =
+                    make_int4(c_first, d.n_contrib, (st_first < wk.P_s) ? 1 : 0, 0);
+              }
             }
             descs[slot * kMaxPPS + k] = d;
           }
@@ -831,33 +846,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             bytes += p.tile ? 2u * (uint32_t)p.n_dhalf * (uint32_t)p.box_bytes
                             : 2u * (uint32_t)ntok * (uint32_t)p.row_bytes;
           if (first) bytes += (uint32_t)p.q_bytes;
-          // advance the cursor
-          ++cursor;
-          ++vlb;
-          if (vlb == pages_s && cursor < end) {
-            // next sequence with at least one page
-            int32_t nxt = s + 1;
-            for (;;) {
-              if (nxt >= cw + 32) {
-                cw = nxt;
-                cw_ctx = (cw + lane < p.batch) ? p.context_lens[cw + lane] : 0;
-              }
-              const bool has = (cw + lane >= nxt) && (cw + lane < p.batch) &&
-                               vpages_of(cw_ctx, p) > 0;
-              const uint32_t m = __ballot_sync(0xffffffffu, has);
-              if (m) {
-                const int l = __ffs(m) - 1;
-                nxt = cw + l;
-                ctx_s = __shfl_sync(0xffffffffu, cw_ctx, l);
-                break;
-              }
-              nxt = cw + 32;
-            }
-            P_s += pages_s;
-            s = nxt;
-            vlb = 0;
-            pages_s = vpages_of(ctx_s, p);
-          }
+          wk.advance(p, end, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_expect_tx(&sh.full[slot], bytes);
@@ -941,6 +930,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         const unsigned char *qst = st + (size_t)2 * p.pps * p.vpage_stride;
         const int npg = (int)min((int64_t)p.pps, end - cursor);
         cursor += npg;
+        bool released = false;
         for (int k = 0; k < npg; ++k) {
           const PageDesc d = descs[slot * kMaxPPS + k];
           if (d.flags & kFirst) {
@@ -964,21 +954,26 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             }
           }
           if (d.flags & kLast) {
-            // one counter per (sequence, query-head slice of one warp)
-            const int slices = p.num_q_heads / p.heads_per_warp;
-            int32_t *counter =
-                p.counters + (int64_t)d.seq * slices + hq0 / p.heads_per_warp;
+            // The flush works on registers only: hand the stage back first
+            // when this was its last page, so the producer is not held up.
+            if (k == npg - 1) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh.empty[slot]);
+              released = true;
+            }
             if constexpr (kMma) {
-              cs.template flush<T>(p, d, hq0, p.heads_per_warp, c, lane, counter);
+              cs.template flush<T>(p, d, hq0, p.heads_per_warp, c, lane);
             } else {
-              cs.flush(p, d, hq0, c, lane, counter);
+              cs.flush(p, d, hq0, c, lane);
             }
             if (cs.seg_bad && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
             cs.reset();
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[slot]);
+        if (!released) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.empty[slot]);
+        }
       }
     }
   }
@@ -988,8 +983,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   for (int s = c; s < p.batch; s += p.grid) {
     const int32_t ctx = p.context_lens[s];
     if (vpages_of(ctx, p) > 0) continue;
-    if ((ctx < 0 || (int64_t)ctx > (int64_t)p.max_blocks * p.block_size) && tid == 0)
-      set_error(p.err_word, PA_DEVERR_CONTEXT_LEN);
+    if (tid == 0) {
+      reinterpret_cast<int4 *>(p.seq_merge)[s] = make_int4(0, 0, 0, 0);
+      if (ctx < 0 || (int64_t)ctx > (int64_t)p.max_blocks * p.block_size)
+        set_error(p.err_word, PA_DEVERR_CONTEXT_LEN);
+    }
     const int64_t n = (int64_t)p.num_q_heads * D;
     for (int64_t x = tid; x < n; x += blockDim.x) Elem<T>::store1(p.out, (int64_t)s * n + x, 0.f);
   }
@@ -1012,8 +1010,105 @@ cudaError_t launch_one(const Params &p, size_t smem, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured[dev] = smem;
   }
-  kern<<<p.grid, (NCW + 1) * 32, smem, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3((NCW + 1) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// ---------------------------------------------------------------------------
+// Merge kernel: one warp per (sequence, query-head slice of a consumer warp).
+// Runs after the decode kernel (programmatic launch: it may be scheduled
+// early and waits for the decode grid), when the memory system is quiet.
+// ---------------------------------------------------------------------------
+template <typename Tout, int D>
+__global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Params p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int slices = p.num_q_heads / p.heads_per_warp;
+  const int seq = blockIdx.x / slices;
+  const int hq0 = (blockIdx.x % slices) * p.heads_per_warp;
+  const int4 md = __ldcg(reinterpret_cast<const int4 *>(p.seq_merge) + seq);
+  const int n = md.y;
+  if (n <= 1) return;  // empty, or written directly by its only CTA
+  const int first_slot = md.z;
+  const int64_t orow = (int64_t)seq * p.num_q_heads + hq0;
+  // thread -> 4 consecutive outputs (head, d .. d+3) of this slice
+  for (int f = threadIdx.x * 4; f < p.heads_per_warp * D; f += blockDim.x * 4) {
+    const int h = f / D, d0 = f % D;
+    float M = -INFINITY, W = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    bool bad = false;
+    // contributors in batches of 8: all loads of a batch are in flight together
+    for (int x0 = 0; x0 < n; x0 += 8) {
+      float2 ml[8];
+      float4 o4[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int x = x0 + j;
+        if (x < n) {
+          const int64_t r = ((int64_t)(md.x + x) * 2 + (x == 0 ? first_slot : 0)) *
+                                p.num_q_heads + hq0 + h;
+          ml[j] = __ldcg(reinterpret_cast<const float2 *>(p.part_ml) + r);
+          o4[j] = __ldcg(reinterpret_cast<const float4 *>(p.part_o + r * D + d0));
+        } else {
+          ml[j] = make_float2(-INFINITY, 0.f);
+          o4[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float mb = M;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        bad |= ml[j].y < 0.f;
+        if (ml[j].y > 0.f) mb = fmaxf(mb, ml[j].x);
+      }
+      const float keep = (M == -INFINITY) ? 0.f : ex2(M - mb);
+      W *= keep;
+      acc.x *= keep;
+      acc.y *= keep;
+      acc.z *= keep;
+      acc.w *= keep;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float w = (ml[j].y > 0.f) ? ml[j].y * ex2(ml[j].x - mb) : 0.f;
+        W += w;
+        acc.x += w * o4[j].x;
+        acc.y += w * o4[j].y;
+        acc.z += w * o4[j].z;
+        acc.w += w * o4[j].w;
+      }
+      M = mb;
+    }
+    const float inv = 1.f / W;
+    const int64_t e = (orow + h) * D + d0;
+    Elem<Tout>::store1(p.out, e + 0, bad ? 0.f : acc.x * inv);
+    Elem<Tout>::store1(p.out, e + 1, bad ? 0.f : acc.y * inv);
+    Elem<Tout>::store1(p.out, e + 2, bad ? 0.f : acc.z * inv);
+    Elem<Tout>::store1(p.out, e + 3, bad ? 0.f : acc.w * inv);
+  }
+}
+
+template <typename Tout, int D>
+cudaError_t launch_merge_one(const Params &p, cudaStream_t stream) {
+  const int64_t blocks = (int64_t)p.batch * (p.num_q_heads / p.heads_per_warp);
+  if (blocks == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_kernel<Tout, D>, p);
 }
 
 }  // namespace stream

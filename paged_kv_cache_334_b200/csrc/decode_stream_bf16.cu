@@ -23,5 +23,11 @@ cudaError_t launch_bf16(const Params &p, int head_dim, int group, int hkv, size_
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_merge_bf16(const Params &p, int head_dim, cudaStream_t stream) {
+  if (head_dim == 64) return launch_merge_one<__nv_bfloat16, 64>(p, stream);
+  if (head_dim == 128) return launch_merge_one<__nv_bfloat16, 128>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace stream
 }  // namespace pa

@@ -31,5 +31,11 @@ cudaError_t launch_f32(const Params &p, int head_dim, int group, int hkv, size_t
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_merge_f32(const Params &p, int head_dim, cudaStream_t stream) {
+  if (head_dim == 64) return launch_merge_one<float, 64>(p, stream);
+  if (head_dim == 128) return launch_merge_one<float, 128>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace stream
 }  // namespace pa

@@ -52,7 +52,7 @@ struct Params {
   const int32_t *context_lens;
   float *part_ml;     // [kMaxGrid * 2][Hq][2]: (max in log2 units, normaliser)
   float *part_o;      // [kMaxGrid * 2][Hq][D]: normalised partial output
-  int32_t *counters;  // [batch * Hkv]
+  int32_t *seq_merge;  // [batch][4]: first contributing CTA, contributors, slot of the first
   int32_t *err_word;
   int32_t num_blocks, block_size, num_kv_heads, num_q_heads, max_blocks, batch;
   int32_t vbs, log2_vbs, log2_vpp;  // virtual page tokens; log2 of pages per block
@@ -73,6 +73,9 @@ struct Params {
 
 cudaError_t launch_bf16(const Params &p, int head_dim, int group, int hkv, size_t smem,
                         cudaStream_t stream);
+// Second kernel of pa_decode: merge the partials of sequences split across CTAs.
+cudaError_t launch_merge_bf16(const Params &p, int head_dim, cudaStream_t stream);
+cudaError_t launch_merge_f32(const Params &p, int head_dim, cudaStream_t stream);
 cudaError_t launch_f32(const Params &p, int head_dim, int group, int hkv, size_t smem,
                        cudaStream_t stream);
 

@@ -20,6 +20,10 @@ write_kv_kernel(uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache,
                 const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
                 const int64_t *__restrict__ slot_mapping, int64_t num_slots,
                 int64_t row_vecs, int32_t *err_word) {
+  // The decode kernel that usually follows waits for this grid to finish
+  // (griddepcontrol.wait) before it reads anything; letting it launch now
+  // overlaps its start-up with this copy.
+  asm volatile("griddepcontrol.launch_dependents;");
   const int64_t token = blockIdx.x;
   const int64_t slot = slot_mapping[token];
   if (slot < 0) return;

@@ -231,22 +231,23 @@ def test_block_permutation_gives_bit_identical_output():
     assert torch.equal(out1.view(torch.uint16), out2.view(torch.uint16))
 
 
-def test_repeatable_and_workspace_left_zero():
+def test_repeatable_with_a_reused_workspace():
+    """One workspace, zero-filled once, serves repeated calls: identical bits
+    every time, whatever the previous call left in it."""
     w = wl.make_workload("mixed_bf16", seed=2, batch=16)
     d = upload(w)
     ws = pa.decode_workspace(d["key_cache"], w.batch, w.num_q_heads, w.max_blocks)
     ws.zero_()
     out1 = gpu_write_and_decode(w, d)
-    out2 = torch.empty_like(out1)
-    pa.pa_decode(out2, d["q"], d["key_cache"], d["value_cache"], d["block_tables"],
-                 d["context_lens"], workspace=ws)
+    outs = []
+    for _ in range(3):
+        o = torch.empty_like(out1)
+        pa.pa_decode(o, d["q"], d["key_cache"], d["value_cache"], d["block_tables"],
+                     d["context_lens"], workspace=ws)
+        outs.append(o)
     torch.cuda.synchronize()
-    assert torch.equal(out1.view(torch.uint16), out2.view(torch.uint16))
-    # the counters (the last 256-byte-rounded slice of the workspace, one
-    # int32 per sequence x KV head here) are back to zero
-    ncnt = w.batch * w.num_kv_heads
-    tail = ws[-((ncnt * 4 + 255) // 256 * 256):]
-    assert int(tail.count_nonzero().item()) == 0
+    for o in outs:
+        assert torch.equal(out1.view(torch.uint16), o.view(torch.uint16))
 
 
 def test_non_default_stream():
