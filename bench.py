@@ -2,8 +2,10 @@
 """Benchmark of one paged decode-attention step on B200.
 
 A step is one pass of the hot path over one batch: the cache write of every
-sequence's newest token (pa_write_kv_cache via slot_mapping) followed by the
-fused paged decode (pa_decode), both through the C ABI.  The default workload
+sequence's newest token via slot_mapping followed by the fused paged decode,
+through the C ABI -- by default as one pa_forward_decode call (the write
+happens inside the decode kernel), with ``--step separate`` as
+pa_write_kv_cache followed by pa_decode.  The default workload
 is the bf16 GQA decode batch (batch 32, 32 query / 8 KV heads, head_dim 128,
 block_size 16, context lengths uniform in [128, 2048]); other workloads are
 selectable with --workload.
@@ -14,8 +16,8 @@ tables, context lengths, q, out and the new K/V rows) in GB/s, summed over
 ranks and divided by the slowest rank's time; each timed step is preceded by
 an L2 flush outside its CUDA-event pair.  ``e2e`` is the same metric with the
 per-step inputs copied from pinned host memory and the output read back
-inside the timed region.  ``roofline`` reports the decode kernel alone
-against the measured HBM copy bandwidth; ``cpu_baseline`` times the fp64 CPU
+inside the timed region.  ``roofline`` reports the decode call (the whole
+step when fused) against the measured HBM copy bandwidth; ``cpu_baseline`` times the fp64 CPU
 oracle on the host cores (rank 0, one GPU only).
 
 Multi-GPU (torchrun, one process per GPU): every rank decodes its own
@@ -68,6 +70,9 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--step", choices=("fused", "separate"), default="fused",
+                    help="fused: one pa_forward_decode call per step (cache write inside the "
+                         "decode kernel); separate: pa_write_kv_cache then pa_decode")
     return ap.parse_args(argv)
 
 
@@ -301,7 +306,9 @@ def workload_config(w, args):
         "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
         "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
         "context_tokens": int(w.context_lens.sum()), "seed": args.seed,
-        "step": "pa_write_kv_cache(newest token of every sequence) + pa_decode",
+        "step": ("pa_forward_decode (newest token of every sequence stored inside the decode "
+                 "kernel, then decode)" if args.step == "fused" else
+                 "pa_write_kv_cache(newest token of every sequence) + pa_decode"),
         "l2": "flushed before every timed step (zero-fill then read of 2x L2, outside the events)",
         "parallelism": f"replicas: one independent batch per GPU x{args.gpus}",
     }
@@ -374,7 +381,10 @@ def run_ours(args):
     flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     flush_f32 = flush_buf.view(torch.float32)
     flush_sink = torch.empty((), dtype=torch.float32, device=dev)
-    launches_per_step = 2 if has_new else 1
+    fused = has_new and args.step == "fused"
+    # libpa kernels per step: the persistent decode kernel and its merge
+    # kernel, plus the write kernel when the write is a separate call
+    launches_per_step = 2 + (1 if has_new and not fused else 0)
 
     def flush_l2():
         # Write a buffer twice the L2 size, then read it back: the step's
@@ -384,12 +394,16 @@ def run_ours(args):
         torch.amax(flush_f32, out=flush_sink)
 
     def write():
-        if has_new:
+        if has_new and not fused:
             pa.pa_write_kv_cache(kc, vc, kn, vn, sm, err_word=err, stream=stream)
 
     def decode():
-        pa.pa_decode(out, q, kc, vc, bt, cl, scale=scale, workspace=ws, err_word=err,
-                     stream=stream)
+        if fused:
+            pa.pa_forward_decode(out, q, kc, vc, kn, vn, sm, bt, cl, scale=scale, workspace=ws,
+                                 err_word=err, stream=stream)
+        else:
+            pa.pa_decode(out, q, kc, vc, bt, cl, scale=scale, workspace=ws, err_word=err,
+                         stream=stream)
 
     for _ in range(max(args.warmup, 3)):
         flush_l2()
@@ -410,8 +424,9 @@ def run_ours(args):
     for k in range(K):
         flush_l2()
         ev[k][0].record(stream)
-        write()
-        ev[k][1].record(stream)
+        if not fused:
+            write()
+            ev[k][1].record(stream)
         decode()
         ev[k][2].record(stream)
     torch.cuda.synchronize(dev)
@@ -420,7 +435,8 @@ def run_ours(args):
         dist.barrier()
     clk = clocks.stop()
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    # the timed kernel call: pa_forward_decode (the whole step) or pa_decode
+    dec_ms = step_ms if fused else [e[1].elapsed_time(e[2]) for e in ev]
     t_step = statistics.mean(step_ms)
     t_dec = statistics.mean(dec_ms)
 
@@ -459,7 +475,7 @@ def run_ours(args):
         raise RuntimeError(f"device error word {int(err.item())}")
 
     step_bytes = wl.roofline_bytes(w)
-    dec_bytes = wl.roofline_bytes(w, include_write=False)
+    dec_bytes = step_bytes if fused else wl.roofline_bytes(w, include_write=False)
     t_step_max = reduce_scalar(t_step, "max", dist, dev)
     bytes_all = reduce_scalar(step_bytes, "sum", dist, dev)
     seqs_all = reduce_scalar(w.batch, "sum", dist, dev)
@@ -500,7 +516,8 @@ def run_ours(args):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
-            "kernel": "pa_decode", "algorithmic_bytes_per_launch": dec_bytes,
+            "kernel": "pa_forward_decode" if fused else "pa_decode",
+            "algorithmic_bytes_per_launch": dec_bytes,
             "launch_us": t_dec * 1e3, "peak_source": peak_src,
         },
         "e2e": e2e_line,

@@ -156,6 +156,46 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
                     pa_stream_t stream);
 
 /*
+ * pa_forward_decode -- one decode step: store each sequence's newest token,
+ * then attend over its whole history, in one call.
+ *
+ * The attention backend's decode entry takes the query, the cache pool, the
+ * block tables, the context lengths and the slot mapping together ([route]
+ * section "FlashAttention, FlashInfer and engineering reuse"): it writes the
+ * current token's K/V by slot mapping and reads the history by block table
+ * ([teaching] section "How PagedAttention plugs into mini vLLM").
+ *
+ * k_new, v_new are [batch, num_kv_heads, head_dim]: row b is the newest
+ * token of sequence b, at position context_lens[b] - 1 (context_lens
+ * include it).  slot_mapping is [batch] int64.  For each b with
+ * slot_mapping[b] >= 0 the row is stored exactly as pa_write_kv_cache
+ * would, PROVIDED that slot_mapping[b] is the slot the block table gives
+ * position context_lens[b] - 1 (physical block block_tables[b, (ctx-1) /
+ * block_size], offset (ctx-1) % block_size, both in range); any other
+ * non-negative slot sets PA_DEVERR_SLOT, that row is not stored and
+ * sequence b's output is written as zeros (its history would be
+ * incomplete).  slot_mapping[b] < 0 stores nothing.  Then out = pa_decode of the same
+ * arguments, with the stored rows visible.  A cache position that another
+ * sequence's visible history also maps (a shared page) must not be written
+ * in the same call: the order of that write and that read is unspecified.
+ *
+ * The result equals pa_write_kv_cache(..., num_tokens = batch) followed by
+ * pa_decode whenever every slot passes the check.  Workspace, streams and
+ * the remaining errors are those of pa_decode.  The row is stored inside the
+ * decode kernel, by the warp that loads the token's page, just before it
+ * loads it; for shapes outside the persistent kernel's set (see pa_decode's
+ * implementation notes in the library source) a separate write kernel with
+ * the same check runs first.
+ */
+pa_status pa_forward_decode(const pa_cache_desc *cache, void *out, const void *q,
+                            void *key_cache, void *value_cache, const void *k_new,
+                            const void *v_new, const int64_t *slot_mapping,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                            float scale, void *workspace, size_t workspace_bytes,
+                            int32_t *err_word, pa_stream_t stream);
+
+/*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
  * memory.
  *

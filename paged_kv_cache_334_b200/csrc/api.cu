@@ -264,6 +264,131 @@ namespace pa {
 void set_last_error_message(const char *msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
 }  // namespace pa
 
+// pa_decode, and pa_forward_decode when k_new / v_new / slot_mapping are set.
+static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *q, void *key_cache,
+                      void *value_cache, const void *k_new, const void *v_new,
+                      const int64_t *slot_mapping, const int32_t *block_tables,
+                      const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+                      int32_t max_blocks_per_seq, float scale, void *workspace,
+                      size_t workspace_bytes, int32_t *err_word, pa_stream_t stream) {
+  pa_status s = check_decode_common(cache, q, key_cache, value_cache, block_tables,
+                                    context_lens, batch, num_q_heads,
+                                    max_blocks_per_seq, scale);
+  if (s != PA_OK) return s;
+  const bool fused = slot_mapping != nullptr;
+  if (fused && batch > 0) {
+    if ((s = check_ptr(k_new, "k_new")) != PA_OK) return s;
+    if ((s = check_ptr(v_new, "v_new")) != PA_OK) return s;
+  }
+  if (batch == 0) return PA_OK;
+  if ((s = check_ptr(out, "out")) != PA_OK) return s;
+  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+  if (workspace_bytes < w.total)
+    return fail(PA_ERR_INVALID_ARG, "workspace too small%s: need %lld bytes", "",
+                (long long)w.total);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
+  char *ws = static_cast<char *>(workspace);
+  if (w.stream) {
+    StreamPlan sp = plan_stream(cache, num_q_heads);
+    const int sms = device_sm_count();
+    if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
+    pa::stream::Params p{};
+    if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, sp.vbs) &&
+                     encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs)))
+      sp = plan_stream(cache, num_q_heads, /*allow_tile=*/false);
+    p.q = q;
+    p.out = out;
+    p.key_cache = key_cache;
+    p.value_cache = value_cache;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.slot_mapping = slot_mapping;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.part_ml = reinterpret_cast<float *>(ws + w.part_max);
+    p.part_o = reinterpret_cast<float *>(ws + w.part_out);
+    p.seq_merge = reinterpret_cast<int32_t *>(ws + w.counters);
+    p.err_word = err_word;
+    p.num_blocks = cache->num_blocks;
+    p.block_size = cache->block_size;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.num_q_heads = num_q_heads;
+    p.max_blocks = max_blocks_per_seq;
+    p.batch = batch;
+    p.vbs = sp.vbs;
+    p.log2_vbs = sp.log2_vbs;
+    p.log2_vpp = sp.log2_vpp;
+    p.row_bytes = sp.row_bytes;
+    p.row_pitch = sp.row_pitch;
+    p.vpage_stride = sp.vpage_stride;
+    p.q_bytes = sp.q_bytes;
+    p.pps = sp.pps;
+    p.stages = sp.stages;
+    p.stage_bytes = sp.stage_bytes;
+    p.hdr_bytes = pa::stream::kHdrBytes;
+    p.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int group = num_q_heads / cache->num_kv_heads;
+    p.group = group;
+    p.heads_per_warp = sp.heads_per_warp;
+    p.warps_per_kv = sp.warps_per_kv;
+    p.tile = sp.tile ? 1 : 0;
+    p.box_bytes = sp.box_bytes;
+    p.n_dhalf = sp.n_dhalf;
+    cudaError_t e = (cache->dtype == PA_DTYPE_BF16)
+                        ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
+                                                  sp.smem, static_cast<cudaStream_t>(stream))
+                        : pa::stream::launch_f32(p, cache->head_dim, group, cache->num_kv_heads,
+                                                 sp.smem, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    e = (cache->dtype == PA_DTYPE_BF16)
+            ? pa::stream::launch_merge_bf16(p, cache->head_dim, static_cast<cudaStream_t>(stream))
+            : pa::stream::launch_merge_f32(p, cache->head_dim, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+  }
+  if (fused) {
+    // shapes of the partition kernel: the same checked write, then the decode
+    const int64_t row_bytes =
+        (int64_t)cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype);
+    cudaError_t e = pa::launch_write_kv(cache->dtype, cache->block_size, cache->num_blocks,
+                                        row_bytes, key_cache, value_cache, k_new, v_new,
+                                        slot_mapping, batch, err_word,
+                                        static_cast<cudaStream_t>(stream), block_tables,
+                                        context_lens, max_blocks_per_seq);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "write_kv launch: %s", cudaGetErrorString(e));
+  }
+  pa::DecodeArgs a{};
+  a.q = q;
+  a.out = out;
+  a.key_cache = key_cache;
+  a.value_cache = value_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.part_max = reinterpret_cast<float *>(ws + w.part_max);
+  a.part_sum = reinterpret_cast<float *>(ws + w.part_sum);
+  a.part_out = reinterpret_cast<float *>(ws + w.part_out);
+  a.counters = reinterpret_cast<int32_t *>(ws + w.counters);
+  a.err_word = err_word;
+  a.dtype = cache->dtype;
+  a.num_blocks = cache->num_blocks;
+  a.block_size = cache->block_size;
+  a.num_kv_heads = cache->num_kv_heads;
+  a.head_dim = cache->head_dim;
+  a.batch = batch;
+  a.num_q_heads = num_q_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.part_tokens = kDecodePartitionTokens;
+  a.max_parts = w.max_parts;
+  a.scale = scale;
+  a.merge = true;
+  a.slot_mapping = slot_mapping;
+  cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
 extern "C" {
 
 int32_t pa_version(void) { return 100; }
@@ -321,102 +446,25 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
                     int32_t max_blocks_per_seq, float scale, void *workspace,
                     size_t workspace_bytes, int32_t *err_word,
                     pa_stream_t stream) {
-  pa_status s = check_decode_common(cache, q, key_cache, value_cache, block_tables,
-                                    context_lens, batch, num_q_heads,
-                                    max_blocks_per_seq, scale);
-  if (s != PA_OK) return s;
-  if (batch == 0) return PA_OK;
-  if ((s = check_ptr(out, "out")) != PA_OK) return s;
-  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
-  if (workspace_bytes < w.total)
-    return fail(PA_ERR_INVALID_ARG, "workspace too small%s: need %lld bytes", "",
-                (long long)w.total);
-  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
-    return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
-  char *ws = static_cast<char *>(workspace);
-  if (w.stream) {
-    StreamPlan sp = plan_stream(cache, num_q_heads);
-    const int sms = device_sm_count();
-    if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
-    pa::stream::Params p{};
-    if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, sp.vbs) &&
-                     encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs)))
-      sp = plan_stream(cache, num_q_heads, /*allow_tile=*/false);
-    p.q = q;
-    p.out = out;
-    p.key_cache = key_cache;
-    p.value_cache = value_cache;
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    p.part_ml = reinterpret_cast<float *>(ws + w.part_max);
-    p.part_o = reinterpret_cast<float *>(ws + w.part_out);
-    p.seq_merge = reinterpret_cast<int32_t *>(ws + w.counters);
-    p.err_word = err_word;
-    p.num_blocks = cache->num_blocks;
-    p.block_size = cache->block_size;
-    p.num_kv_heads = cache->num_kv_heads;
-    p.num_q_heads = num_q_heads;
-    p.max_blocks = max_blocks_per_seq;
-    p.batch = batch;
-    p.vbs = sp.vbs;
-    p.log2_vbs = sp.log2_vbs;
-    p.log2_vpp = sp.log2_vpp;
-    p.row_bytes = sp.row_bytes;
-    p.row_pitch = sp.row_pitch;
-    p.vpage_stride = sp.vpage_stride;
-    p.q_bytes = sp.q_bytes;
-    p.pps = sp.pps;
-    p.stages = sp.stages;
-    p.stage_bytes = sp.stage_bytes;
-    p.hdr_bytes = pa::stream::kHdrBytes;
-    p.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    const int group = num_q_heads / cache->num_kv_heads;
-    p.group = group;
-    p.heads_per_warp = sp.heads_per_warp;
-    p.warps_per_kv = sp.warps_per_kv;
-    p.tile = sp.tile ? 1 : 0;
-    p.box_bytes = sp.box_bytes;
-    p.n_dhalf = sp.n_dhalf;
-    cudaError_t e = (cache->dtype == PA_DTYPE_BF16)
-                        ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
-                                                  sp.smem, static_cast<cudaStream_t>(stream))
-                        : pa::stream::launch_f32(p, cache->head_dim, group, cache->num_kv_heads,
-                                                 sp.smem, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    e = (cache->dtype == PA_DTYPE_BF16)
-            ? pa::stream::launch_merge_bf16(p, cache->head_dim, static_cast<cudaStream_t>(stream))
-            : pa::stream::launch_merge_f32(p, cache->head_dim, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
-    return PA_OK;
-  }
-  pa::DecodeArgs a{};
-  a.q = q;
-  a.out = out;
-  a.key_cache = key_cache;
-  a.value_cache = value_cache;
-  a.block_tables = block_tables;
-  a.context_lens = context_lens;
-  a.part_max = reinterpret_cast<float *>(ws + w.part_max);
-  a.part_sum = reinterpret_cast<float *>(ws + w.part_sum);
-  a.part_out = reinterpret_cast<float *>(ws + w.part_out);
-  a.counters = reinterpret_cast<int32_t *>(ws + w.counters);
-  a.err_word = err_word;
-  a.dtype = cache->dtype;
-  a.num_blocks = cache->num_blocks;
-  a.block_size = cache->block_size;
-  a.num_kv_heads = cache->num_kv_heads;
-  a.head_dim = cache->head_dim;
-  a.batch = batch;
-  a.num_q_heads = num_q_heads;
-  a.max_blocks = max_blocks_per_seq;
-  a.part_tokens = kDecodePartitionTokens;
-  a.max_parts = w.max_parts;
-  a.scale = scale;
-  a.merge = true;
-  cudaError_t e = pa::launch_decode(a, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-  return PA_OK;
+  // the caches are only read when no slot mapping is given
+  return decode_impl(cache, out, q, const_cast<void *>(key_cache),
+                     const_cast<void *>(value_cache), nullptr, nullptr, nullptr, block_tables,
+                     context_lens, batch, num_q_heads, max_blocks_per_seq, scale, workspace,
+                     workspace_bytes, err_word, stream);
+}
+
+pa_status pa_forward_decode(const pa_cache_desc *cache, void *out, const void *q,
+                            void *key_cache, void *value_cache, const void *k_new,
+                            const void *v_new, const int64_t *slot_mapping,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                            float scale, void *workspace, size_t workspace_bytes,
+                            int32_t *err_word, pa_stream_t stream) {
+  if (slot_mapping == nullptr && batch > 0)
+    return fail(PA_ERR_INVALID_ARG, "slot_mapping is NULL%s");
+  return decode_impl(cache, out, q, key_cache, value_cache, k_new, v_new, slot_mapping,
+                     block_tables, context_lens, batch, num_q_heads, max_blocks_per_seq, scale,
+                     workspace, workspace_bytes, err_word, stream);
 }
 
 pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,

@@ -54,6 +54,7 @@ struct KParams {
   float *part_out;
   int32_t *counters;
   int32_t *err_word;
+  const int64_t *slot_mapping;
   int32_t num_blocks, block_size, log2_block_size, num_kv_heads;
   int32_t num_q_heads, group, head_tiles, max_blocks;
   int32_t part_tokens, max_parts;
@@ -133,16 +134,29 @@ __global__ void __launch_bounds__(kThreads, (GT >= 8) ? 2 : 4)
   const int npages = ((t_end - 1) >> p.log2_block_size) - lb0 + 1;
 
   // Block-table slice of this partition, validated once.
-  int bad = 0;
+  int bad_block = 0;
   for (int i = tid; i < npages; i += kThreads) {
     int pb = p.block_tables[(int64_t)b * p.max_blocks + lb0 + i];
     if (pb < 0 || pb >= p.num_blocks) {
-      bad = 1;
+      bad_block = 1;
       pb = 0;
     }
     s_pages[i] = pb;
   }
-  bad = __syncthreads_or(bad);
+  // Fused write (checked by the write kernel that ran before): the partition
+  // holding the new token fails when its slot is not the table's.
+  bool bad_slot = false;
+  if (p.slot_mapping != nullptr && t_end == ctx) {
+    const int64_t slot = p.slot_mapping[b];
+    if (slot >= 0) {
+      const int pos = ctx - 1;
+      const int pbl = p.block_tables[(int64_t)b * p.max_blocks + (pos >> p.log2_block_size)];
+      bad_slot = pbl < 0 || pbl >= p.num_blocks ||
+                 slot != (int64_t)pbl * p.block_size + (pos & (p.block_size - 1));
+    }
+  }
+  bad_block = __syncthreads_or(bad_block);
+  const int bad = bad_block || bad_slot;
 
   const int tg = lane / C::LPT;  // token slot of this lane in a warp load
   const int j = lane % C::LPT;   // 16-byte chunk of the row this lane reads
@@ -334,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, (GT >= 8) ? 2 : 4)
       p.part_out[ix * D + d] = o;
     }
   }
-  if (bad && tid == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
+  if (bad_block && tid == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
+  if (bad_slot && tid == 0) set_error(p.err_word, PA_DEVERR_SLOT);
   if (!p.merge || direct) return;
 
   // Last CTA of this (sequence, KV head, head tile) merges the partials.
@@ -409,6 +424,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   kp.part_out = a.part_out;
   kp.counters = a.counters;
   kp.err_word = a.err_word;
+  kp.slot_mapping = a.slot_mapping;
   kp.num_blocks = a.num_blocks;
   kp.block_size = a.block_size;
   int lg = 0;

@@ -26,7 +26,10 @@
 //     - otherwise: 1-D bulk copies (cp.async.bulk) of the valid token rows,
 //       landing at a pitch of row_bytes + 16 for the tensor-core consumers
 //       (eight consecutive tokens in eight different bank groups);
-//   plus the sequence's query rows when a sequence segment starts.
+//   plus the sequence's query rows when a sequence segment starts.  With a
+//   slot mapping (pa_forward_decode) the producer that reaches a sequence's
+//   last page first stores the new token's K/V rows into that page (plain
+//   stores + an async-proxy fence) and then copies the page in.
 // * Consumer warps keep the online-softmax state (running max, normaliser,
 //   fp32 accumulator) of up to 8 query heads of one KV head for the current
 //   sequence segment.
@@ -57,6 +60,9 @@ namespace stream {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legitimate wait
 constexpr int kFirst = 1, kLast = 2, kBad = 4;
+// Block tables up to this size are prefetched into L2 at kernel start.
+constexpr uint64_t kTablePrefetchMax = 16ull << 20;
+constexpr int kSeqCache = 256;
 
 struct alignas(16) PageDesc {
   int32_t seq, ntok, flags, n_contrib;
@@ -124,6 +130,19 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
       "[%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
+}
+// Hints (no effect on results): bring a tensor map into the descriptor cache,
+// a byte range of global memory into L2 (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *g, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(g), "r"(bytes) : "memory");
+}
+// Orders this thread's earlier generic-proxy global stores before its later
+// async-proxy (bulk / tensor copy) accesses of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -219,6 +238,11 @@ struct alignas(16) Shared {
   int64_t red[32];
   int64_t P_begin;
   int32_t s_begin, vlb_begin, abort_flag, pad;
+  // Batches of up to kSeqCache sequences: context lengths and new-token
+  // slots read once by the prologue, so that the producer never waits on a
+  // global load of them behind its own bulk copies.
+  int64_t slot_c[kSeqCache];
+  int32_t ctx_c[kSeqCache];
 };
 
 // ===========================================================================
@@ -399,7 +423,12 @@ struct MmaConsumer {
       page_t<false>(kp, vp, ntok, p, h, col_bytes, lane);
   }
 
-  // End of a segment: write out[...] directly or a partial + merge.
+  // End of a segment: write out[...] directly (n_contrib == 1) or this CTA's
+  // normalised partial for the merge kernel.  Two rounds of lane swaps turn
+  // the MMA layout into four consecutive d per lane, so that every store
+  // moves 16 bytes (fp32) or 8 bytes (bf16): with q = g % 4, an even-g lane
+  // ends with head 2t and an odd-g lane with head 2t + 1, at d = 16k +
+  // (g - q) + (q < 2 ? 0 : 8) .. + 3.
   template <typename Tout>
   __device__ __forceinline__ void flush(const Params &p, const PageDesc &d, int hq0, int nh,
                                         int c, int lane) {
@@ -410,49 +439,46 @@ struct MmaConsumer {
       L0 += __shfl_xor_sync(0xffffffffu, L0, mask);
       L1 += __shfl_xor_sync(0xffffffffu, L1, mask);
     }
-    const int h0 = 2 * t, h1 = 2 * t + 1;
-    const int64_t orow = (int64_t)d.seq * p.num_q_heads + hq0;
-    if (d.n_contrib == 1) {
-      const float i0 = 1.f / L0, i1 = 1.f / L1;
+    const bool odd = g & 1;
+    const int q = g & 3;
+    const int hh = 2 * t + (odd ? 1 : 0);  // head of this lane's values
+    const float inv = seg_bad ? 0.f : 1.f / (odd ? L1 : L0);
+    const int dcol = (g - q) + (q < 2 ? 0 : 8);
+    float4 v[KS];
 #pragma unroll
-      for (int k = 0; k < KS; ++k) {
-        const int dd = k * 16 + g;
-        if (h0 < nh) {
-          Elem<Tout>::store1(p.out, (orow + h0) * D + dd, seg_bad ? 0.f : o[k][0] * i0);
-          Elem<Tout>::store1(p.out, (orow + h0) * D + dd + 8, seg_bad ? 0.f : o[k][2] * i0);
-        }
-        if (h1 < nh) {
-          Elem<Tout>::store1(p.out, (orow + h1) * D + dd, seg_bad ? 0.f : o[k][1] * i1);
-          Elem<Tout>::store1(p.out, (orow + h1) * D + dd + 8, seg_bad ? 0.f : o[k][3] * i1);
-        }
+    for (int k = 0; k < KS; ++k) {
+      // round 1 (lanes g, g ^ 1): pairs (d, d + 1) of one head, at +0 and +8
+      const float s0 = __shfl_xor_sync(0xffffffffu, odd ? o[k][0] : o[k][1], 4);
+      const float s2 = __shfl_xor_sync(0xffffffffu, odd ? o[k][2] : o[k][3], 4);
+      const float lo0 = odd ? s0 : o[k][0], lo1 = odd ? o[k][1] : s0;
+      const float hi0 = odd ? s2 : o[k][2], hi1 = odd ? o[k][3] : s2;
+      // round 2 (lanes g, g ^ 2): q < 2 keeps the +0 pairs, q >= 2 the +8 pairs
+      const float r0 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi0 : lo0, 8);
+      const float r1 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi1 : lo1, 8);
+      v[k] = q < 2 ? make_float4(lo0 * inv, lo1 * inv, r0 * inv, r1 * inv)
+                   : make_float4(r0 * inv, r1 * inv, hi0 * inv, hi1 * inv);
+    }
+    if (d.n_contrib == 1) {
+      if (hh < nh) {
+        const int64_t row = ((int64_t)d.seq * p.num_q_heads + hq0 + hh) * D;
+#pragma unroll
+        for (int k = 0; k < KS; ++k) Elem<Tout>::store4(p.out, row + k * 16 + dcol, v[k]);
       }
       return;
     }
     const int64_t prow = ((int64_t)c * 2 + (d.slot_bits & 1)) * p.num_q_heads + hq0;
     if (g == 0) {
-      if (h0 < nh) {
-        p.part_ml[(prow + h0) * 2 + 0] = m0_;
-        p.part_ml[(prow + h0) * 2 + 1] = seg_bad ? -1.f : L0;
-      }
-      if (h1 < nh) {
-        p.part_ml[(prow + h1) * 2 + 0] = m1_;
-        p.part_ml[(prow + h1) * 2 + 1] = seg_bad ? -1.f : L1;
-      }
+      if (2 * t < nh)
+        *reinterpret_cast<float2 *>(p.part_ml + (prow + 2 * t) * 2) =
+            make_float2(m0_, seg_bad ? -1.f : L0);
+      if (2 * t + 1 < nh)
+        *reinterpret_cast<float2 *>(p.part_ml + (prow + 2 * t + 1) * 2) =
+            make_float2(m1_, seg_bad ? -1.f : L1);
     }
-    {
-      const float i0 = 1.f / L0, i1 = 1.f / L1;
+    if (hh < nh) {
+      float *row = p.part_o + (prow + hh) * D;
 #pragma unroll
-      for (int k = 0; k < KS; ++k) {
-        const int dd = k * 16 + g;
-        if (h0 < nh) {
-          p.part_o[(prow + h0) * D + dd] = seg_bad ? 0.f : o[k][0] * i0;
-          p.part_o[(prow + h0) * D + dd + 8] = seg_bad ? 0.f : o[k][2] * i0;
-        }
-        if (h1 < nh) {
-          p.part_o[(prow + h1) * D + dd] = seg_bad ? 0.f : o[k][1] * i1;
-          p.part_o[(prow + h1) * D + dd + 8] = seg_bad ? 0.f : o[k][3] * i1;
-        }
-      }
+      for (int k = 0; k < KS; ++k) *reinterpret_cast<float4 *>(row + k * 16 + dcol) = v[k];
     }
     // merged later by the merge kernel
   }
@@ -657,30 +683,94 @@ struct PageWalker {
   int32_t s, vlb, ctx_s, pages_s;
   int32_t cw, cw_ctx;             // context-length window: lane l holds sequence cw + l
   int32_t tw_seq, tw_lb, tw_val;  // table window: lane l holds entry tw_lb + l of tw_seq
+  int64_t cw_slot, slot_s;        // fused write: slot of sequence cw + l; of sequence s
+  int32_t tn_seq, tn_lb, tn_val;  // next table window, loading ahead of use
   int64_t P_s, cursor;
 
-  __device__ __forceinline__ void init(const Params &p, int32_t s0, int32_t vlb0, int64_t P0,
-                                       int64_t cur0, int lane) {
+  const Shared *shc;  // context lengths / slots cached in shared memory, or NULL
+
+  __device__ __forceinline__ void load_window(const Params &p, int lane) {
+    const bool in = cw + lane < p.batch;
+    if (shc != nullptr) {
+      cw_ctx = in ? shc->ctx_c[cw + lane] : 0;
+      cw_slot = in ? shc->slot_c[cw + lane] : -1;
+    } else {
+      cw_ctx = in ? p.context_lens[cw + lane] : 0;
+      cw_slot = (in && p.slot_mapping != nullptr) ? p.slot_mapping[cw + lane] : -1;
+    }
+  }
+  // Fused write: when this CTA owns the sequence's last page, start moving
+  // the new token's rows towards L2 now; they are copied at that page.
+  __device__ __forceinline__ void prefetch_new_rows(const Params &p, int64_t end, int lane) {
+    if (p.slot_mapping != nullptr && lane == 0 && slot_s >= 0 && P_s + pages_s <= end) {
+      const int64_t off = (int64_t)s * p.row_bytes;
+      prefetch_l2(static_cast<const unsigned char *>(p.k_new) + off, (uint32_t)p.row_bytes);
+      prefetch_l2(static_cast<const unsigned char *>(p.v_new) + off, (uint32_t)p.row_bytes);
+    }
+  }
+  __device__ __forceinline__ void init(const Params &p, const Shared *cache, int32_t s0,
+                                       int32_t vlb0, int64_t P0, int64_t cur0, int64_t end,
+                                       int lane) {
+    shc = cache;
     s = s0;
     vlb = vlb0;
     P_s = P0;
     cursor = cur0;
     cw = s0;
-    cw_ctx = (cw + lane < p.batch) ? p.context_lens[cw + lane] : 0;
+    load_window(p, lane);
     ctx_s = __shfl_sync(0xffffffffu, cw_ctx, 0);
+    slot_s = __shfl_sync(0xffffffffu, cw_slot, 0);
     pages_s = vpages_of(ctx_s, p);
     tw_seq = -1;
     tw_lb = 0;
     tw_val = -1;
+    tn_seq = -1;
+    tn_lb = 0;
+    tn_val = -1;
+    prefetch_new_rows(p, end, lane);
+  }
+  // Block-table window (32 entries of one sequence from entry lb) into lane
+  // registers: the load is only issued here, and waited for at first use.
+  __device__ __forceinline__ int32_t load_table(const Params &p, int32_t seq, int32_t lb,
+                                                int lane) const {
+    const int32_t e = lb + lane;
+    return (e < p.max_blocks) ? p.block_tables[(int64_t)seq * p.max_blocks + e] : -1;
+  }
+  // Start loading the window after the current one: the rest of a long
+  // sequence, else the next sequence with visible pages, looked up in the
+  // cached context lengths (nothing is prefetched without the cache).
+  __device__ __forceinline__ void prefetch_next_window(const Params &p, int64_t end,
+                                                       int lane) {
+    const int32_t blocks = (ctx_s + p.block_size - 1) / p.block_size;
+    if (tw_lb + 32 < blocks) {
+      tn_seq = s;
+      tn_lb = tw_lb + 32;
+    } else {
+      if (shc == nullptr) return;
+      const int64_t next_page = P_s + pages_s;  // stream index of the next sequence's page
+      if (next_page >= end) return;             // this CTA's range ends first
+      int32_t n = s + 1;
+      while (n < p.batch && n < s + 33 && vpages_of(shc->ctx_c[n], p) == 0) ++n;
+      if (n >= p.batch || n >= s + 33) return;
+      tn_seq = n;
+      tn_lb = 0;
+    }
+    tn_val = load_table(p, tn_seq, tn_lb, lane);
   }
   // Physical block of the current page.
-  __device__ __forceinline__ int32_t block(const Params &p, int lane) {
+  __device__ __forceinline__ int32_t block(const Params &p, int64_t end, int lane) {
     const int32_t lb = vlb >> p.log2_vpp;
     if (s != tw_seq || lb >= tw_lb + 32) {
+      if (s == tn_seq && lb >= tn_lb && lb < tn_lb + 32) {
+        tw_val = tn_val;  // prefetched
+        tw_lb = tn_lb;
+      } else {
+        tw_lb = lb;
+        tw_val = load_table(p, s, lb, lane);
+      }
       tw_seq = s;
-      tw_lb = lb;
-      const int32_t e = lb + lane;
-      tw_val = (e < p.max_blocks) ? p.block_tables[(int64_t)s * p.max_blocks + e] : -1;
+      tn_seq = -1;
+      prefetch_next_window(p, end, lane);
     }
     return __shfl_sync(0xffffffffu, tw_val, lb - tw_lb);
   }
@@ -696,7 +786,7 @@ struct PageWalker {
       for (;;) {
         if (nxt >= cw + 32) {
           cw = nxt;
-          cw_ctx = (cw + lane < p.batch) ? p.context_lens[cw + lane] : 0;
+          load_window(p, lane);
         }
         const bool has =
             (cw + lane >= nxt) && (cw + lane < p.batch) && vpages_of(cw_ctx, p) > 0;
@@ -705,6 +795,7 @@ struct PageWalker {
           const int l = __ffs(m) - 1;
           nxt = cw + l;
           ctx_s = __shfl_sync(0xffffffffu, cw_ctx, l);
+          slot_s = __shfl_sync(0xffffffffu, cw_slot, l);
           break;
         }
         nxt = cw + 32;
@@ -713,9 +804,47 @@ struct PageWalker {
       s = nxt;
       vlb = 0;
       pages_s = vpages_of(ctx_s, p);
+      prefetch_new_rows(p, end, lane);
     }
   }
 };
+
+// Fused cache write of sequence s's new token to `slot` (all lanes of the
+// producer warp): row_bytes of K and of V, 16-byte vectors, loads batched
+// ahead of the stores.  Each lane then fences its stores against the tensor
+// copy that will read the page back.
+__device__ __forceinline__ void write_new_rows(const Params &p, int32_t s, int64_t slot,
+                                               int lane) {
+  const int n = p.row_bytes >> 4;
+  const uint4 *ks = reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.k_new) +
+                                                    (int64_t)s * p.row_bytes);
+  const uint4 *vs = reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.v_new) +
+                                                    (int64_t)s * p.row_bytes);
+  uint4 *kd = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.key_cache) +
+                                        slot * p.row_bytes);
+  uint4 *vd = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.value_cache) +
+                                        slot * p.row_bytes);
+  for (int x0 = lane; x0 < n; x0 += 4 * 32) {
+    uint4 a[4], b[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int x = x0 + 32 * u;
+      if (x < n) {
+        a[u] = __ldg(ks + x);
+        b[u] = __ldg(vs + x);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int x = x0 + 32 * u;
+      if (x < n) {
+        kd[x] = a[u];
+        vd[x] = b[u];
+      }
+    }
+  }
+  fence_proxy_async_global();
+}
 
 // ===========================================================================
 // The kernel.  T = element type; D = head_dim; G = query heads per KV head
@@ -744,6 +873,25 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
+  // Hints first (they read nothing into registers): the tensor maps, and this
+  // CTA's share of the block table into L2, so that the first table lookups
+  // after the scan of context lengths hit L2.
+  if (tid == 0 && p.tile) {
+    prefetch_tensormap(&p.tmap_k);
+    prefetch_tensormap(&p.tmap_v);
+  }
+  if (tid == 32) {
+    const uint64_t bytes = (uint64_t)p.batch * (uint64_t)p.max_blocks * 4u;
+    if (bytes <= kTablePrefetchMax) {
+      const uint64_t base = reinterpret_cast<uint64_t>(p.block_tables);
+      const uint64_t chunk = ((bytes + p.grid - 1) / p.grid + 15) & ~15ull;
+      uint64_t lo = base + (uint64_t)c * chunk, hi = lo + chunk;
+      if (hi > base + bytes) hi = base + bytes;
+      lo = (lo + 15) & ~15ull;
+      hi &= ~15ull;
+      if (hi > lo) prefetch_l2(reinterpret_cast<const void *>(lo), (uint32_t)(hi - lo));
+    }
+  }
   // Launched with programmatic stream serialisation: this CTA may start
   // while the previous kernel of the stream still runs.  Nothing it reads or
   // writes is touched before that kernel has finished and flushed.
@@ -762,34 +910,68 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   }
 
   // ---- Prologue: total virtual pages T, this CTA's range and first page.
-  int64_t T_loc = 0;
-  for (int base = 0; base < p.batch; base += blockDim.x) {
-    const int s = base + tid;
-    const int64_t v = (s < p.batch) ? vpages_of(p.context_lens[s], p) : 0;
-    T_loc += block_sum(v, sh.red);
-  }
-  const int64_t Tp = T_loc;
-  const int32_t g_eff = (int32_t)((Tp < p.grid) ? Tp : p.grid);
-  const bool active = c < g_eff;
-  int64_t start = 0, end = 0;
-  if (active) {
-    start = (int64_t)c * Tp / g_eff;
-    end = (int64_t)(c + 1) * Tp / g_eff;
-    int64_t run = 0;
-    for (int base = 0; base < p.batch; base += blockDim.x) {
-      const int s = base + tid;
-      const int64_t v = (s < p.batch) ? vpages_of(p.context_lens[s], p) : 0;
-      int64_t tot;
-      const int64_t P = run + block_exclusive_scan(v, sh.red, &tot);
+  int64_t Tp, start = 0, end = 0;
+  int32_t g_eff;
+  const bool cached = p.batch <= kSeqCache;
+  if (p.batch <= (int)blockDim.x) {
+    // one scan gives both the total and every sequence's first page
+    int32_t ctx = 0;
+    if (tid < p.batch) {
+      ctx = p.context_lens[tid];
+      if (cached) {
+        sh.ctx_c[tid] = ctx;
+        sh.slot_c[tid] = (p.slot_mapping != nullptr) ? p.slot_mapping[tid] : -1;
+      }
+    }
+    const int64_t v = (tid < p.batch) ? vpages_of(ctx, p) : 0;
+    const int64_t P = block_exclusive_scan(v, sh.red, &Tp);
+    g_eff = (int32_t)((Tp < p.grid) ? Tp : p.grid);
+    if (c < g_eff) {
+      start = (int64_t)c * Tp / g_eff;
+      end = (int64_t)(c + 1) * Tp / g_eff;
       if (v > 0 && P <= start && start < P + v) {
-        sh.s_begin = s;
+        sh.s_begin = tid;
         sh.vlb_begin = (int32_t)(start - P);
         sh.P_begin = P;
       }
-      run += tot;
-      if (run > start) break;  // uniform: every thread sees the same `run`
+    }
+  } else {
+    int64_t T_loc = 0;
+    for (int base = 0; base < p.batch; base += blockDim.x) {
+      const int s = base + tid;
+      int32_t ctx = 0;
+      if (s < p.batch) {
+        ctx = p.context_lens[s];
+        if (cached) {
+          sh.ctx_c[s] = ctx;
+          sh.slot_c[s] = (p.slot_mapping != nullptr) ? p.slot_mapping[s] : -1;
+        }
+      }
+      const int64_t v = (s < p.batch) ? vpages_of(ctx, p) : 0;
+      T_loc += block_sum(v, sh.red);
+    }
+    Tp = T_loc;
+    g_eff = (int32_t)((Tp < p.grid) ? Tp : p.grid);
+    if (c < g_eff) {
+      start = (int64_t)c * Tp / g_eff;
+      end = (int64_t)(c + 1) * Tp / g_eff;
+      int64_t run = 0;
+      for (int base = 0; base < p.batch; base += blockDim.x) {
+        const int s = base + tid;
+        const int64_t v = (s < p.batch) ? vpages_of(p.context_lens[s], p) : 0;
+        int64_t tot;
+        const int64_t P = run + block_exclusive_scan(v, sh.red, &tot);
+        if (v > 0 && P <= start && start < P + v) {
+          sh.s_begin = s;
+          sh.vlb_begin = (int32_t)(start - P);
+          sh.P_begin = P;
+        }
+        run += tot;
+        if (run > start) break;  // uniform: every thread sees the same `run`
+      }
     }
   }
+  const bool active = c < g_eff;
   __syncthreads();
 
   const bool per_row = p.row_pitch != p.row_bytes;
@@ -798,7 +980,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     if (warp == 0) {
       // ===================== producer =====================
       PageWalker wk;
-      wk.init(p, sh.s_begin, sh.vlb_begin, sh.P_begin, start, lane);
+      wk.init(p, cached ? &sh : nullptr, sh.s_begin, sh.vlb_begin, sh.P_begin, start, end,
+              lane);
       bool ok = true;
       int issued = 0;
       for (int i = 0; i < n_stages && ok; ++i) {
@@ -810,12 +993,30 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         }
         const int npg = (int)min((int64_t)p.pps, end - wk.cursor);
         uint32_t bytes = 0;
+        bool wrote = false;
         for (int k = 0; k < npg; ++k) {
-          const int32_t pb = wk.block(p, lane);
+          const int32_t pb = wk.block(p, end, lane);
           const int32_t ntok = wk.ntok(p);
           const bool first = (wk.vlb == 0) || (wk.cursor == start);
-          const bool last = (wk.vlb == wk.pages_s - 1) || (wk.cursor == end - 1);
-          const bool bad = pb < 0 || pb >= p.num_blocks;
+          const bool seq_last = wk.vlb == wk.pages_s - 1;
+          const bool last = seq_last || (wk.cursor == end - 1);
+          const bool bad_block = pb < 0 || pb >= p.num_blocks;
+          bool bad = bad_block;
+          if (bad_block && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
+          if (p.slot_mapping != nullptr && seq_last && wk.slot_s >= 0) {
+            // Fused cache write: the new token sits at position ctx - 1, in
+            // this page; its slot must be the one the table gives it, else
+            // nothing is stored and the sequence's output is zeroed.
+            const int32_t pos = wk.ctx_s - 1;
+            const int64_t want = (int64_t)pb * p.block_size + (pos & (p.block_size - 1));
+            if (!bad_block && wk.slot_s == want) {
+              write_new_rows(p, wk.s, want, lane);
+              wrote = true;
+            } else {
+              bad = true;
+              if (lane == 0) set_error(p.err_word, PA_DEVERR_SLOT);
+            }
+          }
           if (lane == 0) {
             PageDesc d;
             d.seq = wk.s;
@@ -849,6 +1050,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           wk.advance(p, end, lane);
         }
         __syncwarp();
+        // the rows written above are read back by this stage's copies
+        if (wrote) fence_proxy_async_global();
         if (lane == 0) mbar_arrive_expect_tx(&sh.full[slot], bytes);
         __syncwarp();
         unsigned char *st = stages + (size_t)slot * p.stage_bytes;
@@ -966,7 +1169,6 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             } else {
               cs.flush(p, d, hq0, c, lane);
             }
-            if (cs.seg_bad && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
             cs.reset();
           }
         }
@@ -987,6 +1189,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       reinterpret_cast<int4 *>(p.seq_merge)[s] = make_int4(0, 0, 0, 0);
       if (ctx < 0 || (int64_t)ctx > (int64_t)p.max_blocks * p.block_size)
         set_error(p.err_word, PA_DEVERR_CONTEXT_LEN);
+      // fused write: no visible position for the new token
+      if (p.slot_mapping != nullptr && p.slot_mapping[s] >= 0)
+        set_error(p.err_word, PA_DEVERR_SLOT);
     }
     const int64_t n = (int64_t)p.num_q_heads * D;
     for (int64_t x = tid; x < n; x += blockDim.x) Elem<T>::store1(p.out, (int64_t)s * n + x, 0.f);

@@ -35,6 +35,14 @@ struct Elem<float> {
   __device__ __forceinline__ static void store1(void *p, int64_t i, float x) {
     static_cast<float *>(p)[i] = x;
   }
+  // Elements i and i + 1 (i even, base 16-byte aligned).
+  __device__ __forceinline__ static void store2(void *p, int64_t i, float a, float b) {
+    *reinterpret_cast<float2 *>(static_cast<float *>(p) + i) = make_float2(a, b);
+  }
+  // Elements i .. i + 3 (i a multiple of 4, base 16-byte aligned).
+  __device__ __forceinline__ static void store4(void *p, int64_t i, float4 v) {
+    *reinterpret_cast<float4 *>(static_cast<float *>(p) + i) = v;
+  }
 };
 
 template <>
@@ -56,6 +64,22 @@ struct Elem<__nv_bfloat16> {
   }
   __device__ __forceinline__ static void store1(void *p, int64_t i, float x) {
     static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+  }
+  // Elements i and i + 1 (i even, base 16-byte aligned), each rounded to
+  // nearest even.
+  __device__ __forceinline__ static void store2(void *p, int64_t i, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(p) + i) =
+        __floats2bfloat162_rn(a, b);
+  }
+  // Elements i .. i + 3 (i a multiple of 4, base 16-byte aligned), rounded to
+  // nearest even.
+  __device__ __forceinline__ static void store4(void *p, int64_t i, float4 v) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t *>(&lo);
+    u.y = *reinterpret_cast<const uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p) + i) = u;
   }
 };
 

@@ -20,6 +20,9 @@ struct DecodeArgs {
   float *part_out;   // [B, Hq, max_parts, D]
   int32_t *counters; // [B * Hkv * head_tiles]; pa_decode only
   int32_t *err_word;
+  // pa_forward_decode: a sequence whose new-token slot is not the one its
+  // table gives position ctx - 1 is flagged PA_DEVERR_SLOT and zeroed.
+  const int64_t *slot_mapping;
   int32_t dtype;
   int32_t num_blocks, block_size, num_kv_heads, head_dim;
   int32_t batch, num_q_heads, max_blocks;
@@ -46,8 +49,14 @@ struct Params {
   CUtensorMap tmap_v;
   const void *q;
   void *out;
-  const void *key_cache;
-  const void *value_cache;
+  void *key_cache;    // written only by the fused cache write (slot_mapping set)
+  void *value_cache;
+  // Fused cache write (pa_forward_decode), all NULL for pa_decode: row b of
+  // k_new / v_new ([batch][Hkv][D]) goes to slot_mapping[b] when that is the
+  // slot of position context_lens[b] - 1 of sequence b.
+  const void *k_new;
+  const void *v_new;
+  const int64_t *slot_mapping;
   const int32_t *block_tables;
   const int32_t *context_lens;
   float *part_ml;     // [kMaxGrid * 2][Hq][2]: (max in log2 units, normaliser)
@@ -84,12 +93,17 @@ cudaError_t launch_f32(const Params &p, int head_dim, int group, int hkv, size_t
 // Query heads handled together by one CTA for a GQA group of `group` heads.
 int decode_head_tile(int group);
 
+// With block_tables / context_lens set (num_tokens = batch, token b = the
+// newest token of sequence b), a token is written only when its slot is the
+// one the table gives position context_lens[b] - 1; others are flagged.
 cudaError_t launch_write_kv(int32_t dtype, int32_t block_size,
                             int32_t num_blocks, int64_t row_bytes,
                             void *key_cache, void *value_cache,
                             const void *k_new, const void *v_new,
                             const int64_t *slot_mapping, int32_t num_tokens,
-                            int32_t *err_word, cudaStream_t stream);
+                            int32_t *err_word, cudaStream_t stream,
+                            const int32_t *block_tables = nullptr,
+                            const int32_t *context_lens = nullptr, int32_t max_blocks = 0);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 

@@ -19,7 +19,10 @@ __global__ void __launch_bounds__(128)
 write_kv_kernel(uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache,
                 const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
                 const int64_t *__restrict__ slot_mapping, int64_t num_slots,
-                int64_t row_vecs, int32_t *err_word) {
+                int64_t row_vecs, int32_t *err_word,
+                const int32_t *__restrict__ block_tables,
+                const int32_t *__restrict__ context_lens, int32_t max_blocks,
+                int32_t block_size, int32_t num_blocks) {
   // The decode kernel that usually follows waits for this grid to finish
   // (griddepcontrol.wait) before it reads anything; letting it launch now
   // overlaps its start-up with this copy.
@@ -27,7 +30,20 @@ write_kv_kernel(uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache,
   const int64_t token = blockIdx.x;
   const int64_t slot = slot_mapping[token];
   if (slot < 0) return;
-  if (slot >= num_slots) {
+  bool ok = slot < num_slots;
+  if (ok && block_tables != nullptr) {
+    // decode step: token b is sequence b's newest, at position ctx - 1; only
+    // the slot the block table gives that position is accepted
+    const int32_t ctx = context_lens[token];
+    ok = ctx > 0 && (int64_t)ctx <= (int64_t)max_blocks * block_size;
+    if (ok) {
+      const int32_t pos = ctx - 1;
+      const int32_t pb = block_tables[token * (int64_t)max_blocks + pos / block_size];
+      ok = pb >= 0 && pb < num_blocks &&
+           slot == (int64_t)pb * block_size + pos % block_size;
+    }
+  }
+  if (!ok) {
     if (blockIdx.y == 0 && threadIdx.x == 0) set_error(err_word, PA_DEVERR_SLOT);
     return;
   }
@@ -47,7 +63,9 @@ cudaError_t launch_write_kv(int32_t dtype, int32_t block_size,
                             void *key_cache, void *value_cache,
                             const void *k_new, const void *v_new,
                             const int64_t *slot_mapping, int32_t num_tokens,
-                            int32_t *err_word, cudaStream_t stream) {
+                            int32_t *err_word, cudaStream_t stream,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            int32_t max_blocks) {
   (void)dtype;
   if (num_tokens == 0) return cudaSuccess;
   const int64_t row_vecs = row_bytes / 16;
@@ -58,7 +76,8 @@ cudaError_t launch_write_kv(int32_t dtype, int32_t block_size,
   write_kv_kernel<<<grid, threads, 0, stream>>>(
       static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache),
       static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
-      slot_mapping, (int64_t)num_blocks * block_size, row_vecs, err_word);
+      slot_mapping, (int64_t)num_blocks * block_size, row_vecs, err_word, block_tables,
+      context_lens, max_blocks, block_size, num_blocks);
   return cudaGetLastError();
 }
 

@@ -39,7 +39,7 @@ PA_DEVERR_SLOT = 4
 EXPORTED_SYMBOLS = (
     "pa_version", "pa_status_string", "pa_last_error_message", "pa_write_kv_cache",
     "pa_decode_workspace_bytes", "pa_decode", "pa_decode_splitk", "pa_reduce",
-    "pa_decode_noalloc",
+    "pa_decode_noalloc", "pa_forward_decode",
 )
 
 # Size of the fixed device scratch array pa_decode_noalloc uses.
@@ -92,6 +92,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_reduce.restype = ctypes.c_int
     lib.pa_decode_noalloc.argtypes = [D, P, P, P, P, P, P, i32, i32, i32, f32, P, P]
     lib.pa_decode_noalloc.restype = ctypes.c_int
+    lib.pa_forward_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, i32, i32, i32, f32, P, sz,
+                                      P, P]
+    lib.pa_forward_decode.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -193,6 +196,34 @@ def pa_decode(out, q, key_cache, value_cache, block_tables, context_lens,
     _check(lib.pa_decode(
         ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
         _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
+        _dev(workspace, "workspace"), int(workspace.numel() * workspace.element_size()),
+        _dev(err_word, "err_word", torch.int32), _stream(stream)))
+    return out
+
+
+def pa_forward_decode(out, q, key_cache, value_cache, k_new, v_new, slot_mapping,
+                      block_tables, context_lens, scale: Optional[float] = None,
+                      workspace: Optional[torch.Tensor] = None,
+                      err_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step: store each sequence's newest K/V row at its slot, then
+    decode over the whole history into `out` (see include/pa.h)."""
+    lib = load()
+    desc = cache_desc(key_cache)
+    B, Hq, Dq = q.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if slot_mapping.numel() != B:
+        raise ValueError("slot_mapping must hold one slot per sequence")
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dq)
+    if workspace is None:
+        workspace = decode_workspace(key_cache, B, Hq, MB)
+    _check(lib.pa_forward_decode(
+        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
+        _dev(k_new, "k_new", key_cache.dtype), _dev(v_new, "v_new", key_cache.dtype),
+        _dev(slot_mapping, "slot_mapping", torch.int64),
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
         _dev(workspace, "workspace"), int(workspace.numel() * workspace.element_size()),

@@ -146,3 +146,22 @@ def test_noalloc_size_limit_and_argument_checks(lib):
              None) == pa.PA_ERR_UNSUPPORTED
     assert f(ctypes.byref(_desc()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 32, 4, 0.1, None,
              None) == pa.PA_OK
+
+
+def test_forward_decode_argument_checks(lib):
+    """pa_forward_decode: the slot mapping and the new rows are required and
+    checked before any device work; the rest are pa_decode's checks."""
+    f = lib.pa_forward_decode
+    d = _desc()
+
+    def call(k_new=FAKE, v_new=FAKE, sm=FAKE, B=2, Hq=32, dsc=d):
+        return f(ctypes.byref(dsc), FAKE, FAKE, FAKE, FAKE, k_new, v_new, sm, FAKE, FAKE, B, Hq,
+                 4, 0.1, FAKE, 1 << 30, None, None)
+
+    assert call(sm=None) == pa.PA_ERR_INVALID_ARG
+    assert b"slot_mapping" in lib.pa_last_error_message()
+    assert call(k_new=None) == pa.PA_ERR_INVALID_ARG
+    assert call(v_new=MISALIGNED) == pa.PA_ERR_INVALID_ARG
+    assert call(Hq=30) == pa.PA_ERR_INVALID_ARG
+    assert call(dsc=_desc(d=96)) == pa.PA_ERR_UNSUPPORTED
+    assert call(B=0, sm=None, k_new=None, v_new=None) == pa.PA_OK
