@@ -119,12 +119,21 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   const int32_t group = num_q_heads / hkv;
   const bool bf16 = c->dtype == PA_DTYPE_BF16;
   if (bf16) {
-    // tensor-core consumers: one warp per (KV head, 8 query heads)
-    if (group > 8 && group % 8 != 0) return s;
-    s.heads_per_warp = group < 8 ? group : 8;
-    s.warps_per_kv = group > 8 ? group / 8 : 1;
-    const int32_t ncw = hkv * s.warps_per_kv;
-    if (ncw != 4 && ncw != 8 && ncw != 16) return s;
+    // tensor-core consumers: one warp per (KV head, 16 query heads) when the
+    // group is a multiple of 16, else per (KV head, up to 8 query heads)
+    auto ncw_ok = [&](int32_t per_kv) {
+      const int32_t ncw = hkv * per_kv;
+      return ncw == 4 || ncw == 8 || ncw == 16;
+    };
+    if (group % 16 == 0 && ncw_ok(group / 16)) {
+      s.heads_per_warp = 16;
+      s.warps_per_kv = group / 16;
+    } else {
+      if (group > 8 && group % 8 != 0) return s;
+      s.heads_per_warp = group < 8 ? group : 8;
+      s.warps_per_kv = group > 8 ? group / 8 : 1;
+      if (!ncw_ok(s.warps_per_kv)) return s;
+    }
   } else {
     // CUDA-core consumers: one warp per KV head
     if (hkv != 4 && hkv != 8) return s;

@@ -485,6 +485,218 @@ struct MmaConsumer {
 };
 
 // ===========================================================================
+// bf16 consumer for large GQA / MQA groups (a multiple of 16 query heads per
+// KV head): the warp's 16 query heads are the M side of the tensor-core
+// tiles, so Q stays in registers as the A operand of S = Q K^T, the scores
+// of one head sit in one lane quad (row statistics need two shuffles), and P
+// is already the A operand of O += P V.  Lane (r = lane / 4, c = lane % 4)
+// holds rows r and r + 8 (heads hq0 + r, hq0 + r + 8); score column
+// (token) 8n + 2c (+1) of n tile n; output column d = 8j + 2c (+1) of d tile j.
+// ===========================================================================
+template <int D>
+struct HeadRowConsumer {
+  static constexpr int KS = D / 16;  // k steps of QK
+  static constexpr int NJ = D / 8;   // d tiles of PV
+  uint32_t qa[KS][4];                // Q (16 heads x D) as A fragments
+  float o[NJ][4];                    // O (16 heads x D) accumulators
+  float m0_, m1_, l0, l1;            // rows r, r + 8: running max, this lane's partial sum
+  float scale_log2_;
+  bool seg_bad;
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[j][e] = 0.f;
+    m0_ = m1_ = -INFINITY;
+    l0 = l1 = 0.f;
+    seg_bad = false;
+  }
+
+  __device__ __forceinline__ void load_q(const __nv_bfloat16 *qs, int hq0, int nh, int lane) {
+    (void)nh;  // always 16
+    const int r = lane >> 2, c = lane & 3;
+    const uint32_t *row0 = reinterpret_cast<const uint32_t *>(qs + (size_t)(hq0 + r) * D);
+    const uint32_t *row1 = reinterpret_cast<const uint32_t *>(qs + (size_t)(hq0 + r + 8) * D);
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      qa[k][0] = row0[(k * 16 + 2 * c) >> 1];
+      qa[k][1] = row1[(k * 16 + 2 * c) >> 1];
+      qa[k][2] = row0[(k * 16 + 2 * c + 8) >> 1];
+      qa[k][3] = row1[(k * 16 + 2 * c + 8) >> 1];
+    }
+  }
+
+  // Shared-memory address of 16 bytes of token row `tok`, d chunk `ch`
+  // (8 elements): TL = swizzled boxes [d half][KV head][vbs tokens][128 B],
+  // else rows `row_pitch` apart with this head's slice at col_bytes.
+  template <bool TL>
+  __device__ __forceinline__ uint32_t row_addr(const unsigned char *base, int tok, int ch,
+                                               const Params &p, int h, int col_bytes) const {
+    if (TL)
+      return smem_u32(base + (ch >> 3) * p.box_bytes + (h * p.vbs + tok) * 128 +
+                      (((ch & 7) ^ (tok & 7)) << 4));
+    return smem_u32(base + tok * p.row_pitch + col_bytes + ch * 16);
+  }
+
+  // Tokens [m0, m0 + 16 * NH) of a staged page (NH = 1 or 2 groups of 16),
+  // ntok valid tokens in the page.
+  template <int NH, bool TL>
+  __device__ __forceinline__ void chunk(const unsigned char *kp, const unsigned char *vp, int m0,
+                                        int ntok, const Params &p, int h, int col_bytes,
+                                        int lane) {
+    constexpr int NN = 2 * NH;  // n tiles of 8 tokens
+    const int c = lane & 3;
+    float s[NN][4];
+#pragma unroll
+    for (int n = 0; n < NN; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
+    // K rows as B operands: one ldmatrix.x4 gives two n tiles x one k step
+    const int kt = (lane & 7) + ((lane >> 4) << 3);
+    const int kc = (lane >> 3) & 1;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+#pragma unroll
+      for (int u = 0; u < NH; ++u) {
+        uint32_t b[4];
+        ldsm_x4(b, row_addr<TL>(kp, m0 + 16 * u + kt, 2 * k + kc, p, h, col_bytes));
+        mma_16816(s[2 * u], qa[k], b[0], b[1]);
+        mma_16816(s[2 * u + 1], qa[k], b[2], b[3]);
+      }
+    }
+    // scale to log2 units, mask tokens past the page, row maxima
+    float x0 = -INFINITY, x1 = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < NN; ++n) {
+      const int t0 = m0 + 8 * n + 2 * c;
+      s[n][0] = t0 < ntok ? s[n][0] * scale_log2_ : -INFINITY;
+      s[n][1] = t0 + 1 < ntok ? s[n][1] * scale_log2_ : -INFINITY;
+      s[n][2] = t0 < ntok ? s[n][2] * scale_log2_ : -INFINITY;
+      s[n][3] = t0 + 1 < ntok ? s[n][3] * scale_log2_ : -INFINITY;
+      x0 = fmaxf(x0, fmaxf(s[n][0], s[n][1]));
+      x1 = fmaxf(x1, fmaxf(s[n][2], s[n][3]));
+    }
+#pragma unroll
+    for (int mask = 1; mask < 4; mask <<= 1) {
+      x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, mask));
+      x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, mask));
+    }
+    const float n0 = fmaxf(m0_, x0), n1 = fmaxf(m1_, x1);
+    const float a0 = ex2(m0_ - n0), a1 = ex2(m1_ - n1);
+    m0_ = n0;
+    m1_ = n1;
+    uint32_t pa[NH][4];
+    float add0 = 0.f, add1 = 0.f;
+#pragma unroll
+    for (int n = 0; n < NN; ++n) {
+      const float p0 = ex2(s[n][0] - n0), p1 = ex2(s[n][1] - n0);
+      const float p2 = ex2(s[n][2] - n1), p3 = ex2(s[n][3] - n1);
+      add0 += p0 + p1;
+      add1 += p2 + p3;
+      pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(p0, p1);
+      pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+    }
+    l0 = l0 * a0 + add0;
+    l1 = l1 * a1 + add1;
+    if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        o[j][0] *= a0;
+        o[j][1] *= a0;
+        o[j][2] *= a1;
+        o[j][3] *= a1;
+      }
+    }
+    // V rows as B operands (transposed): one ldmatrix.x4 gives two d tiles
+    // x one 16-token k step.  V rows past ntok may hold anything; their P is
+    // 0 and their values are zeroed here so that 0 * NaN cannot occur.
+    const int vt = (lane & 7) + (((lane >> 3) & 1) << 3);
+    const int vc = lane >> 4;
+#pragma unroll
+    for (int u = 0; u < NH; ++u) {
+      const int base = m0 + 16 * u;
+      uint32_t mk0 = 0xffffffffu, mk1 = 0xffffffffu;
+      if (base + 16 > ntok) {
+        mk0 = (base + 2 * c < ntok ? 0x0000ffffu : 0u) | (base + 2 * c + 1 < ntok ? 0xffff0000u : 0u);
+        mk1 = (base + 2 * c + 8 < ntok ? 0x0000ffffu : 0u) |
+              (base + 2 * c + 9 < ntok ? 0xffff0000u : 0u);
+      }
+#pragma unroll
+      for (int jj = 0; jj < NJ / 2; ++jj) {
+        uint32_t b[4];
+        ldsm_x4_trans(b, row_addr<TL>(vp, base + vt, 2 * jj + vc, p, h, col_bytes));
+        b[0] &= mk0;
+        b[1] &= mk1;
+        b[2] &= mk0;
+        b[3] &= mk1;
+        mma_16816(o[2 * jj], pa[u], b[0], b[1]);
+        mma_16816(o[2 * jj + 1], pa[u], b[2], b[3]);
+      }
+    }
+  }
+
+  template <bool TL>
+  __device__ __forceinline__ void page_t(const unsigned char *kp, const unsigned char *vp,
+                                         int ntok, const Params &p, int h, int col_bytes,
+                                         int lane) {
+    int m0 = 0;
+    for (; m0 + 16 < ntok; m0 += 32) chunk<2, TL>(kp, vp, m0, ntok, p, h, col_bytes, lane);
+    if (m0 < ntok) chunk<1, TL>(kp, vp, m0, ntok, p, h, col_bytes, lane);
+  }
+
+  __device__ __forceinline__ void page(const unsigned char *kp, const unsigned char *vp,
+                                       int ntok, const Params &p, int h, int col_bytes,
+                                       int lane) {
+    if (p.tile)
+      page_t<true>(kp, vp, ntok, p, h, col_bytes, lane);
+    else
+      page_t<false>(kp, vp, ntok, p, h, col_bytes, lane);
+  }
+
+  // End of a segment: out[...] directly (n_contrib == 1) or this CTA's
+  // normalised partial for the merge kernel.
+  template <typename Tout>
+  __device__ __forceinline__ void flush(const Params &p, const PageDesc &d, int hq0, int nh,
+                                        int c_idx, int lane) {
+    (void)nh;
+    const int r = lane >> 2, c = lane & 3;
+    float L0 = l0, L1 = l1;
+#pragma unroll
+    for (int mask = 1; mask < 4; mask <<= 1) {
+      L0 += __shfl_xor_sync(0xffffffffu, L0, mask);
+      L1 += __shfl_xor_sync(0xffffffffu, L1, mask);
+    }
+    const float i0 = seg_bad ? 0.f : 1.f / L0, i1 = seg_bad ? 0.f : 1.f / L1;
+    if (d.n_contrib == 1) {
+      const int64_t row0 = ((int64_t)d.seq * p.num_q_heads + hq0 + r) * D;
+      const int64_t row1 = row0 + 8 * D;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        Elem<Tout>::store2(p.out, row0 + 8 * j + 2 * c, o[j][0] * i0, o[j][1] * i0);
+        Elem<Tout>::store2(p.out, row1 + 8 * j + 2 * c, o[j][2] * i1, o[j][3] * i1);
+      }
+      return;
+    }
+    const int64_t prow = ((int64_t)c_idx * 2 + (d.slot_bits & 1)) * p.num_q_heads + hq0;
+    if (c == 0) {
+      *reinterpret_cast<float2 *>(p.part_ml + (prow + r) * 2) =
+          make_float2(m0_, seg_bad ? -1.f : L0);
+      *reinterpret_cast<float2 *>(p.part_ml + (prow + r + 8) * 2) =
+          make_float2(m1_, seg_bad ? -1.f : L1);
+    }
+    float *orow0 = p.part_o + (prow + r) * D;
+    float *orow1 = p.part_o + (prow + r + 8) * D;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      *reinterpret_cast<float2 *>(orow0 + 8 * j + 2 * c) = make_float2(o[j][0] * i0, o[j][1] * i0);
+      *reinterpret_cast<float2 *>(orow1 + 8 * j + 2 * c) = make_float2(o[j][2] * i1, o[j][3] * i1);
+    }
+    // merged later by the merge kernel
+  }
+};
+
+// ===========================================================================
 // fp32 consumer: CUDA-core FMAs for G query heads of one KV head.
 // ===========================================================================
 template <typename T, int D, int G>
@@ -848,7 +1060,9 @@ __device__ __forceinline__ void write_new_rows(const Params &p, int32_t s, int64
 
 // ===========================================================================
 // The kernel.  T = element type; D = head_dim; G = query heads per KV head
-// for the fp32 consumer (unused, 0, for bf16); NCW = consumer warps.
+// for the fp32 consumer; for bf16, G = 16 selects the head-row consumer (16
+// heads per warp) and G = 0 the token-row one (up to 8 heads per warp);
+// NCW = consumer warps.
 // ===========================================================================
 template <typename T, int D, int G, int NCW>
 __global__ void __launch_bounds__((NCW + 1) * 32, 1)
@@ -860,7 +1074,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 "header region");
   static_assert(sizeof(Shared) % 16 == 0 && sizeof(PageDesc) % 16 == 0,
                 "descriptors and score buffers need 16-byte alignment");
-  using Cons = typename std::conditional<kMma, MmaConsumer<D>,
+  using MmaCons =
+      typename std::conditional<G == 16, HeadRowConsumer<D>, MmaConsumer<D>>::type;
+  using Cons = typename std::conditional<kMma, MmaCons,
                                          FmaConsumer<T, D, (G > 0 ? G : 1)>>::type;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Shared &sh = *reinterpret_cast<Shared *>(smem_raw);

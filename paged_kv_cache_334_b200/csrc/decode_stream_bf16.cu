@@ -1,25 +1,32 @@
 // bf16 instantiations of the persistent paged decode kernel (tensor-core
-// consumers; any group size, NCW = KV heads x ceil(group / 8) warps).
+// consumers): groups that are a multiple of 16 query heads use the head-row
+// consumer (16 heads per warp), others the token-row consumer (up to 8 heads
+// per warp); NCW = KV heads x warps per KV head, 4, 8 or 16.
 #include "decode_stream.cuh"
 
 namespace pa {
 namespace stream {
 
-template <int D>
+template <int D, int CONS>
 static cudaError_t launch_ncw(const Params &p, int ncw, size_t smem, cudaStream_t stream) {
   switch (ncw) {
-    case 4: return launch_one<__nv_bfloat16, D, 0, 4>(p, smem, stream);
-    case 8: return launch_one<__nv_bfloat16, D, 0, 8>(p, smem, stream);
-    case 16: return launch_one<__nv_bfloat16, D, 0, 16>(p, smem, stream);
+    case 4: return launch_one<__nv_bfloat16, D, CONS, 4>(p, smem, stream);
+    case 8: return launch_one<__nv_bfloat16, D, CONS, 8>(p, smem, stream);
+    case 16: return launch_one<__nv_bfloat16, D, CONS, 16>(p, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_bf16(const Params &p, int head_dim, int group, int hkv, size_t smem,
                         cudaStream_t stream) {
-  const int ncw = hkv * (group > 8 ? group / 8 : 1);
-  if (head_dim == 64) return launch_ncw<64>(p, ncw, smem, stream);
-  if (head_dim == 128) return launch_ncw<128>(p, ncw, smem, stream);
+  (void)group;
+  const int ncw = hkv * p.warps_per_kv;
+  const bool rows = p.heads_per_warp == 16;
+  if (head_dim == 64)
+    return rows ? launch_ncw<64, 16>(p, ncw, smem, stream) : launch_ncw<64, 0>(p, ncw, smem, stream);
+  if (head_dim == 128)
+    return rows ? launch_ncw<128, 16>(p, ncw, smem, stream)
+                : launch_ncw<128, 0>(p, ncw, smem, stream);
   return cudaErrorInvalidValue;
 }
 

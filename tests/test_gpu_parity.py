@@ -365,6 +365,14 @@ STREAM_SHAPES = [
     (wl.DTYPE_BF16, 8, 8, 128, 1),
     (wl.DTYPE_BF16, 32, 8, 128, 256),
     (wl.DTYPE_F32, 4, 4, 128, 4),
+    # groups of 16k heads: 16 query heads per warp on the MMA row side
+    (wl.DTYPE_BF16, 64, 4, 128, 16),
+    (wl.DTYPE_BF16, 64, 1, 128, 32),
+    (wl.DTYPE_BF16, 64, 1, 64, 32),
+    (wl.DTYPE_BF16, 128, 2, 128, 16),
+    (wl.DTYPE_BF16, 64, 1, 128, 8),
+    (wl.DTYPE_BF16, 256, 4, 128, 16),
+    (wl.DTYPE_BF16, 32, 2, 128, 8),
 ]
 
 
