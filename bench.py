@@ -53,7 +53,7 @@ METRIC = "decode-attention KV GB/s & fraction of B200 HBM peak; seq-tokens/s per
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc")
 # sources that define the decode kernel's code and launch shape
-DECODE_SOURCES = ("decode_stream.cuh", "decode_stream_bf16.cu", "decode_stream_f32.cu",
+DECODE_SOURCES = ("decode_stream.cuh", "decode_stream_bf16.cu", "decode_stream_f32.cu", "sm100_ptx.cuh",
                   "pa_common.cuh", "pa_launch.h", "api.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.md")
 

@@ -72,6 +72,9 @@ typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
 /* A pipeline wait inside a kernel gave up (never expected; the outputs of
  * that call are incomplete and its workspace must be zero-filled again). */
 #define PA_DEVERR_TIMEOUT 8
+/* pa_decode_shared_prefix: a sequence whose table does not start with the
+ * shared prefix pages or whose context is shorter than the prefix. */
+#define PA_DEVERR_PREFIX 16
 
 /* Shape of the physical KV cache pool ([teaching] section "First define a
  * simple KV cache layout": [num_blocks, block_size, num_heads, head_dim],
@@ -194,6 +197,40 @@ pa_status pa_forward_decode(const pa_cache_desc *cache, void *out, const void *q
                             int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
                             float scale, void *workspace, size_t workspace_bytes,
                             int32_t *err_word, pa_stream_t stream);
+
+/*
+ * pa_decode_shared_prefix -- pa_decode for a batch whose sequences all start
+ * with the same pages (a shared prompt prefix).
+ *
+ * [serving] section 6 "Prefix caching": requests with a common prefix share
+ * its KV pages.  Here the prefix is the first prefix_blocks entries of
+ * block_tables row 0, and every sequence's table must start with the same
+ * entries and every context_lens[b] must be >= prefix_blocks * block_size.
+ * out is the same as pa_decode's (up to rounding); internally the suffix
+ * past the prefix is decoded per sequence and the prefix, read by every
+ * (sequence, query head) of a KV head, runs as dense tensor-core tiles of
+ * 128 rows x 128 prefix tokens (tcgen05) whose epilogue merges the two
+ * parts with the running-max rescaling ([route] section "The core idea of
+ * high-performance PagedAttention").
+ *
+ * A sequence whose table or length does not contain the prefix sets
+ * PA_DEVERR_PREFIX and its output is zeroed; a bad prefix block id sets
+ * PA_DEVERR_BLOCK_ID and zeroes every output.  Shapes: bf16, head_dim 64
+ * or 128, query heads per KV head dividing 128, block_size 8..128 (a power
+ * of two), prefix_blocks <= 2048, and a shape pa_decode serves with its
+ * persistent kernel (else PA_ERR_UNSUPPORTED).  prefix_blocks == 0 is
+ * pa_decode.  workspace: at least pa_decode_shared_prefix_workspace_bytes
+ * bytes, 256-byte aligned, zero-filled before first use (as pa_decode's).
+ */
+size_t pa_decode_shared_prefix_workspace_bytes(const pa_cache_desc *cache, int32_t batch,
+                                               int32_t num_q_heads, int32_t max_blocks_per_seq,
+                                               int32_t prefix_blocks);
+pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const void *q,
+                                  const void *key_cache, const void *value_cache,
+                                  const int32_t *block_tables, const int32_t *context_lens,
+                                  int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                                  int32_t prefix_blocks, float scale, void *workspace,
+                                  size_t workspace_bytes, int32_t *err_word, pa_stream_t stream);
 
 /*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device

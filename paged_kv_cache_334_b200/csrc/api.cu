@@ -274,12 +274,17 @@ void set_last_error_message(const char *msg) { snprintf(g_msg, sizeof g_msg, "%s
 }  // namespace pa
 
 // pa_decode, and pa_forward_decode when k_new / v_new / slot_mapping are set.
+// With prefix_blocks > 0 (pa_decode_shared_prefix, persistent kernel only):
+// the first prefix_blocks pages of every sequence are left out and each
+// (sequence, query head) result goes to seq_ml / seq_o as a partial.
 static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *q, void *key_cache,
                       void *value_cache, const void *k_new, const void *v_new,
                       const int64_t *slot_mapping, const int32_t *block_tables,
                       const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
                       int32_t max_blocks_per_seq, float scale, void *workspace,
-                      size_t workspace_bytes, int32_t *err_word, pa_stream_t stream) {
+                      size_t workspace_bytes, int32_t *err_word, pa_stream_t stream,
+                      int32_t prefix_blocks = 0, float *seq_ml = nullptr,
+                      float *seq_o = nullptr) {
   pa_status s = check_decode_common(cache, q, key_cache, value_cache, block_tables,
                                     context_lens, batch, num_q_heads,
                                     max_blocks_per_seq, scale);
@@ -298,6 +303,8 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
     return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
   char *ws = static_cast<char *>(workspace);
+  if (prefix_blocks > 0 && !w.stream)
+    return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs the persistent kernel's shapes%s");
   if (w.stream) {
     StreamPlan sp = plan_stream(cache, num_q_heads);
     const int sms = device_sm_count();
@@ -313,8 +320,10 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
     p.k_new = k_new;
     p.v_new = v_new;
     p.slot_mapping = slot_mapping;
-    p.block_tables = block_tables;
+    p.block_tables = block_tables + prefix_blocks;
     p.context_lens = context_lens;
+    p.seq_ml = seq_ml;
+    p.seq_o = seq_o;
     p.part_ml = reinterpret_cast<float *>(ws + w.part_max);
     p.part_o = reinterpret_cast<float *>(ws + w.part_out);
     p.seq_merge = reinterpret_cast<int32_t *>(ws + w.counters);
@@ -323,7 +332,9 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
     p.block_size = cache->block_size;
     p.num_kv_heads = cache->num_kv_heads;
     p.num_q_heads = num_q_heads;
-    p.max_blocks = max_blocks_per_seq;
+    p.max_blocks = max_blocks_per_seq - prefix_blocks;
+    p.table_stride = max_blocks_per_seq;
+    p.tok_offset = prefix_blocks * cache->block_size;
     p.batch = batch;
     p.vbs = sp.vbs;
     p.log2_vbs = sp.log2_vbs;
@@ -474,6 +485,120 @@ pa_status pa_forward_decode(const pa_cache_desc *cache, void *out, const void *q
   return decode_impl(cache, out, q, key_cache, value_cache, k_new, v_new, slot_mapping,
                      block_tables, context_lens, batch, num_q_heads, max_blocks_per_seq, scale,
                      workspace, workspace_bytes, err_word, stream);
+}
+
+size_t pa_decode_shared_prefix_workspace_bytes(const pa_cache_desc *cache, int32_t batch,
+                                               int32_t num_q_heads, int32_t max_blocks_per_seq,
+                                               int32_t prefix_blocks) {
+  if (check_cache(cache) != PA_OK || batch < 0 || num_q_heads <= 0 ||
+      num_q_heads % cache->num_kv_heads != 0 || prefix_blocks < 0 ||
+      max_blocks_per_seq < prefix_blocks)
+    return 0;
+  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+  const size_t rows = (size_t)batch * num_q_heads;
+  return w.total + round_up(rows * 2 * sizeof(float)) +
+         round_up(rows * (size_t)cache->head_dim * sizeof(float));
+}
+
+pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const void *q,
+                                  const void *key_cache, const void *value_cache,
+                                  const int32_t *block_tables, const int32_t *context_lens,
+                                  int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                                  int32_t prefix_blocks, float scale, void *workspace,
+                                  size_t workspace_bytes, int32_t *err_word, pa_stream_t stream) {
+  pa_status s = check_decode_common(cache, q, key_cache, value_cache, block_tables,
+                                    context_lens, batch, num_q_heads, max_blocks_per_seq, scale);
+  if (s != PA_OK) return s;
+  if (prefix_blocks < 0 || prefix_blocks > max_blocks_per_seq)
+    return fail(PA_ERR_INVALID_ARG, "prefix_blocks must be in [0, max_blocks_per_seq]%s (%lld)",
+                "", prefix_blocks);
+  if (prefix_blocks == 0)
+    return pa_decode(cache, out, q, key_cache, value_cache, block_tables, context_lens, batch,
+                     num_q_heads, max_blocks_per_seq, scale, workspace, workspace_bytes,
+                     err_word, stream);
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  const int32_t bs = cache->block_size;
+  if (cache->dtype != PA_DTYPE_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode is bf16 only%s");
+  if (group > 128 || 128 % group != 0)
+    return fail(PA_ERR_UNSUPPORTED,
+                "shared-prefix decode needs 128 %% (query heads per KV head) == 0%s (%lld)", "",
+                group);
+  if (bs < 8 || bs > 128)
+    return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs block_size in [8, 128]%s (%lld)",
+                "", bs);
+  if (prefix_blocks > pa::kMaxPrefixBlocks)
+    return fail(PA_ERR_UNSUPPORTED, "more than 2048 shared prefix blocks%s (%lld)", "",
+                prefix_blocks);
+  if (batch == 0) return PA_OK;
+  if ((s = check_ptr(out, "out")) != PA_OK) return s;
+  const size_t need = pa_decode_shared_prefix_workspace_bytes(cache, batch, num_q_heads,
+                                                              max_blocks_per_seq, prefix_blocks);
+  if (workspace_bytes < need)
+    return fail(PA_ERR_INVALID_ARG, "workspace too small%s: need %lld bytes", "", (long long)need);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
+  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+  const size_t rows = (size_t)batch * num_q_heads;
+  char *ws = static_cast<char *>(workspace);
+  float *seq_ml = reinterpret_cast<float *>(ws + w.total);
+  float *seq_o = reinterpret_cast<float *>(ws + w.total + round_up(rows * 2 * sizeof(float)));
+  // 1. the suffix of every sequence, as one partial per (sequence, head)
+  s = decode_impl(cache, out, q, const_cast<void *>(key_cache), const_cast<void *>(value_cache),
+                  nullptr, nullptr, nullptr, block_tables, context_lens, batch, num_q_heads,
+                  max_blocks_per_seq, scale, workspace, w.total, err_word, stream, prefix_blocks,
+                  seq_ml, seq_o);
+  if (s != PA_OK) return s;
+  // 2. the shared prefix on the tensor cores, folded with the suffix partials
+  pa::PrefixParams pp{};
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable%s");
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim, (cuuint64_t)num_q_heads,
+                                (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)cache->head_dim * 2,
+                                   (cuuint64_t)num_q_heads * cache->head_dim * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(128 / group)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&pp.tmap_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
+  }
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim,
+                                (cuuint64_t)cache->num_blocks * (cuuint64_t)bs,
+                                (cuuint64_t)cache->num_kv_heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)cache->num_kv_heads * cache->head_dim * 2,
+                                   (cuuint64_t)cache->head_dim * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)bs, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    for (int which = 0; which < 2; ++which) {
+      if (fn(which ? &pp.tmap_v : &pp.tmap_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(which ? value_cache : key_cache), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return fail(PA_ERR_CUDA, "cannot describe the caches for the tensor copies%s");
+    }
+  }
+  pp.block_tables = block_tables;
+  pp.context_lens = context_lens;
+  pp.seq_ml = seq_ml;
+  pp.seq_o = seq_o;
+  pp.out = out;
+  pp.err_word = err_word;
+  pp.batch = batch;
+  pp.num_q_heads = num_q_heads;
+  pp.num_kv_heads = cache->num_kv_heads;
+  pp.group = group;
+  pp.block_size = bs;
+  pp.table_stride = max_blocks_per_seq;
+  pp.prefix_blocks = prefix_blocks;
+  pp.num_blocks = cache->num_blocks;
+  pp.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = pa::launch_prefix(pp, cache->head_dim, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(e));
+  return PA_OK;
 }
 
 pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,

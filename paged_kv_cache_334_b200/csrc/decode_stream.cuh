@@ -54,11 +54,11 @@
 
 #include "pa_common.cuh"
 #include "pa_launch.h"
+#include "sm100_ptx.cuh"
 
 namespace pa {
 namespace stream {
 
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legitimate wait
 constexpr int kFirst = 1, kLast = 2, kBad = 4;
 // Block tables up to this size are prefetched into L2 at kernel start.
 constexpr uint64_t kTablePrefetchMax = 16ull << 20;
@@ -69,117 +69,10 @@ struct alignas(16) PageDesc {
   int32_t c_first, slot_bits, pb, toff;
 };
 
-// ---------------------------------------------------------------------------
-// PTX wrappers: mbarrier, 1-D bulk copy (no multicast), warp-level MMA.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
-      "selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait; false when kWaitLimitNs passes or the CTA's abort flag is set.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int32_t *abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15) == 0) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) return false;
-    }
-  }
-}
-__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gsrc, uint32_t bytes,
-                                         uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-// Tiled tensor copy of one box (coordinates innermost first), no multicast.
-__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, int x, int y,
-                                            int z, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
-      "[%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
-// Hints (no effect on results): bring a tensor map into the descriptor cache,
-// a byte range of global memory into L2 (16-byte aligned, multiple of 16).
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-__device__ __forceinline__ void prefetch_l2(const void *g, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(g), "r"(bytes) : "memory");
-}
-// Orders this thread's earlier generic-proxy global stores before its later
-// async-proxy (bulk / tensor copy) accesses of global memory.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-// D += A (16x16, row) * B (16x8, col), bf16 inputs, fp32 accumulation.
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                          uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-// Two fp32 -> packed bf16x2 (round to nearest even); `lo` in the low half.
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-// 2^x with the hardware approximation (inputs here are <= 0: softmax
-// weights; results below the normal range flush to zero).
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
+// Tokens of sequence s this call attends to (all of them, or the suffix
+// past the shared prefix in suffix mode).
+__device__ __forceinline__ int32_t visible_len(const Params &p, int s) {
+  return p.context_lens[s] - p.tok_offset;
 }
 
 __device__ __forceinline__ int32_t vpages_of(int32_t ctx, const Params &p) {
@@ -459,6 +352,23 @@ struct MmaConsumer {
                    : make_float4(r0 * inv, r1 * inv, hi0 * inv, hi1 * inv);
     }
     if (d.n_contrib == 1) {
+      if (p.seq_o != nullptr) {
+        // suffix mode: the sequence's result as a partial for the prefix pass
+        const int64_t row = (int64_t)d.seq * p.num_q_heads + hq0;
+        if (g == 0) {
+          if (2 * t < nh)
+            reinterpret_cast<float2 *>(p.seq_ml)[row + 2 * t] = make_float2(m0_, seg_bad ? -1.f : L0);
+          if (2 * t + 1 < nh)
+            reinterpret_cast<float2 *>(p.seq_ml)[row + 2 * t + 1] =
+                make_float2(m1_, seg_bad ? -1.f : L1);
+        }
+        if (hh < nh) {
+#pragma unroll
+          for (int k = 0; k < KS; ++k)
+            *reinterpret_cast<float4 *>(p.seq_o + (row + hh) * D + k * 16 + dcol) = v[k];
+        }
+        return;
+      }
       if (hh < nh) {
         const int64_t row = ((int64_t)d.seq * p.num_q_heads + hq0 + hh) * D;
 #pragma unroll
@@ -668,6 +578,22 @@ struct HeadRowConsumer {
       L1 += __shfl_xor_sync(0xffffffffu, L1, mask);
     }
     const float i0 = seg_bad ? 0.f : 1.f / L0, i1 = seg_bad ? 0.f : 1.f / L1;
+    if (d.n_contrib == 1 && p.seq_o != nullptr) {
+      // suffix mode: the sequence's result as a partial for the prefix pass
+      const int64_t row = (int64_t)d.seq * p.num_q_heads + hq0 + r;
+      if (c == 0) {
+        reinterpret_cast<float2 *>(p.seq_ml)[row] = make_float2(m0_, seg_bad ? -1.f : L0);
+        reinterpret_cast<float2 *>(p.seq_ml)[row + 8] = make_float2(m1_, seg_bad ? -1.f : L1);
+      }
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        *reinterpret_cast<float2 *>(p.seq_o + row * D + 8 * j + 2 * c) =
+            make_float2(o[j][0] * i0, o[j][1] * i0);
+        *reinterpret_cast<float2 *>(p.seq_o + (row + 8) * D + 8 * j + 2 * c) =
+            make_float2(o[j][2] * i1, o[j][3] * i1);
+      }
+      return;
+    }
     if (d.n_contrib == 1) {
       const int64_t row0 = ((int64_t)d.seq * p.num_q_heads + hq0 + r) * D;
       const int64_t row1 = row0 + 8 * D;
@@ -907,7 +833,7 @@ struct PageWalker {
       cw_ctx = in ? shc->ctx_c[cw + lane] : 0;
       cw_slot = in ? shc->slot_c[cw + lane] : -1;
     } else {
-      cw_ctx = in ? p.context_lens[cw + lane] : 0;
+      cw_ctx = in ? visible_len(p, cw + lane) : 0;
       cw_slot = (in && p.slot_mapping != nullptr) ? p.slot_mapping[cw + lane] : -1;
     }
   }
@@ -946,7 +872,7 @@ struct PageWalker {
   __device__ __forceinline__ int32_t load_table(const Params &p, int32_t seq, int32_t lb,
                                                 int lane) const {
     const int32_t e = lb + lane;
-    return (e < p.max_blocks) ? p.block_tables[(int64_t)seq * p.max_blocks + e] : -1;
+    return (e < p.max_blocks) ? p.block_tables[(int64_t)seq * p.table_stride + e] : -1;
   }
   // Start loading the window after the current one: the rest of a long
   // sequence, else the next sequence with visible pages, looked up in the
@@ -1068,7 +994,8 @@ template <typename T, int D, int G, int NCW>
 __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     decode_stream_kernel(const __grid_constant__ Params p) {
   constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
-  constexpr int kScoreFloats = kMma ? 1 : FmaConsumer<T, D, (G > 0 ? G : 1)>::E;
+  constexpr int kFmaG = kMma ? 1 : (G > 0 ? G : 1);  // fp32 consumer's group
+  constexpr int kScoreFloats = kMma ? 1 : FmaConsumer<T, D, kFmaG>::E;
   static_assert(sizeof(Shared) + sizeof(PageDesc) * kMaxStages * kMaxPPS +
                         sizeof(float) * NCW * kScoreFloats <= kHdrBytes,
                 "header region");
@@ -1076,8 +1003,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 "descriptors and score buffers need 16-byte alignment");
   using MmaCons =
       typename std::conditional<G == 16, HeadRowConsumer<D>, MmaConsumer<D>>::type;
-  using Cons = typename std::conditional<kMma, MmaCons,
-                                         FmaConsumer<T, D, (G > 0 ? G : 1)>>::type;
+  using Cons = typename std::conditional<kMma, MmaCons, FmaConsumer<T, D, kFmaG>>::type;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Shared &sh = *reinterpret_cast<Shared *>(smem_raw);
   PageDesc *descs = reinterpret_cast<PageDesc *>(smem_raw + sizeof(Shared));
@@ -1133,7 +1059,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     // one scan gives both the total and every sequence's first page
     int32_t ctx = 0;
     if (tid < p.batch) {
-      ctx = p.context_lens[tid];
+      ctx = visible_len(p, tid);
       if (cached) {
         sh.ctx_c[tid] = ctx;
         sh.slot_c[tid] = (p.slot_mapping != nullptr) ? p.slot_mapping[tid] : -1;
@@ -1157,7 +1083,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       const int s = base + tid;
       int32_t ctx = 0;
       if (s < p.batch) {
-        ctx = p.context_lens[s];
+        ctx = visible_len(p, s);
         if (cached) {
           sh.ctx_c[s] = ctx;
           sh.slot_c[s] = (p.slot_mapping != nullptr) ? p.slot_mapping[s] : -1;
@@ -1174,7 +1100,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       int64_t run = 0;
       for (int base = 0; base < p.batch; base += blockDim.x) {
         const int s = base + tid;
-        const int64_t v = (s < p.batch) ? vpages_of(p.context_lens[s], p) : 0;
+        const int64_t v = (s < p.batch) ? vpages_of(visible_len(p, s), p) : 0;
         int64_t tot;
         const int64_t P = run + block_exclusive_scan(v, sh.red, &tot);
         if (v > 0 && P <= start && start < P + v) {
@@ -1398,19 +1324,29 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 
   // ---- Sequences with no visible page: zero output (and flag bad lengths).
   __syncthreads();
+
   for (int s = c; s < p.batch; s += p.grid) {
+    if (vpages_of(visible_len(p, s), p) > 0) continue;
     const int32_t ctx = p.context_lens[s];
-    if (vpages_of(ctx, p) > 0) continue;
     if (tid == 0) {
       reinterpret_cast<int4 *>(p.seq_merge)[s] = make_int4(0, 0, 0, 0);
-      if (ctx < 0 || (int64_t)ctx > (int64_t)p.max_blocks * p.block_size)
+      if (ctx < 0 || (int64_t)ctx > (int64_t)p.table_stride * p.block_size)
         set_error(p.err_word, PA_DEVERR_CONTEXT_LEN);
       // fused write: no visible position for the new token
       if (p.slot_mapping != nullptr && p.slot_mapping[s] >= 0)
         set_error(p.err_word, PA_DEVERR_SLOT);
     }
     const int64_t n = (int64_t)p.num_q_heads * D;
-    for (int64_t x = tid; x < n; x += blockDim.x) Elem<T>::store1(p.out, (int64_t)s * n + x, 0.f);
+    if (p.seq_o != nullptr) {
+      // empty suffix: a partial that weighs nothing
+      for (int64_t x = tid; x < n; x += blockDim.x) p.seq_o[(int64_t)s * n + x] = 0.f;
+      for (int x = tid; x < p.num_q_heads; x += blockDim.x)
+        reinterpret_cast<float2 *>(p.seq_ml)[(int64_t)s * p.num_q_heads + x] =
+            make_float2(-INFINITY, 0.f);
+    } else {
+      for (int64_t x = tid; x < n; x += blockDim.x)
+        Elem<T>::store1(p.out, (int64_t)s * n + x, 0.f);
+    }
   }
 }
 
@@ -1452,6 +1388,9 @@ cudaError_t launch_one(const Params &p, size_t smem, cudaStream_t stream) {
 template <typename Tout, int D>
 __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Params p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // a following kernel launched programmatically (the shared-prefix pass)
+  // may start; it waits for this grid before reading what it writes
+  asm volatile("griddepcontrol.launch_dependents;");
   const int slices = p.num_q_heads / p.heads_per_warp;
   const int seq = blockIdx.x / slices;
   const int hq0 = (blockIdx.x % slices) * p.heads_per_warp;
@@ -1508,6 +1447,15 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Para
     }
     const float inv = 1.f / W;
     const int64_t e = (orow + h) * D + d0;
+    if (p.seq_o != nullptr) {
+      // suffix mode: the merged result as a partial for the prefix pass
+      *reinterpret_cast<float4 *>(p.seq_o + e) =
+          bad ? make_float4(0.f, 0.f, 0.f, 0.f)
+              : make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      if (d0 == 0)
+        reinterpret_cast<float2 *>(p.seq_ml)[orow + h] = make_float2(M, bad ? -1.f : W);
+      continue;
+    }
     Elem<Tout>::store1(p.out, e + 0, bad ? 0.f : acc.x * inv);
     Elem<Tout>::store1(p.out, e + 1, bad ? 0.f : acc.y * inv);
     Elem<Tout>::store1(p.out, e + 2, bad ? 0.f : acc.z * inv);

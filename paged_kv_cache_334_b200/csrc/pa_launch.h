@@ -63,6 +63,14 @@ struct Params {
   float *part_o;      // [kMaxGrid * 2][Hq][D]: normalised partial output
   int32_t *seq_merge;  // [batch][4]: first contributing CTA, contributors, slot of the first
   int32_t *err_word;
+  // Suffix mode (shared-prefix decode): the first tok_offset tokens of every
+  // sequence are left out (block_tables then points tok_offset / block_size
+  // entries into each row, rows table_stride entries apart, max_blocks of
+  // them usable) and each (sequence, query head) result goes to seq_ml (max
+  // in log2 units, normaliser) and seq_o (normalised output) instead of out.
+  float *seq_ml;
+  float *seq_o;
+  int32_t tok_offset, table_stride;
   int32_t num_blocks, block_size, num_kv_heads, num_q_heads, max_blocks, batch;
   int32_t vbs, log2_vbs, log2_vpp;  // virtual page tokens; log2 of pages per block
   int32_t row_bytes;                // one token row, all KV heads (global layout)
@@ -89,6 +97,28 @@ cudaError_t launch_f32(const Params &p, int head_dim, int group, int hkv, size_t
                        cudaStream_t stream);
 
 }  // namespace stream
+
+// Arguments of the shared-prefix kernel (prefix.cu).
+constexpr int kMaxPrefixBlocks = 2048;
+struct PrefixParams {
+  // 3-D tiled views: q (head_dim, query head, sequence) with boxes of 64 x
+  // group x 128 / group, and the caches (head_dim, token row, KV head) with
+  // boxes of 64 x block_size x 1; all with 128-byte swizzle.
+  CUtensorMap tmap_q;
+  CUtensorMap tmap_k;
+  CUtensorMap tmap_v;
+  const int32_t *block_tables;  // rows of table_stride entries; the prefix is row 0's first entries
+  const int32_t *context_lens;
+  const float *seq_ml;          // [batch][Hq] (max in log2 units, normaliser) of each suffix
+  const float *seq_o;           // [batch][Hq][D] normalised suffix output
+  void *out;
+  int32_t *err_word;
+  int32_t batch, num_q_heads, num_kv_heads, group, block_size, table_stride, prefix_blocks,
+      num_blocks;
+  float scale_log2;
+};
+size_t prefix_smem_bytes(int head_dim);
+cudaError_t launch_prefix(const PrefixParams &p, int head_dim, cudaStream_t stream);
 
 // Query heads handled together by one CTA for a GQA group of `group` heads.
 int decode_head_tile(int group);

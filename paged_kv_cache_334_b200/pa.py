@@ -35,11 +35,14 @@ PA_DTYPE_BF16 = 1
 PA_DEVERR_BLOCK_ID = 1
 PA_DEVERR_CONTEXT_LEN = 2
 PA_DEVERR_SLOT = 4
+PA_DEVERR_TIMEOUT = 8
+PA_DEVERR_PREFIX = 16
 
 EXPORTED_SYMBOLS = (
     "pa_version", "pa_status_string", "pa_last_error_message", "pa_write_kv_cache",
     "pa_decode_workspace_bytes", "pa_decode", "pa_decode_splitk", "pa_reduce",
-    "pa_decode_noalloc", "pa_forward_decode",
+    "pa_decode_noalloc", "pa_forward_decode", "pa_decode_shared_prefix",
+    "pa_decode_shared_prefix_workspace_bytes",
 )
 
 # Size of the fixed device scratch array pa_decode_noalloc uses.
@@ -95,6 +98,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_forward_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, i32, i32, i32, f32, P, sz,
                                       P, P]
     lib.pa_forward_decode.restype = ctypes.c_int
+    lib.pa_decode_shared_prefix_workspace_bytes.argtypes = [D, i32, i32, i32, i32]
+    lib.pa_decode_shared_prefix_workspace_bytes.restype = sz
+    lib.pa_decode_shared_prefix.argtypes = [D, P, P, P, P, P, P, i32, i32, i32, i32, f32, P, sz,
+                                            P, P]
+    lib.pa_decode_shared_prefix.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -228,6 +236,37 @@ def pa_forward_decode(out, q, key_cache, value_cache, k_new, v_new, slot_mapping
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
         _dev(workspace, "workspace"), int(workspace.numel() * workspace.element_size()),
         _dev(err_word, "err_word", torch.int32), _stream(stream)))
+    return out
+
+
+def pa_decode_shared_prefix(out, q, key_cache, value_cache, block_tables, context_lens,
+                            prefix_blocks: int, scale: Optional[float] = None,
+                            workspace: Optional[torch.Tensor] = None,
+                            err_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pa_decode for a batch whose tables all start with the same
+    prefix_blocks pages (see include/pa.h)."""
+    lib = load()
+    desc = cache_desc(key_cache)
+    B, Hq, Dq = q.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dq)
+    if workspace is None:
+        n = int(lib.pa_decode_shared_prefix_workspace_bytes(ctypes.byref(desc), B, Hq, MB,
+                                                            int(prefix_blocks)))
+        key = (key_cache.device, n, "prefix")
+        workspace = _workspaces.get(key)
+        if workspace is None:
+            workspace = torch.zeros(max(n, 256), dtype=torch.uint8, device=key_cache.device)
+            _workspaces[key] = workspace
+    _check(lib.pa_decode_shared_prefix(
+        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, int(prefix_blocks),
+        float(scale), _dev(workspace, "workspace"),
+        int(workspace.numel() * workspace.element_size()), _dev(err_word, "err_word", torch.int32),
+        _stream(stream)))
     return out
 
 

@@ -241,13 +241,18 @@ def make_workload(name: str, seed: int = 0, batch: Optional[int] = None) -> Work
 def custom_workload(*, dtype: str, batch: int, num_q_heads: int, num_kv_heads: int,
                     head_dim: int, block_size: int, context_lens, seed: int = 0,
                     slack: float = 0.2, max_blocks: Optional[int] = None,
-                    new_tokens: bool = False) -> Workload:
-    """A workload with explicit context lengths (edge cases, sweeps)."""
+                    new_tokens: bool = False, prefix_blocks: int = 0) -> Workload:
+    """A workload with explicit context lengths (edge cases, sweeps).  With
+    prefix_blocks > 0 every table starts with the same physical blocks (a
+    shared prompt prefix); every context must cover them."""
     rng = np.random.Generator(np.random.PCG64(seed))
     ctx = np.asarray(context_lens, dtype=np.int32)
     need = max([_pages(int(c), block_size) for c in ctx] + [1])
     MB = max_blocks if max_blocks is not None else need
-    tables, NB = _scattered_tables(rng, np.maximum(ctx, 0), block_size, MB, slack=slack)
+    if prefix_blocks:
+        assert all(int(c) >= prefix_blocks * block_size for c in ctx), "context shorter than prefix"
+    tables, NB = _scattered_tables(rng, np.maximum(ctx, 0), block_size, MB, slack=slack,
+                                   prefix_blocks=prefix_blocks)
     NB = max(NB, 1)
     return _finish("custom", dtype, rng, batch, num_q_heads, num_kv_heads, head_dim,
                    block_size, NB, MB, ctx, tables,
