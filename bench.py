@@ -70,9 +70,11 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--step", choices=("fused", "separate"), default="fused",
+    ap.add_argument("--step", choices=("fused", "separate", "prefix"), default="fused",
                     help="fused: one pa_forward_decode call per step (cache write inside the "
-                         "decode kernel); separate: pa_write_kv_cache then pa_decode")
+                         "decode kernel); separate: pa_write_kv_cache then pa_decode; prefix: "
+                         "pa_write_kv_cache then pa_decode_shared_prefix (workloads with a "
+                         "shared prefix)")
     return ap.parse_args(argv)
 
 
@@ -191,6 +193,21 @@ class ClockSampler:
 # measured peaks and ncu traffic
 # ---------------------------------------------------------------------------
 
+def tensor_peak():
+    """Dense bf16 tensor-core peak (burst: the call is timed alone)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "MEASURED_PEAKS.json bf16_tflops (of measured)"
+    except Exception:
+        return 1590.0, "1.59 PFLOP/s fallback (of fallback)"
+
+
+def attention_flops(w) -> float:
+    """QK and PV of every visible (token, query head): 2 * 2 * D flops each."""
+    return 4.0 * float(w.context_lens.sum()) * w.num_q_heads * w.head_dim
+
+
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -306,9 +323,11 @@ def workload_config(w, args):
         "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
         "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
         "context_tokens": int(w.context_lens.sum()), "seed": args.seed,
-        "step": ("pa_forward_decode (newest token of every sequence stored inside the decode "
-                 "kernel, then decode)" if args.step == "fused" else
-                 "pa_write_kv_cache(newest token of every sequence) + pa_decode"),
+        "step": {"fused": "pa_forward_decode (newest token of every sequence stored inside the "
+                          "decode kernel, then decode)",
+                 "separate": "pa_write_kv_cache(newest token of every sequence) + pa_decode",
+                 "prefix": "pa_write_kv_cache(newest token of every sequence) + "
+                           "pa_decode_shared_prefix"}[args.step],
         "l2": "flushed before every timed step (zero-fill then read of 2x L2, outside the events)",
         "parallelism": f"replicas: one independent batch per GPU x{args.gpus}",
     }
@@ -382,9 +401,13 @@ def run_ours(args):
     flush_f32 = flush_buf.view(torch.float32)
     flush_sink = torch.empty((), dtype=torch.float32, device=dev)
     fused = has_new and args.step == "fused"
+    prefix = args.step == "prefix"
+    if prefix and not w.shared_prefix_blocks:
+        raise SystemExit(f"--step prefix needs a workload with a shared prefix, not {w.name}")
     # libpa kernels per step: the persistent decode kernel and its merge
-    # kernel, plus the write kernel when the write is a separate call
-    launches_per_step = 2 + (1 if has_new and not fused else 0)
+    # kernel, plus the write kernel when the write is a separate call, plus
+    # the prefix kernel of the shared-prefix path
+    launches_per_step = 2 + (1 if has_new and not fused else 0) + (1 if prefix else 0)
 
     def flush_l2():
         # Write a buffer twice the L2 size, then read it back: the step's
@@ -398,7 +421,10 @@ def run_ours(args):
             pa.pa_write_kv_cache(kc, vc, kn, vn, sm, err_word=err, stream=stream)
 
     def decode():
-        if fused:
+        if prefix:
+            pa.pa_decode_shared_prefix(out, q, kc, vc, bt, cl, w.shared_prefix_blocks, scale=scale,
+                                       err_word=err, stream=stream)
+        elif fused:
             pa.pa_forward_decode(out, q, kc, vc, kn, vn, sm, bt, cl, scale=scale, workspace=ws,
                                  err_word=err, stream=stream)
         else:
@@ -496,6 +522,18 @@ def run_ours(args):
 
     peak, peak_src = hbm_peak()
     achieved = dec_bytes / (t_dec * 1e-3) / 1e9
+    roofline_tensor = None
+    if prefix:
+        # a shared prefix makes the call a contraction (32 flop per byte for
+        # 64 heads per KV head): its roofline is the tensor-core peak
+        tpeak, tpeak_src = tensor_peak()
+        tach = attention_flops(w) / (t_dec * 1e-3) / 1e12
+        roofline_tensor = {
+            "bound": "tensor", "achieved": tach, "peak": tpeak, "unit": "TFLOP/s",
+            "frac": tach / tpeak, "traffic": None, "kernel": "pa_decode_shared_prefix",
+            "flops_per_launch": attention_flops(w), "launch_us": t_dec * 1e3,
+            "peak_source": tpeak_src, "hbm_gbs": achieved, "hbm_frac": achieved / peak,
+        }
     line = {
         "metric": METRIC,
         "value": bytes_all / (t_step_max * 1e-3) / 1e9,
@@ -513,10 +551,11 @@ def run_ours(args):
         "seq_tokens_per_s": seqs_all / (t_step_max * 1e-3),
         "context_tokens_per_s": ctx_all / (t_step_max * 1e-3),
         "hbm_frac_step": (bytes_all / (t_step_max * 1e-3) / 1e9) / (peak * world),
-        "roofline": {
+        "roofline": roofline_tensor if prefix else {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
-            "kernel": "pa_forward_decode" if fused else "pa_decode",
+            "kernel": ("pa_forward_decode" if fused else
+                       "pa_decode_shared_prefix" if prefix else "pa_decode"),
             "algorithmic_bytes_per_launch": dec_bytes,
             "launch_us": t_dec * 1e3, "peak_source": peak_src,
         },

@@ -18,11 +18,16 @@
 //
 // One CTA per (tile of 128 rows, KV head), 6 warps:
 //   warp 0     tiled copies (no multicast): the Q tile once, then K and V of
-//              each 128-token prefix tile into a 2-stage ring;
+//              each 128-token prefix tile into separate rings (3 K stages, 2
+//              V stages), so that a K stage comes back as soon as its S
+//              product is done;
 //   warp 1     issues tcgen05.mma: S_b = Q K^T (M 128, N 128, K = D), then
 //              O += P_{b'} V for the previous tile (A = P in tensor memory);
-//   warps 2-5  softmax: one row per thread (tensor-memory lane 32 (warp % 4)
-//              + lane), then the epilogue.
+//   warps 2-9  softmax, two warps per tensor-memory subpartition: warp w
+//              owns row 32 (w % 4) + lane and half of each tile's 128
+//              columns (and of O's); the pair exchanges row maxima (and at
+//              the end the normaliser) through shared memory with a bounded
+//              mbarrier handshake; then the epilogue.
 // Tensor memory (512 columns): O [0, D), S_b [D + 128 b, +128), P_b (bf16
 // pairs) [D + 256 + 64 b, +64).  The running max is raised only when a score
 // exceeds it by more than 8 (log2 units), so P < 2^8 and O is rescaled
@@ -42,15 +47,20 @@ using namespace pa::stream;
 
 constexpr int kRows = 128;       // M: (sequence, query head) rows of one tile
 constexpr int kTok = 128;        // N of S: prefix tokens per tile
-constexpr int kThreads = 192;    // 6 warps
+constexpr int kThreads = 320;    // 10 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr float kSlack = 8.f;    // lazy rescaling threshold (log2 units)
 constexpr int kBox = kRows * 128;  // bytes of one 64-element-wide half of a 128-row tile
+constexpr int kKStages = 3, kVStages = 2;
 
 struct alignas(16) Shared {
-  uint64_t qfull, full[2], empty[2], sfull[2], sfree[2], pfull[2], pfree[2], mma_done;
+  uint64_t qfull, kfull[kKStages], kempty[kKStages], vfull[kVStages], vempty[kVStages];
+  uint64_t sfull[2], sfree[2], pfull[2], pfree[2], mma_done;
+  uint64_t xbar[4][2], xend[4];  // softmax pair handshakes (per subpartition)
   uint32_t tmem_base;
   int32_t abort_flag, bad_prefix, pad;
+  float xm[2][2][kRows];  // [tile parity][column half][row] partial row maxima
+  float xl[2][kRows];     // [column half][row] partial normalisers
   int32_t ids[kMaxPrefixBlocks];  // the shared prefix's physical blocks
 };
 
@@ -78,9 +88,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char *tiles =
       smem_raw + (((smem_u32(smem_raw) + sizeof(Shared) + 1023u) & ~1023u) - smem_u32(smem_raw));
   unsigned char *qt = tiles;                          // NH x [128 rows][128 B]
-  unsigned char *kv = tiles + NH * kBox;              // stage s: K then V, NH x kBox each
-  auto k_stage = [&](int s) { return kv + (size_t)s * 2 * NH * kBox; };
-  auto v_stage = [&](int s) { return kv + (size_t)s * 2 * NH * kBox + NH * kBox; };
+  unsigned char *kring = tiles + NH * kBox;           // K stage s: NH x kBox
+  unsigned char *vring = kring + kKStages * NH * kBox;  // V stage s: NH x kBox
+  auto k_stage = [&](int s) { return kring + (size_t)s * NH * kBox; };
+  auto v_stage = [&](int s) { return vring + (size_t)s * NH * kBox; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;                  // KV head
@@ -94,15 +105,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&p.tmap_k);
     prefetch_tensormap(&p.tmap_v);
     mbar_init(&sh.qfull, 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sh.kfull[i], 1);
+      mbar_init(&sh.kempty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sh.vfull[i], 1);
+      mbar_init(&sh.vempty[i], 1);
+    }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sh.full[b], 1);
-      mbar_init(&sh.empty[b], 1);
       mbar_init(&sh.sfull[b], 1);
-      mbar_init(&sh.sfree[b], 4);
-      mbar_init(&sh.pfull[b], 4);
+      mbar_init(&sh.sfree[b], 8);
+      mbar_init(&sh.pfull[b], 8);
       mbar_init(&sh.pfree[b], 1);
     }
     mbar_init(&sh.mma_done, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&sh.xbar[q][0], 64);
+      mbar_init(&sh.xbar[q][1], 64);
+      mbar_init(&sh.xend[q], 64);
+    }
     sh.abort_flag = 0;
     sh.bad_prefix = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -133,24 +155,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int dh = 0; dh < NH; ++dh)
         tma_load_3d(qt + dh * kBox, &p.tmap_q, dh * 64, h * p.group, s0, &sh.qfull);
     }
-    for (int t = 0; t < n_tiles; ++t) {
-      const int s = t & 1;
-      if (t >= 2 && !wait_all(&sh.empty[s], ((t >> 1) - 1) & 1, sh, p, lane)) break;
+    const uint32_t page_bytes = (uint32_t)p.block_size * 128u;
+    // one tile of K or V: its pages' boxes land back to back per d half
+    auto load = [&](const CUtensorMap *map, unsigned char *dst, uint64_t *bar, int t) {
       const int npg = min(ppt, p.prefix_blocks - t * ppt);
       if (lane == 0) {
-        const uint32_t page_bytes = (uint32_t)p.block_size * 128u;
-        mbar_arrive_expect_tx(&sh.full[s], 2u * NH * (uint32_t)npg * page_bytes);
+        mbar_arrive_expect_tx(bar, (uint32_t)NH * (uint32_t)npg * page_bytes);
         for (int i = 0; i < npg; ++i) {
           const int pb = sh.ids[t * ppt + i];
-          for (int dh = 0; dh < NH; ++dh) {
-            tma_load_3d(k_stage(s) + dh * kBox + i * page_bytes, &p.tmap_k, dh * 64,
-                        pb * p.block_size, h, &sh.full[s]);
-            tma_load_3d(v_stage(s) + dh * kBox + i * page_bytes, &p.tmap_v, dh * 64,
-                        pb * p.block_size, h, &sh.full[s]);
-          }
+          for (int dh = 0; dh < NH; ++dh)
+            tma_load_3d(dst + dh * kBox + i * page_bytes, map, dh * 64, pb * p.block_size, h, bar);
         }
       }
       __syncwarp();
+    };
+    // K runs one tile ahead of V: V(t) is needed only after the softmax of t
+    for (int t = 0; t <= n_tiles; ++t) {
+      if (t < n_tiles) {
+        const int ks = t % kKStages;
+        if (t >= kKStages &&
+            !wait_all(&sh.kempty[ks], ((t / kKStages) - 1) & 1, sh, p, lane))
+          break;
+        load(&p.tmap_k, k_stage(ks), &sh.kfull[ks], t);
+      }
+      if (t >= 1) {
+        const int u = t - 1, vs = u % kVStages;
+        if (u >= kVStages &&
+            !wait_all(&sh.vempty[vs], ((u / kVStages) - 1) & 1, sh, p, lane))
+          break;
+        load(&p.tmap_v, v_stage(vs), &sh.vfull[vs], u);
+      }
     }
   } else if (warp == 1) {
     // ===================== tensor-core issue =====================
@@ -158,12 +192,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t id_o = idesc_bf16(kRows, D, true);
     bool ok = wait_all(&sh.qfull, 0, sh, p, lane);
     auto issue_pv = [&](int u) -> bool {
-      const int b = u & 1;
+      const int b = u & 1, vst = u % kVStages;
+      if (!wait_all(&sh.vfull[vst], (u / kVStages) & 1, sh, p, lane)) return false;
       if (!wait_all(&sh.pfull[b], (u >> 1) & 1, sh, p, lane)) return false;
       const int ntok = min(ppt, p.prefix_blocks - u * ppt) * p.block_size;
       if (ntok < kTok) {
         // rows past the prefix in the last tile may hold anything
-        unsigned char *vs = v_stage(b);
+        unsigned char *vs = v_stage(vst);
         const int units = (kTok - ntok) * 8;
         for (int x = lane; x < units * NH; x += 32) {
           const int dh = x / units, rem = x - dh * units;
@@ -175,20 +210,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t va = smem_u32(v_stage(b));
+        const uint32_t va = smem_u32(v_stage(vst));
         for (int ks = 0; ks < kTok / 16; ++ks)
           tc_mma_ts(tm + Cols<D>::O, tm + Cols<D>::P + 64 * b + 8 * ks,
                     sw128_desc(va + 2048 * ks, (uint32_t)kBox, 1024), id_o,
                     (u == 0 && ks == 0) ? 0u : 1u);
         tc_commit(&sh.pfree[b]);
-        tc_commit(&sh.empty[b]);
+        tc_commit(&sh.vempty[vst]);
       }
       __syncwarp();
       return true;
     };
     for (int t = 0; t < n_tiles && ok; ++t) {
-      const int b = t & 1;
-      if (!wait_all(&sh.full[b], (t >> 1) & 1, sh, p, lane)) {
+      const int b = t & 1, kst = t % kKStages;
+      if (!wait_all(&sh.kfull[kst], (t / kKStages) & 1, sh, p, lane)) {
         ok = false;
         break;
       }
@@ -198,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t qa = smem_u32(qt), ka = smem_u32(k_stage(b));
+        const uint32_t qa = smem_u32(qt), ka = smem_u32(k_stage(kst));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32;
@@ -206,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sw128_desc(ka + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(&sh.sfull[b]);
+        tc_commit(&sh.kempty[kst]);  // K stage free once S is computed
       }
       __syncwarp();
       if (t >= 1 && !issue_pv(t - 1)) ok = false;
@@ -213,8 +249,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
   } else {
     // ===================== softmax and epilogue =====================
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const int r = 32 * (warp & 3) + lane;  // this thread's row
+    const int sp = warp & 3;               // tensor-memory subpartition
+    const int half = (warp - 2) >> 2;      // which 64 of a tile's 128 columns
+    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+    const int r = 32 * sp + lane;          // this thread's row
+    const int grow = row0 + r;
+    const int seq = grow / p.group;
+    const int hq = h * p.group + grow % p.group;
+    const bool valid = seq < p.batch;
+    constexpr int HC = kTok / 2;           // score columns per thread
+    constexpr int HD = D / 2;              // output columns per thread
+    // The sequence must contain the declared prefix.  Checked before the
+    // tiles (independent loads, in flight together) so that the latency
+    // hides behind the first copies and products.
+    bool mismatch = false;
+    if (valid) {
+      mismatch = p.context_lens[seq] < p.prefix_blocks * p.block_size;
+      const int32_t *trow = p.block_tables + (int64_t)seq * p.table_stride;
+      for (int i0 = 0; i0 < p.prefix_blocks; i0 += 16) {
+        int32_t e[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) e[j] = (i0 + j < p.prefix_blocks) ? trow[i0 + j] : 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          mismatch |= (i0 + j < p.prefix_blocks) && e[j] != sh.ids[i0 + j];
+      }
+    }
+    // partner handshake: both warps of the pair arrive, then wait (bounded)
+    auto pair_sync = [&](uint64_t *bar, uint32_t parity) -> bool {
+      mbar_arrive(bar);
+      return wait_all(bar, parity, sh, p, lane);
+    };
+    const float sl = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
@@ -225,11 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float sc[kTok];
+      float sc[HC];
 #pragma unroll
-      for (int c = 0; c < kTok / 16; ++c) {
+      for (int c = 0; c < HC / 16; ++c) {
         uint32_t raw[16];
-        tc_ld16(tm + lane_base + Cols<D>::S + kTok * b + 16 * c, raw);
+        tc_ld16(tm + lane_base + Cols<D>::S + kTok * b + HC * half + 16 * c, raw);
 #pragma unroll
         for (int j = 0; j < 16; ++j) sc[16 * c + j] = __uint_as_float(raw[j]);
       }
@@ -237,31 +303,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.sfree[b]);
+      // scores stay raw where possible: with scale > 0 the maximum of the
+      // scaled scores is the scaled maximum and 2^(s scale - m) is one fused
+      // multiply-add and one ex2 per score
+      const bool scaled = ntok < kTok || sl < 0.f;
+      if (scaled) {
+#pragma unroll
+        for (int j = 0; j < HC; ++j) sc[j] = (HC * half + j < ntok) ? sc[j] * sl : -INFINITY;
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < kTok; ++j) {
-        sc[j] = j < ntok ? sc[j] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sc[j]);
+      for (int j = 0; j < HC; ++j) mx = fmaxf(mx, sc[j]);
+      sh.xm[b][half][r] = scaled ? mx : mx * sl;
+      if (!pair_sync(&sh.xbar[sp][b], (t >> 1) & 1)) {
+        ok = false;
+        break;
       }
-      const float m_new = fmaxf(m_used, mx);
+      const float m_new = fmaxf(m_used, fmaxf(sh.xm[b][0][r], sh.xm[b][1][r]));
       const bool need = m_new > m_used + kSlack;
       if (__any_sync(0xffffffffu, need)) {
         const float f = need ? ex2(m_used - m_new) : 1.f;
         if (t >= 1) {
           // O holds the earlier tiles: wait for the last product, rescale
+          // this warp's half of the columns
           if (!wait_all(&sh.pfree[(t - 1) & 1], ((t - 1) >> 1) & 1, sh, p, lane)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 16; ++c) {
+          for (int c = 0; c < HD / 16; ++c) {
             uint32_t o16[16];
-            tc_ld16(tm + lane_base + Cols<D>::O + 16 * c, o16);
+            tc_ld16(tm + lane_base + Cols<D>::O + HD * half + 16 * c, o16);
             tc_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j) o16[j] = __float_as_uint(__uint_as_float(o16[j]) * f);
-            tc_st16(tm + lane_base + Cols<D>::O + 16 * c, o16);
+            tc_st16(tm + lane_base + Cols<D>::O + HD * half + 16 * c, o16);
           }
           tc_wait_st();
         }
@@ -270,11 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_new;
         }
       }
-      uint32_t pk[kTok / 2];
+      uint32_t pk[HC / 2];
       float add = 0.f;
+      const float mul = scaled ? 1.f : sl;
 #pragma unroll
-      for (int j = 0; j < kTok / 2; ++j) {
-        const float p0 = ex2(sc[2 * j] - m_used), p1 = ex2(sc[2 * j + 1] - m_used);
+      for (int j = 0; j < HC / 2; ++j) {
+        const float p0 = ex2(fmaf(sc[2 * j], mul, -m_used));
+        const float p1 = ex2(fmaf(sc[2 * j + 1], mul, -m_used));
         add += p0 + p1;
         pk[j] = pack_bf16x2(p0, p1);
       }
@@ -285,11 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kTok / 32; ++c) {
+      for (int c = 0; c < HC / 32; ++c) {
         uint32_t w16[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) w16[j] = pk[16 * c + j];
-        tc_st16(tm + lane_base + Cols<D>::P + 64 * b + 16 * c, w16);
+        tc_st16(tm + lane_base + Cols<D>::P + (kTok / 2) * b + (HC / 2) * half + 16 * c, w16);
       }
       tc_wait_st();
       tc_fence_before();
@@ -298,54 +377,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && n_tiles > 0 &&
         wait_all(&sh.pfree[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, sh, p, lane)) {
-      tc_fence_after();
-      // the suffix partials are written by the kernels before this one
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      const int grow = row0 + r;
-      const int seq = grow / p.group;
-      const int hq = h * p.group + grow % p.group;
-      const bool valid = seq < p.batch;
-      bool bad = sh.bad_prefix != 0;
-      float ws = 0.f, wp = 1.f;
-      const float *os = nullptr;
-      if (valid) {
-        // the sequence must contain the declared prefix
-        bool mismatch = p.context_lens[seq] < p.prefix_blocks * p.block_size;
-        const int32_t *row = p.block_tables + (int64_t)seq * p.table_stride;
-        for (int i = 0; i < p.prefix_blocks && !mismatch; ++i) mismatch = row[i] != sh.ids[i];
-        if (mismatch) {
-          bad = true;
-          set_error(p.err_word, PA_DEVERR_PREFIX);
-        }
-        const float2 ml = reinterpret_cast<const float2 *>(p.seq_ml)[(int64_t)seq * p.num_q_heads + hq];
-        bad |= ml.y < 0.f;  // a bad page in the suffix
-        const float M = fmaxf(m_used, ml.x);
-        wp = ex2(m_used - M);
-        ws = ml.y > 0.f ? ml.y * ex2(ml.x - M) : 0.f;
-        os = p.seq_o + ((int64_t)seq * p.num_q_heads + hq) * D;
-      }
-      const float inv = 1.f / (l * wp + ws);
-#pragma unroll 1
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t o16[16];
-        tc_ld16(tm + lane_base + Cols<D>::O + 16 * c, o16);
-        tc_wait_ld();
+      // the pair's normalisers add up to the row's
+      sh.xl[half][r] = l;
+      if (pair_sync(&sh.xend[sp], 0)) {
+        const float l_row = sh.xl[0][r] + sh.xl[1][r];
+        tc_fence_after();
+        // the suffix partials are written by the kernels before this one
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        bool bad = sh.bad_prefix != 0;
+        float ws = 0.f, wp = 1.f;
+        const float *os = nullptr;
         if (valid) {
-          float y[16];
-#pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            const float4 sv = ws > 0.f ? *reinterpret_cast<const float4 *>(os + 16 * c + j)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-            y[j + 0] = bad ? 0.f : (__uint_as_float(o16[j + 0]) * wp + sv.x * ws) * inv;
-            y[j + 1] = bad ? 0.f : (__uint_as_float(o16[j + 1]) * wp + sv.y * ws) * inv;
-            y[j + 2] = bad ? 0.f : (__uint_as_float(o16[j + 2]) * wp + sv.z * ws) * inv;
-            y[j + 3] = bad ? 0.f : (__uint_as_float(o16[j + 3]) * wp + sv.w * ws) * inv;
+          if (mismatch) {
+            bad = true;
+            if (half == 0) set_error(p.err_word, PA_DEVERR_PREFIX);
           }
-          const int64_t e = ((int64_t)seq * p.num_q_heads + hq) * D + 16 * c;
+          const float2 ml =
+              reinterpret_cast<const float2 *>(p.seq_ml)[(int64_t)seq * p.num_q_heads + hq];
+          bad |= ml.y < 0.f;  // a bad page in the suffix
+          const float M = fmaxf(m_used, ml.x);
+          wp = ex2(m_used - M);
+          ws = ml.y > 0.f ? ml.y * ex2(ml.x - M) : 0.f;
+          os = p.seq_o + ((int64_t)seq * p.num_q_heads + hq) * D;
+        }
+        const float inv = 1.f / (l_row * wp + ws);
+#pragma unroll 1
+        for (int c = 0; c < HD / 16; ++c) {
+          const int col = HD * half + 16 * c;
+          uint32_t o16[16];
+          tc_ld16(tm + lane_base + Cols<D>::O + col, o16);
+          tc_wait_ld();
+          if (valid) {
+            float y[16];
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            Elem<__nv_bfloat16>::store4(p.out, e + j,
-                                        make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]));
+            for (int j = 0; j < 16; j += 4) {
+              const float4 sv = ws > 0.f ? *reinterpret_cast<const float4 *>(os + col + j)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+              y[j + 0] = bad ? 0.f : (__uint_as_float(o16[j + 0]) * wp + sv.x * ws) * inv;
+              y[j + 1] = bad ? 0.f : (__uint_as_float(o16[j + 1]) * wp + sv.y * ws) * inv;
+              y[j + 2] = bad ? 0.f : (__uint_as_float(o16[j + 2]) * wp + sv.z * ws) * inv;
+              y[j + 3] = bad ? 0.f : (__uint_as_float(o16[j + 3]) * wp + sv.w * ws) * inv;
+            }
+            const int64_t e = ((int64_t)seq * p.num_q_heads + hq) * D + col;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4)
+              Elem<__nv_bfloat16>::store4(p.out, e + j,
+                                          make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]));
+          }
         }
       }
     }
@@ -396,8 +474,9 @@ cudaError_t launch_d(const PrefixParams &p, cudaStream_t stream) {
 
 size_t prefix_smem_bytes(int head_dim) {
   const size_t nh = (size_t)head_dim / 64;
-  // header, 1 KB alignment slack, the Q tile, two stages of K and V
-  return sizeof(prefix::Shared) + 1024 + nh * prefix::kBox * (1 + 2 * 2);
+  // header, 1 KB alignment slack, the Q tile, the K and V rings
+  return sizeof(prefix::Shared) + 1024 +
+         nh * prefix::kBox * (1 + prefix::kKStages + prefix::kVStages);
 }
 
 cudaError_t launch_prefix(const PrefixParams &p, int head_dim, cudaStream_t stream) {

@@ -82,6 +82,7 @@ class Workload:
     partition_tokens: Optional[int] = None
     seed: int = 0
     description: str = ""
+    shared_prefix_blocks: int = 0  # leading table entries every sequence shares
 
     @property
     def elem_bytes(self) -> int:
@@ -232,9 +233,11 @@ def make_workload(name: str, seed: int = 0, batch: Optional[int] = None) -> Work
         ctx = (prefix + suffix).astype(np.int32)
         MB = _pages(prefix + 1024, bs)
         tables, NB = _scattered_tables(rng, ctx, bs, MB, prefix_blocks=prefix // bs)
-        return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
-                       tables, new_tokens=True, seed=seed,
-                       description=f"B{B} Hq64/Hkv1 D128 bs32, 2048 shared prefix + U[1,1024] suffix, bf16")
+        w = _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
+                    tables, new_tokens=True, seed=seed,
+                    description=f"B{B} Hq64/Hkv1 D128 bs32, 2048 shared prefix + U[1,1024] suffix, bf16")
+        w.shared_prefix_blocks = prefix // bs
+        return w
     raise ValueError(f"unknown workload {name!r}; known: {WORKLOADS}")
 
 
@@ -254,10 +257,12 @@ def custom_workload(*, dtype: str, batch: int, num_q_heads: int, num_kv_heads: i
     tables, NB = _scattered_tables(rng, np.maximum(ctx, 0), block_size, MB, slack=slack,
                                    prefix_blocks=prefix_blocks)
     NB = max(NB, 1)
-    return _finish("custom", dtype, rng, batch, num_q_heads, num_kv_heads, head_dim,
-                   block_size, NB, MB, ctx, tables,
-                   new_tokens=new_tokens, seed=seed,
-                   description=f"custom ctx={list(map(int, ctx))[:8]}...")
+    w = _finish("custom", dtype, rng, batch, num_q_heads, num_kv_heads, head_dim,
+                block_size, NB, MB, ctx, tables,
+                new_tokens=new_tokens, seed=seed,
+                description=f"custom ctx={list(map(int, ctx))[:8]}...")
+    w.shared_prefix_blocks = prefix_blocks
+    return w
 
 
 def roofline_bytes(w: Workload, include_write: bool = True) -> int:
