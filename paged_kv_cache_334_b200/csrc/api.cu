@@ -267,6 +267,31 @@ WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
   return w;
 }
 
+// pa_decode_shared_prefix with the suffix on the tensor cores (suffix.cu):
+// the shapes it serves, and its workspace (partials per (CTA, slot, query
+// head), one merge record per (sequence, KV head), the per-row results).
+bool suffix_kernel_serves(const pa_cache_desc *c, int32_t group) {
+  return c->dtype == PA_DTYPE_BF16 && (group == 64 || group == 128) &&
+         (c->head_dim == 64 || c->head_dim == 128);
+}
+
+struct SuffixLayout {
+  size_t part_ml, part_o, merge, seq_ml, seq_o, total;
+};
+
+SuffixLayout suffix_layout(const pa_cache_desc *c, int32_t batch, int32_t num_q_heads) {
+  SuffixLayout l{};
+  const size_t slots = (size_t)pa::stream::kMaxGrid * 2 * num_q_heads;
+  const size_t rows = (size_t)batch * num_q_heads;
+  l.part_ml = 0;
+  l.part_o = round_up(slots * 2 * sizeof(float));
+  l.merge = round_up(l.part_o + slots * c->head_dim * sizeof(float));
+  l.seq_ml = round_up(l.merge + (size_t)batch * c->num_kv_heads * 4 * sizeof(int32_t));
+  l.seq_o = round_up(l.seq_ml + rows * 2 * sizeof(float));
+  l.total = round_up(l.seq_o + rows * (size_t)c->head_dim * sizeof(float));
+  return l;
+}
+
 }  // namespace
 
 namespace pa {
@@ -496,8 +521,10 @@ size_t pa_decode_shared_prefix_workspace_bytes(const pa_cache_desc *cache, int32
     return 0;
   const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
   const size_t rows = (size_t)batch * num_q_heads;
-  return w.total + round_up(rows * 2 * sizeof(float)) +
-         round_up(rows * (size_t)cache->head_dim * sizeof(float));
+  const size_t stream_path = w.total + round_up(rows * 2 * sizeof(float)) +
+                             round_up(rows * (size_t)cache->head_dim * sizeof(float));
+  const size_t tensor_path = suffix_layout(cache, batch, num_q_heads).total;
+  return stream_path > tensor_path ? stream_path : tensor_path;
 }
 
 pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const void *q,
@@ -538,34 +565,26 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
     return fail(PA_ERR_INVALID_ARG, "workspace too small%s: need %lld bytes", "", (long long)need);
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
     return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
-  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
-  const size_t rows = (size_t)batch * num_q_heads;
   char *ws = static_cast<char *>(workspace);
-  float *seq_ml = reinterpret_cast<float *>(ws + w.total);
-  float *seq_o = reinterpret_cast<float *>(ws + w.total + round_up(rows * 2 * sizeof(float)));
-  // 1. the suffix of every sequence, as one partial per (sequence, head)
-  s = decode_impl(cache, out, q, const_cast<void *>(key_cache), const_cast<void *>(value_cache),
-                  nullptr, nullptr, nullptr, block_tables, context_lens, batch, num_q_heads,
-                  max_blocks_per_seq, scale, workspace, w.total, err_word, stream, prefix_blocks,
-                  seq_ml, seq_o);
-  if (s != PA_OK) return s;
-  // 2. the shared prefix on the tensor cores, folded with the suffix partials
-  pa::PrefixParams pp{};
   PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
-  if (fn == nullptr) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable%s");
-  {
+  if (fn == nullptr) return fail(PA_ERR_CUDA, "cannot describe tensors for the tensor copies%s");
+  // q (head_dim, query head, sequence) with boxes of 64 x rows_h x rows_s
+  auto encode_q = [&](CUtensorMap *map, cuuint32_t rows_h, cuuint32_t rows_s) -> bool {
     const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim, (cuuint64_t)num_q_heads,
                                 (cuuint64_t)batch};
     const cuuint64_t strides[2] = {(cuuint64_t)cache->head_dim * 2,
                                    (cuuint64_t)num_q_heads * cache->head_dim * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(128 / group)};
+    const cuuint32_t box[3] = {64, rows_h, rows_s};
     const cuuint32_t estr[3] = {1, 1, 1};
-    if (fn(&pp.tmap_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides,
-           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
-  }
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  pa::PrefixParams pp{};
+  if (!encode_q(&pp.tmap_q, (cuuint32_t)group, (cuuint32_t)(128 / group)))
+    return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
   {
+    // caches (head_dim, token row of the pool, KV head), boxes of 64 x bs x 1
     const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim,
                                 (cuuint64_t)cache->num_blocks * (cuuint64_t)bs,
                                 (cuuint64_t)cache->num_kv_heads};
@@ -581,10 +600,62 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
         return fail(PA_ERR_CUDA, "cannot describe the caches for the tensor copies%s");
     }
   }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  // 1. the suffix of every (sequence, KV head): on the tensor cores for
+  //    groups of 64 or 128 query heads, else on the page-stream kernel; one
+  //    (max, normaliser, normalised output) per row, or partials of cut pairs
+  if (suffix_kernel_serves(cache, group)) {
+    const SuffixLayout l = suffix_layout(cache, batch, num_q_heads);
+    const int sms = device_sm_count();
+    if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
+    pa::SuffixParams sp{};
+    if (!encode_q(&sp.tmap_q, (cuuint32_t)group, 1))
+      return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
+    sp.tmap_k = pp.tmap_k;
+    sp.tmap_v = pp.tmap_v;
+    sp.block_tables = block_tables;
+    sp.context_lens = context_lens;
+    sp.seq_ml = reinterpret_cast<float *>(ws + l.seq_ml);
+    sp.seq_o = reinterpret_cast<float *>(ws + l.seq_o);
+    sp.part_ml = reinterpret_cast<float *>(ws + l.part_ml);
+    sp.part_o = reinterpret_cast<float *>(ws + l.part_o);
+    sp.merge = reinterpret_cast<int32_t *>(ws + l.merge);
+    sp.err_word = err_word;
+    sp.batch = batch;
+    sp.num_q_heads = num_q_heads;
+    sp.num_kv_heads = cache->num_kv_heads;
+    sp.group = group;
+    sp.block_size = bs;
+    sp.table_stride = max_blocks_per_seq;
+    sp.prefix_blocks = prefix_blocks;
+    sp.num_blocks = cache->num_blocks;
+    sp.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
+    sp.scale_log2 = scale_log2;
+    const cudaError_t e = pa::launch_suffix(sp, cache->head_dim, st);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "suffix launch: %s", cudaGetErrorString(e));
+    pp.seq_ml = sp.seq_ml;
+    pp.seq_o = sp.seq_o;
+    pp.merge = sp.merge;
+    pp.part_ml = sp.part_ml;
+    pp.part_o = sp.part_o;
+  } else {
+    const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+    const size_t rows = (size_t)batch * num_q_heads;
+    float *seq_ml = reinterpret_cast<float *>(ws + w.total);
+    float *seq_o = reinterpret_cast<float *>(ws + w.total + round_up(rows * 2 * sizeof(float)));
+    s = decode_impl(cache, out, q, const_cast<void *>(key_cache), const_cast<void *>(value_cache),
+                    nullptr, nullptr, nullptr, block_tables, context_lens, batch, num_q_heads,
+                    max_blocks_per_seq, scale, workspace, w.total, err_word, stream, prefix_blocks,
+                    seq_ml, seq_o);
+    if (s != PA_OK) return s;
+    pp.seq_ml = seq_ml;
+    pp.seq_o = seq_o;
+    pp.merge = nullptr;
+  }
+  // 2. the shared prefix on the tensor cores, folded with the suffix
   pp.block_tables = block_tables;
   pp.context_lens = context_lens;
-  pp.seq_ml = seq_ml;
-  pp.seq_o = seq_o;
   pp.out = out;
   pp.err_word = err_word;
   pp.batch = batch;
@@ -595,8 +666,8 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
   pp.table_stride = max_blocks_per_seq;
   pp.prefix_blocks = prefix_blocks;
   pp.num_blocks = cache->num_blocks;
-  pp.scale_log2 = scale * 1.4426950408889634f;
-  const cudaError_t e = pa::launch_prefix(pp, cache->head_dim, static_cast<cudaStream_t>(stream));
+  pp.scale_log2 = scale_log2;
+  const cudaError_t e = pa::launch_prefix(pp, cache->head_dim, st);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(e));
   return PA_OK;
 }

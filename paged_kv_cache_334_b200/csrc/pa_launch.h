@@ -111,6 +111,13 @@ struct PrefixParams {
   const int32_t *context_lens;
   const float *seq_ml;          // [batch][Hq] (max in log2 units, normaliser) of each suffix
   const float *seq_o;           // [batch][Hq][D] normalised suffix output
+  // Suffixes left by the suffix kernel (suffix.cu): when `merge` is set,
+  // (sequence, KV head) pair i's record merge[4i..4i+3] = (first CTA, number
+  // of CTAs n, slot of the first CTA, bad); n == 1: the result is in
+  // seq_ml / seq_o, n >= 2: in part_ml / part_o rows (CTA * 2 + slot) * Hq + hq,
+  // n == 0: no suffix.  NULL: seq_ml / seq_o hold every row's suffix.
+  const int32_t *merge;
+  const float *part_ml, *part_o;
   void *out;
   int32_t *err_word;
   int32_t batch, num_q_heads, num_kv_heads, group, block_size, table_stride, prefix_blocks,
@@ -119,6 +126,26 @@ struct PrefixParams {
 };
 size_t prefix_smem_bytes(int head_dim);
 cudaError_t launch_prefix(const PrefixParams &p, int head_dim, cudaStream_t stream);
+
+// Arguments of the suffix kernel (suffix.cu): the tokens past the shared
+// prefix of every (sequence, KV head) pair on the tensor cores, for groups
+// of 64 or 128 query heads per KV head.
+struct SuffixParams {
+  CUtensorMap tmap_q;  // q (head_dim, query head, sequence), boxes of 64 x group x 1
+  CUtensorMap tmap_k;  // caches as in PrefixParams
+  CUtensorMap tmap_v;
+  const int32_t *block_tables;
+  const int32_t *context_lens;
+  float *seq_ml, *seq_o;    // pairs inside one CTA's range: [batch][Hq][2], [batch][Hq][D]
+  float *part_ml, *part_o;  // cut pairs: [grid * 2][Hq][2], [grid * 2][Hq][D]
+  int32_t *merge;           // [batch * Hkv][4], as read by the prefix kernel
+  int32_t *err_word;
+  int32_t batch, num_q_heads, num_kv_heads, group, block_size, table_stride, prefix_blocks,
+      num_blocks, grid;
+  float scale_log2;
+};
+size_t suffix_smem_bytes(int head_dim, int group);
+cudaError_t launch_suffix(const SuffixParams &p, int head_dim, cudaStream_t stream);
 
 // Query heads handled together by one CTA for a GQA group of `group` heads.
 int decode_head_tile(int group);

@@ -11,10 +11,13 @@
 // FlashAttention forward pass ([route] page "From correct to faster: the
 // PagedAttention optimisation route", section "The core idea of
 // high-performance PagedAttention": online softmax, no score matrix in
-// memory).  The suffix past the prefix is decoded first by the persistent
-// page-stream kernel in suffix mode, which leaves one (max, sum, normalised
-// output) partial per row; this kernel's epilogue folds that partial in with
-// the running-max rescaling and writes the output.
+// memory).  The suffix past the prefix is decoded first: for groups of 64 or
+// 128 query heads by the tensor-core suffix kernel (suffix.cu), which leaves
+// one (max, sum, normalised output) per row or, for a (sequence, KV head)
+// pair cut between its CTAs, one such partial per CTA with a record of where
+// they are; for other groups by the persistent page-stream kernel in suffix
+// mode and its merge kernel, one partial per row.  This kernel's epilogue
+// folds the parts in with the running-max rescaling and writes the output.
 //
 // One CTA per (tile of 128 rows, KV head), 6 warps:
 //   warp 0     tiled copies (no multicast): the Q tile once, then K and V of
@@ -385,22 +388,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the suffix partials are written by the kernels before this one
         asm volatile("griddepcontrol.wait;" ::: "memory");
         bool bad = sh.bad_prefix != 0;
-        float ws = 0.f, wp = 1.f;
-        const float *os = nullptr;
+        // The suffix as n contributions (max, normaliser, normalised output):
+        // one row of seq_ml / seq_o, or (merge records) the partials of the
+        // CTAs of the suffix kernel that cut the pair, or none.
+        const int64_t row = (int64_t)seq * p.num_q_heads + hq;
+        int n = 1, cf = 0, fs = 0;
         if (valid) {
           if (mismatch) {
             bad = true;
             if (half == 0) set_error(p.err_word, PA_DEVERR_PREFIX);
           }
-          const float2 ml =
-              reinterpret_cast<const float2 *>(p.seq_ml)[(int64_t)seq * p.num_q_heads + hq];
-          bad |= ml.y < 0.f;  // a bad page in the suffix
-          const float M = fmaxf(m_used, ml.x);
-          wp = ex2(m_used - M);
-          ws = ml.y > 0.f ? ml.y * ex2(ml.x - M) : 0.f;
-          os = p.seq_o + ((int64_t)seq * p.num_q_heads + hq) * D;
+          if (p.merge != nullptr) {
+            const int4 md = reinterpret_cast<const int4 *>(p.merge)[(int64_t)seq * p.num_kv_heads + h];
+            cf = md.x;
+            n = md.y;
+            fs = md.z;
+            bad |= md.w != 0;  // a length outside the table
+          }
+        } else {
+          n = 0;
         }
-        const float inv = 1.f / (l_row * wp + ws);
+        const float2 *mls = reinterpret_cast<const float2 *>(n == 1 ? p.seq_ml : p.part_ml);
+        const float *obase = n == 1 ? p.seq_o : p.part_o;
+        auto crow = [&](int x) -> int64_t {
+          return n == 1 ? row : ((int64_t)(cf + x) * 2 + (x == 0 ? fs : 0)) * p.num_q_heads + hq;
+        };
+        // running-max merge: M over every part, weights l 2^(m - M)
+        float M = m_used;
+        for (int x = 0; x < n; ++x) {
+          const float2 ml = mls[crow(x)];
+          bad |= ml.y < 0.f;  // a bad page in the suffix
+          if (ml.y > 0.f) M = fmaxf(M, ml.x);
+        }
+        const float wp = ex2(m_used - M);
+        float W = l_row * wp;
+        for (int x = 0; x < n; ++x) {
+          const float2 ml = mls[crow(x)];
+          if (ml.y > 0.f) W += ml.y * ex2(ml.x - M);
+        }
+        const float inv = 1.f / W;
 #pragma unroll 1
         for (int c = 0; c < HD / 16; ++c) {
           const int col = HD * half + 16 * c;
@@ -410,15 +436,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (valid) {
             float y[16];
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-              const float4 sv = ws > 0.f ? *reinterpret_cast<const float4 *>(os + col + j)
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-              y[j + 0] = bad ? 0.f : (__uint_as_float(o16[j + 0]) * wp + sv.x * ws) * inv;
-              y[j + 1] = bad ? 0.f : (__uint_as_float(o16[j + 1]) * wp + sv.y * ws) * inv;
-              y[j + 2] = bad ? 0.f : (__uint_as_float(o16[j + 2]) * wp + sv.z * ws) * inv;
-              y[j + 3] = bad ? 0.f : (__uint_as_float(o16[j + 3]) * wp + sv.w * ws) * inv;
+            for (int j = 0; j < 16; ++j) y[j] = __uint_as_float(o16[j]) * wp;
+            for (int x = 0; x < n; ++x) {
+              const int64_t cr = crow(x);
+              const float2 ml = mls[cr];
+              if (!(ml.y > 0.f)) continue;
+              const float w = ml.y * ex2(ml.x - M);
+              const float *os = obase + cr * D + col;
+#pragma unroll
+              for (int j = 0; j < 16; j += 4) {
+                const float4 sv = *reinterpret_cast<const float4 *>(os + j);
+                y[j + 0] += w * sv.x;
+                y[j + 1] += w * sv.y;
+                y[j + 2] += w * sv.z;
+                y[j + 3] += w * sv.w;
+              }
             }
-            const int64_t e = ((int64_t)seq * p.num_q_heads + hq) * D + col;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) y[j] = bad ? 0.f : y[j] * inv;
+            const int64_t e = row * D + col;
 #pragma unroll
             for (int j = 0; j < 16; j += 4)
               Elem<__nv_bfloat16>::store4(p.out, e + j,
@@ -474,9 +510,11 @@ cudaError_t launch_d(const PrefixParams &p, cudaStream_t stream) {
 
 size_t prefix_smem_bytes(int head_dim) {
   const size_t nh = (size_t)head_dim / 64;
-  // header, 1 KB alignment slack, the Q tile, the K and V rings
-  return sizeof(prefix::Shared) + 1024 +
-         nh * prefix::kBox * (1 + prefix::kKStages + prefix::kVStages);
+  // header, 1 KB alignment slack, the Q tile, the K and V rings; at least
+  // 120 KB, so that no other CTA holding tensor memory shares the SM
+  const size_t need = sizeof(prefix::Shared) + 1024 +
+                      nh * prefix::kBox * (1 + prefix::kKStages + prefix::kVStages);
+  return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
 cudaError_t launch_prefix(const PrefixParams &p, int head_dim, cudaStream_t stream) {

@@ -80,6 +80,20 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
 __device__ __forceinline__ void prefetch_l2(const void *g, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(g), "r"(bytes) : "memory");
 }
+// 4-byte asynchronous global -> shared copy into the calling thread's open
+// copy group; groups are closed by cp_async_commit and waited for per thread.
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 // Orders this thread's earlier generic-proxy global stores before its later
 // async-proxy (bulk / tensor copy) accesses of global memory.
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -141,3 +141,62 @@ def test_shared_prefix_zero_blocks_is_pa_decode():
                  d["context_lens"])
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# Groups of 64 or 128 query heads per KV head take the tensor-core suffix
+# kernel: 128-token tiles of each (sequence, KV head) pair split evenly over
+# one CTA per SM, partials of pairs cut between CTAs folded in by the prefix
+# kernel's epilogue.
+TENSOR_SUFFIX_CASES = [
+    # Hq, Hkv, D, bs, prefix_blocks, suffix lengths
+    (64, 1, 128, 32, 2, [9000, 7000]),                      # pairs cut across many CTAs
+    (128, 2, 128, 16, 4, [0, 300, 1, 128, 129, 2000, 5]),   # two KV heads, an empty suffix
+    (64, 1, 128, 8, 16, [1, 127, 128, 129, 1000, 257]),     # 16 pages per tile
+    (64, 1, 128, 128, 1, [1, 127, 128, 129, 600, 3]),       # one page per tile
+    (256, 2, 64, 32, 3, [40, 700, 1, 0, 333]),              # 128 heads per KV head, head_dim 64
+    (64, 1, 64, 16, 5, [2500, 2500, 2500, 1, 1, 1, 1, 1]),
+]
+
+
+def _decode_ref(w):
+    return oracle.decode(w.q, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                         1.0 / math.sqrt(w.head_dim))[0]
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,bs,npre,suffix", TENSOR_SUFFIX_CASES)
+def test_tensor_suffix_shapes(Hq, Hkv, D, bs, npre, suffix):
+    lens = [npre * bs + s for s in suffix]
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=len(lens), num_q_heads=Hq,
+                           num_kv_heads=Hkv, head_dim=D, block_size=bs, context_lens=lens,
+                           seed=7 * Hq + D + bs + npre, prefix_blocks=npre)
+    d = upload(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = shared_prefix(d, npre, err)
+    again = shared_prefix(d, npre, err)  # the workspace is reused as is
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert_close(to_f64(out), _decode_ref(w), w.dtype, f"tensor suffix {Hq}/{Hkv} D{D} bs{bs}")
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))
+
+
+def test_tensor_suffix_bad_page_and_length():
+    """A bad page id inside one suffix and a context longer than the table:
+    those two sequences are flagged and zeroed, the others are unaffected."""
+    npre, bs = 2, 32
+    lens = [npre * bs + s for s in (900, 700, 50, 2000, 130)]
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=len(lens), num_q_heads=64,
+                           num_kv_heads=1, head_dim=128, block_size=bs, context_lens=lens,
+                           seed=11, prefix_blocks=npre)
+    d = upload(w)
+    d["block_tables"][1, npre + 5] = w.num_blocks + 3
+    d["context_lens"][2] = w.block_tables.shape[1] * bs + 1
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = shared_prefix(d, npre, err)
+    torch.cuda.synchronize()
+    e = int(err.item())
+    assert e & pa.PA_DEVERR_BLOCK_ID and e & pa.PA_DEVERR_CONTEXT_LEN
+    got = to_f64(out)
+    assert np.all(got[1] == 0) and np.all(got[2] == 0)
+    ref = _decode_ref(w)
+    keep = [0, 3, 4]
+    assert_close(got[keep], ref[keep], w.dtype, "unaffected sequences")
