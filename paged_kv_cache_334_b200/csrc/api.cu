@@ -614,6 +614,20 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
       return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
     sp.tmap_k = pp.tmap_k;
     sp.tmap_v = pp.tmap_v;
+    // fp32 rows of D (seq_o, part_o) for the epilogue's tiled stores
+    auto encode_rows = [&](CUtensorMap *map, char *base, size_t rows) -> bool {
+      const cuuint64_t dims[2] = {(cuuint64_t)cache->head_dim, (cuuint64_t)rows};
+      const cuuint64_t strides[1] = {(cuuint64_t)cache->head_dim * 4};
+      const cuuint32_t box[2] = {32, (cuuint32_t)group};
+      const cuuint32_t estr[2] = {1, 1};
+      return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!encode_rows(&sp.tmap_seq_o, ws + l.seq_o, (size_t)batch * num_q_heads) ||
+        !encode_rows(&sp.tmap_part_o, ws + l.part_o,
+                     (size_t)pa::stream::kMaxGrid * 2 * num_q_heads))
+      return fail(PA_ERR_CUDA, "cannot describe the suffix results for the tensor copies%s");
     sp.block_tables = block_tables;
     sp.context_lens = context_lens;
     sp.seq_ml = reinterpret_cast<float *>(ws + l.seq_ml);

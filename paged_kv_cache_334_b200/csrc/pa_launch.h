@@ -134,6 +134,10 @@ struct SuffixParams {
   CUtensorMap tmap_q;  // q (head_dim, query head, sequence), boxes of 64 x group x 1
   CUtensorMap tmap_k;  // caches as in PrefixParams
   CUtensorMap tmap_v;
+  // fp32 (head_dim, row) views of seq_o and part_o with boxes of 32 x group
+  // and 128-byte swizzle: the epilogue's tiled stores (group 64)
+  CUtensorMap tmap_seq_o;
+  CUtensorMap tmap_part_o;
   const int32_t *block_tables;
   const int32_t *context_lens;
   float *seq_ml, *seq_o;    // pairs inside one CTA's range: [batch][Hq][2], [batch][Hq][D]

@@ -67,14 +67,21 @@ struct alignas(16) Shared {
   int32_t ids[kMaxPrefixBlocks];  // the shared prefix's physical blocks
 };
 
-__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, Shared &sh,
-                                         const PrefixParams &p, int lane) {
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, &sh.abort_flag));
+// Warp-uniform bounded wait: one inline test, the rest out of line (see
+// mbar_wait_slow).
+static __device__ __noinline__ bool wait_all_slow(uint64_t *bar, uint32_t parity, Shared &sh,
+                                           int32_t *err_word, int lane) {
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_slow(bar, parity, &sh.abort_flag));
   if (!ok && lane == 0) {
     sh.abort_flag = 1;
-    set_error(p.err_word, PA_DEVERR_TIMEOUT);
+    set_error(err_word, PA_DEVERR_TIMEOUT);
   }
   return ok;
+}
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, Shared &sh,
+                                         const PrefixParams &p, int lane) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return wait_all_slow(bar, parity, sh, p.err_word, lane);
 }
 
 template <int D>

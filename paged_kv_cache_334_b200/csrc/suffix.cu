@@ -23,7 +23,7 @@
 // of CTAs, slot of the first) for the prefix kernel, which folds the
 // partials in with the same running-max rescaling.
 //
-// 10 warps:
+// 11 warps:
 //   warp 0     walks the range: page ids two tiles ahead (4-byte asynchronous
 //              copies into shared memory), one descriptor per tile, the Q
 //              tile of each pair it starts, K and V tiles into separate rings
@@ -31,7 +31,10 @@
 //   warp 1     tcgen05.mma: S_b = Q K^T, then O += P V of the previous tile;
 //   warps 2-9  softmax, two warps per tensor-memory subpartition (each owns
 //              half of a tile's 128 columns and of O's), and the epilogue of
-//              every pair segment.
+//              every pair segment;
+//   warp 10    (group 64) the epilogue's tiled stores from a staging buffer:
+//              issuing a store waits while the SM's copy engine is busy with
+//              tile loads, so no other warp issues one.
 // Tensor memory (512 columns): O [0, D), S_b [D + 128 b), P_b (bf16 pairs)
 // [D + 256 + 64 b).  An M = 64 accumulator keeps row r in lane
 // (r % 16) + 32 (r / 16): lanes 0-15 of each softmax warp own rows, lanes
@@ -52,7 +55,7 @@ namespace suffix {
 using namespace pa::stream;
 
 constexpr int kTok = 128;             // tokens per tile: N of S, K of P V
-constexpr int kThreads = 320;         // 10 warps
+constexpr int kThreads = 352;         // 11 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr float kSlack = 8.f;         // lazy rescaling threshold (log2 units)
 constexpr int kTileBox = kTok * 128;  // bytes of one 64-wide half of a K or V tile
@@ -68,7 +71,9 @@ template <int D, int M>
 struct Cfg {
   static constexpr int NH = D / 64;                          // 64-wide halves of head_dim
   static constexpr int kQBox = M * 128;                      // one half of a Q tile
-  static constexpr int KS = (D == 128 && M == 128) ? 2 : 3;  // K stages within 227 KB
+  static constexpr int KS = D == 128 ? 2 : 3;                // K stages within 227 KB
+  // group 64: a staging buffer for the epilogue's tiled stores (M x D fp32)
+  static constexpr int kStage = M == 64 ? M * D * 4 : 0;
   static constexpr uint32_t O = 0, S = D, P = D + 2 * kTok;  // tensor-memory columns
 };
 
@@ -82,6 +87,7 @@ struct alignas(16) Shared {
   uint64_t qfull[kQStages], qempty[kQStages], kfull[kMaxKStages], kempty[kMaxKStages];
   uint64_t vfull[kVStages], vempty[kVStages];
   uint64_t sfull[2], sfree[2], pfull[2], pfree[2], ofull, ofree, mma_done;
+  uint64_t staged, stfree;  // epilogue staging (group 64): written / read by the store
   uint64_t dfull[kRing], dempty[kRing];
   uint64_t xbar[4][2], xend[4];  // softmax pair handshakes (per subpartition)
   int64_t red[32];
@@ -92,16 +98,25 @@ struct alignas(16) Shared {
   int32_t pids[kRing][kMaxPPT];  // page ids of a tile, written by asynchronous copies
   float xm[2][2][128];           // [tile parity][column half][row] partial row maxima
   float xl[2][128];              // [column half][row] partial normalisers
+  float2 mlst[128];              // epilogue staging of (max, normaliser) per row
+  int32_t st_row, st_direct;     // the staged pair's first output row, and where it goes
 };
 
-__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, Shared &sh,
-                                         const SuffixParams &p, int lane) {
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, &sh.abort_flag));
+// Warp-uniform bounded wait: one inline test, the rest out of line (see
+// mbar_wait_slow).
+static __device__ __noinline__ bool wait_all_slow(uint64_t *bar, uint32_t parity, Shared &sh,
+                                           int32_t *err_word, int lane) {
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_slow(bar, parity, &sh.abort_flag));
   if (!ok && lane == 0) {
     sh.abort_flag = 1;
-    set_error(p.err_word, PA_DEVERR_TIMEOUT);
+    set_error(err_word, PA_DEVERR_TIMEOUT);
   }
   return ok;
+}
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, Shared &sh,
+                                         const SuffixParams &p, int lane) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return wait_all_slow(bar, parity, sh, p.err_word, lane);
 }
 
 // Exclusive prefix sum of v over the CTA; *total = the sum of every thread's v.
@@ -208,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char *qring = tiles;                             // Q stage: NH x kQBox
   unsigned char *kring = qring + kQStages * NH * C::kQBox;  // K stage: NH x kTileBox
   unsigned char *vring = kring + KS * NH * kTileBox;        // V stage: NH x kTileBox
+  unsigned char *stg = vring + kVStages * NH * kTileBox;    // epilogue staging (group 64)
   auto q_stage = [&](int s) { return qring + (size_t)s * NH * C::kQBox; };
   auto k_stage = [&](int s) { return kring + (size_t)s * NH * kTileBox; };
   auto v_stage = [&](int s) { return vring + (size_t)s * NH * kTileBox; };
@@ -245,6 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sh.ofull, 1);
     mbar_init(&sh.ofree, 8);
     mbar_init(&sh.mma_done, 1);
+    mbar_init(&sh.staged, 8);
+    mbar_init(&sh.stfree, 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.dfull[i], 1);
       mbar_init(&sh.dempty[i], 9);  // the tensor-core warp and the 8 softmax warps
@@ -461,19 +479,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1 && n_units > 0) {
     // ===================== tensor-core issue =====================
+    // Two products are pending at a time, S = Q K^T of the next tile and
+    // O += P V of an earlier one; whichever has its inputs first is issued
+    // first (a bounded poll, like every wait).  A pair's last P V thus never
+    // waits for the next tile's K, and its epilogue starts as early as it can.
     const uint32_t id_s = idesc_bf16(M, kTok, false);
     const uint32_t id_o = idesc_bf16(M, D, true);
-    struct Prev {
+    struct Pend {
       int32_t flags, ntok, seg;
     };
-    auto issue_pv = [&](int v, const Prev &x) -> bool {
+    auto ready = [&](uint64_t *bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
+    };
+    auto issue_pv = [&](int v, const Pend &x) {
       const int b = v & 1, vs = v % kVStages;
-      if (!wait_all(&sh.vfull[vs], (v / kVStages) & 1, sh, p, lane)) return false;
-      if (!wait_all(&sh.pfull[b], (v >> 1) & 1, sh, p, lane)) return false;
       const bool first = (x.flags & kFirst) != 0;
-      // a pair's first product overwrites O: the previous pair's epilogue
-      // must have read it
-      if (first && x.seg >= 1 && !wait_all(&sh.ofree, (x.seg - 1) & 1, sh, p, lane)) return false;
       if (x.ntok < kTok) {
         // rows past the pair's tokens may hold anything (0 * NaN is NaN)
         unsigned char *vsm = v_stage(vs);
@@ -498,55 +518,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (x.flags & kLast) tc_commit(&sh.ofull);
       }
       __syncwarp();
-      return true;
     };
-    bool ok = true;
-    int seg = -1;
-    Prev prev{0, 0, 0};
-    for (int u = 0; u < n_units && ok; ++u) {
-      const int b = u & 1, ks = u % KS;
-      if (!wait_all(&sh.dfull[u % kRing], (u / kRing) & 1, sh, p, lane)) {
-        ok = false;
-        break;
-      }
-      const Desc d = sh.desc[u % kRing];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.dempty[u % kRing]);
-      if (d.flags & kFirst) {
-        ++seg;
-        if (!wait_all(&sh.qfull[seg % kQStages], (seg / kQStages) & 1, sh, p, lane)) {
-          ok = false;
-          break;
+    Pend pend0{0, 0, 0}, pend1{0, 0, 0};  // tiles whose S is issued, by parity
+    Desc du{};
+    bool have_d = false;  // descriptor of tile u read
+    int u = 0, v = 0;     // next S, next P V
+    int seg = -1;         // pair segment of tile u (once its descriptor is read)
+    uint64_t t_last = global_ns();
+    for (uint32_t spin = 0; v < n_units; ++spin) {
+      bool progressed = false;
+      if (v < u) {
+        const Pend x = (v & 1) ? pend1 : pend0;
+        // a pair's first product overwrites O: the previous pair's epilogue
+        // must have read it
+        if (ready(&sh.vfull[v % kVStages], (v / kVStages) & 1) &&
+            ready(&sh.pfull[v & 1], (v >> 1) & 1) &&
+            (!(x.flags & kFirst) || x.seg == 0 || ready(&sh.ofree, (x.seg - 1) & 1))) {
+          issue_pv(v, x);
+          ++v;
+          progressed = true;
         }
       }
-      if (!wait_all(&sh.kfull[ks], (u / KS) & 1, sh, p, lane)) {
-        ok = false;
-        break;
-      }
-      if (u >= 2 && !wait_all(&sh.sfree[b], ((u >> 1) - 1) & 1, sh, p, lane)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t qa = smem_u32(q_stage(seg % kQStages)), ka = smem_u32(k_stage(ks));
+      if (u < n_units && u - v <= 1) {
+        if (!have_d && ready(&sh.dfull[u % kRing], (u / kRing) & 1)) {
+          du = sh.desc[u % kRing];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.dempty[u % kRing]);
+          if (du.flags & kFirst) ++seg;
+          have_d = true;
+          progressed = true;
+        }
+        const int b = u & 1, ks = u % KS;
+        if (have_d &&
+            (!(du.flags & kFirst) || ready(&sh.qfull[seg % kQStages], (seg / kQStages) & 1)) &&
+            ready(&sh.kfull[ks], (u / KS) & 1) &&
+            (u < 2 || ready(&sh.sfree[b], ((u >> 1) - 1) & 1))) {
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t qa = smem_u32(q_stage(seg % kQStages)), ka = smem_u32(k_stage(ks));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qoff = (uint32_t)(kk >> 2) * C::kQBox + (uint32_t)(kk & 3) * 32;
-          const uint32_t koff = (uint32_t)(kk >> 2) * kTileBox + (uint32_t)(kk & 3) * 32;
-          tc_mma_ss(tm + C::S + kTok * b, sw128_desc(qa + qoff, 16, 1024),
-                    sw128_desc(ka + koff, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qoff = (uint32_t)(kk >> 2) * C::kQBox + (uint32_t)(kk & 3) * 32;
+              const uint32_t koff = (uint32_t)(kk >> 2) * kTileBox + (uint32_t)(kk & 3) * 32;
+              tc_mma_ss(tm + C::S + kTok * b, sw128_desc(qa + qoff, 16, 1024),
+                        sw128_desc(ka + koff, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&sh.sfull[b]);
+            tc_commit(&sh.kempty[ks]);  // K stage free once S is computed
+            if (du.flags & kLast) tc_commit(&sh.qempty[seg % kQStages]);
+          }
+          __syncwarp();
+          const Pend x{du.flags, du.ntok, seg};
+          if (u & 1) {
+            pend1 = x;
+          } else {
+            pend0 = x;
+          }
+          ++u;
+          have_d = false;
+          progressed = true;
         }
-        tc_commit(&sh.sfull[b]);
-        tc_commit(&sh.kempty[ks]);  // K stage free once S is computed
-        if (d.flags & kLast) tc_commit(&sh.qempty[seg % kQStages]);
       }
-      __syncwarp();
-      if (u >= 1 && !issue_pv(u - 1, prev)) ok = false;
-      prev = Prev{d.flags, d.ntok, seg};
+      if (progressed) {
+        t_last = global_ns();
+      } else if ((spin & 15) == 0 &&
+                 (*reinterpret_cast<volatile int32_t *>(&sh.abort_flag) ||
+                  global_ns() - t_last > kWaitLimitNs)) {
+        if (lane == 0) {
+          sh.abort_flag = 1;
+          set_error(p.err_word, PA_DEVERR_TIMEOUT);
+        }
+        break;
+      }
     }
-    if (ok) issue_pv(n_units - 1, prev);
-  } else if (warp >= 2 && n_units > 0) {
+  } else if (warp >= 2 && warp < 10 && n_units > 0) {
     // ===================== softmax and epilogue =====================
     const int sp = warp & 3;           // tensor-memory subpartition
     const int half = (warp - 2) >> 2;  // which 64 of a tile's 128 columns
@@ -669,11 +714,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.ofree);  // the next pair may overwrite O
-        if (row_ok) {
-          const bool direct = (d.flags & kDirect) != 0;
+        const bool direct = (d.flags & kDirect) != 0;
+        const float inv = seg_bad ? 0.f : 1.f / l_row;
+        if constexpr (M == 64) {
+          // Stage the rows in the 128-byte-swizzled layout of tiled stores
+          // of 32 x 64 boxes; one thread stores them and does not wait: a
+          // global store, or a wait for one, in these warps would queue
+          // behind this SM's tile copies.  The staging buffer is reused once
+          // the previous pair's stores have read it.
+          if (seg >= 1 && !wait_all(&sh.stfree, (seg - 1) & 1, sh, p, lane)) break;
+          if (row_ok) {
+#pragma unroll
+            for (int cc = 0; cc < HD / 16; ++cc) {
+#pragma unroll
+              for (int j = 0; j < 16; j += 4) {
+                const int col = HD * half + 16 * cc + j;
+                const int bx = col >> 5, ch = (col & 31) >> 2;
+                *reinterpret_cast<float4 *>(stg + bx * (M * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                    make_float4(__uint_as_float(o[cc][j]) * inv, __uint_as_float(o[cc][j + 1]) * inv,
+                                __uint_as_float(o[cc][j + 2]) * inv,
+                                __uint_as_float(o[cc][j + 3]) * inv);
+              }
+            }
+            if (half == 0) sh.mlst[r] = make_float2(m_used, seg_bad ? -1.f : l_row);
+          }
+          if (warp == 2 && lane == 0) {
+            sh.st_row = d.row;
+            sh.st_direct = direct ? 1 : 0;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.staged);
+        } else if (row_ok) {
           const int64_t row = (int64_t)d.row + r;
           float *dst = (direct ? p.seq_o : p.part_o) + row * D + HD * half;
-          const float inv = seg_bad ? 0.f : 1.f / l_row;
 #pragma unroll
           for (int cc = 0; cc < HD / 16; ++cc) {
 #pragma unroll
@@ -688,6 +762,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if constexpr (M == 64) {
+      // no more pairs: once the last one has left the staging buffer, tell
+      // the store warp (a row of -1)
+      if (seg >= 0) wait_all(&sh.stfree, seg & 1, sh, p, lane);
+      if (warp == 2 && lane == 0) sh.st_row = -1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.staged);
+    }
+  } else if (warp == 10 && M == 64 && n_units > 0) {
+    // ===================== output stores (group 64) =====================
+    // Tiled stores of each staged pair: issuing them waits while this SM's
+    // copy engine is busy with tile loads, so they get a warp of their own.
+    for (int g = 0;; ++g) {
+      if (!wait_all(&sh.staged, g & 1, sh, p, lane)) break;
+      const int32_t row = sh.st_row;
+      if (row < 0) break;
+      if (lane == 0) {
+        const CUtensorMap *map = sh.st_direct ? &p.tmap_seq_o : &p.tmap_part_o;
+        for (int bx = 0; bx < D / 32; ++bx) tma_store_2d(map, bx * 32, row, stg + bx * (M * 128));
+        bulk_s2g((sh.st_direct ? p.seq_ml : p.part_ml) + (int64_t)row * 2, sh.mlst,
+                 (uint32_t)(M * 8));
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(&sh.stfree);  // the softmax warps may stage the next pair
+      }
+      __syncwarp();
+    }
+    // the stores are complete before the CTA ends
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // ---- Sequences with no suffix tile: an empty record for each pair (and
@@ -720,7 +824,8 @@ template <int D, int M>
 size_t smem_bytes() {
   using C = Cfg<D, M>;
   const size_t need = sizeof(Shared) + 1024 +
-                      (size_t)C::NH * (kQStages * C::kQBox + (C::KS + kVStages) * kTileBox);
+                      (size_t)C::NH * (kQStages * C::kQBox + (C::KS + kVStages) * kTileBox) +
+                      C::kStage;
   return need < kMinSmem ? kMinSmem : need;
 }
 
