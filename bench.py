@@ -193,6 +193,13 @@ class ClockSampler:
 # measured peaks and ncu traffic
 # ---------------------------------------------------------------------------
 
+def tensor_path(w) -> bool:
+    """The shapes libpa decodes on tcgen05 tiles (64 or 128 query heads per
+    KV head, bf16, head_dim 64 or 128, block_size 8..128)."""
+    return (w.dtype == wl.DTYPE_BF16 and w.group in (64, 128) and w.head_dim in (64, 128)
+            and 8 <= w.block_size <= 128)
+
+
 def tensor_peak():
     """Dense bf16 tensor-core peak (burst: the call is timed alone)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -404,10 +411,17 @@ def run_ours(args):
     prefix = args.step == "prefix"
     if prefix and not w.shared_prefix_blocks:
         raise SystemExit(f"--step prefix needs a workload with a shared prefix, not {w.name}")
-    # libpa kernels per step: the persistent decode kernel and its merge
-    # kernel, plus the write kernel when the write is a separate call, plus
-    # the prefix kernel of the shared-prefix path
-    launches_per_step = 2 + (1 if has_new and not fused else 0) + (1 if prefix else 0)
+    # libpa kernels per step.  Groups of 64 or 128 query heads (tensor-core
+    # path): the checked write (inside pa_forward_decode or as its own call),
+    # the tile kernel and its finishing pass; with a shared prefix the tile
+    # kernel and the prefix kernel.  Other groups: the persistent decode
+    # kernel and its merge kernel, plus the write kernel when the write is a
+    # separate call, plus the prefix kernel of the shared-prefix path.
+    tensor = tensor_path(w)
+    if tensor:
+        launches_per_step = 2 if prefix else 2 + (1 if has_new else 0)
+    else:
+        launches_per_step = 2 + (1 if has_new and not fused else 0) + (1 if prefix else 0)
 
     def flush_l2():
         # Write a buffer twice the L2 size, then read it back: the step's
@@ -523,14 +537,17 @@ def run_ours(args):
     peak, peak_src = hbm_peak()
     achieved = dec_bytes / (t_dec * 1e-3) / 1e9
     roofline_tensor = None
-    if prefix:
-        # a shared prefix makes the call a contraction (32 flop per byte for
-        # 64 heads per KV head): its roofline is the tensor-core peak
+    if prefix or tensor:
+        # 64 or 128 query heads per KV head (32 or 64 flop per byte of KV),
+        # and a shared prefix, make the call a contraction: its roofline is
+        # the tensor-core peak
         tpeak, tpeak_src = tensor_peak()
         tach = attention_flops(w) / (t_dec * 1e-3) / 1e12
         roofline_tensor = {
             "bound": "tensor", "achieved": tach, "peak": tpeak, "unit": "TFLOP/s",
-            "frac": tach / tpeak, "traffic": None, "kernel": "pa_decode_shared_prefix",
+            "frac": tach / tpeak, "traffic": None,
+            "kernel": ("pa_decode_shared_prefix" if prefix else
+                       "pa_forward_decode" if fused else "pa_decode"),
             "flops_per_launch": attention_flops(w), "launch_us": t_dec * 1e3,
             "peak_source": tpeak_src, "hbm_gbs": achieved, "hbm_frac": achieved / peak,
         }
@@ -551,7 +568,7 @@ def run_ours(args):
         "seq_tokens_per_s": seqs_all / (t_step_max * 1e-3),
         "context_tokens_per_s": ctx_all / (t_step_max * 1e-3),
         "hbm_frac_step": (bytes_all / (t_step_max * 1e-3) / 1e9) / (peak * world),
-        "roofline": roofline_tensor if prefix else {
+        "roofline": roofline_tensor if roofline_tensor is not None else {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
             "kernel": ("pa_forward_decode" if fused else

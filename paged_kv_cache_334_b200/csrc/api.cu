@@ -233,11 +233,25 @@ struct WorkspaceLayout {
   size_t part_max, part_sum, part_out, counters, total;
   int32_t max_parts;
   bool stream;
+  bool tensor;  // the tensor-core path (suffix.cu) with no prefix
 };
 
+bool suffix_kernel_serves(const pa_cache_desc *c, int32_t group);
+struct SuffixLayout {
+  size_t part_ml, part_o, merge, seq_ml, seq_o, total;
+};
+SuffixLayout suffix_layout(const pa_cache_desc *c, int32_t batch, int32_t num_q_heads);
+
 WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
-                              int32_t num_q_heads, int32_t max_blocks) {
+                              int32_t num_q_heads, int32_t max_blocks,
+                              bool allow_tensor = true) {
   WorkspaceLayout w{};
+  if (allow_tensor && suffix_kernel_serves(c, num_q_heads / c->num_kv_heads)) {
+    // groups of 64 or 128 query heads: decode on the tensor cores
+    w.tensor = true;
+    w.total = suffix_layout(c, batch, num_q_heads).total;
+    return w;
+  }
   const StreamPlan sp = plan_stream(c, num_q_heads);
   if (sp.ok) {
     // persistent kernel: (max, sum) and output per (CTA, head/tail slot, query
@@ -272,12 +286,9 @@ WorkspaceLayout decode_layout(const pa_cache_desc *c, int32_t batch,
 // head), one merge record per (sequence, KV head), the per-row results).
 bool suffix_kernel_serves(const pa_cache_desc *c, int32_t group) {
   return c->dtype == PA_DTYPE_BF16 && (group == 64 || group == 128) &&
-         (c->head_dim == 64 || c->head_dim == 128);
+         (c->head_dim == 64 || c->head_dim == 128) && c->block_size >= 8 &&
+         c->block_size <= 128;
 }
-
-struct SuffixLayout {
-  size_t part_ml, part_o, merge, seq_ml, seq_o, total;
-};
 
 SuffixLayout suffix_layout(const pa_cache_desc *c, int32_t batch, int32_t num_q_heads) {
   SuffixLayout l{};
@@ -290,6 +301,85 @@ SuffixLayout suffix_layout(const pa_cache_desc *c, int32_t batch, int32_t num_q_
   l.seq_o = round_up(l.seq_ml + rows * 2 * sizeof(float));
   l.total = round_up(l.seq_o + rows * (size_t)c->head_dim * sizeof(float));
   return l;
+}
+
+// Arguments and tensor maps of the suffix kernel: q (boxes of 64 x group x
+// 1), the caches (64 x block_size x 1), and the fp32 rows it stores.
+pa_status make_suffix_params(const pa_cache_desc *cache, const void *q, const void *key_cache,
+                             const void *value_cache, const int32_t *block_tables,
+                             const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+                             int32_t max_blocks_per_seq, int32_t prefix_blocks, float scale,
+                             char *ws, int32_t *err_word, pa::SuffixParams *sp) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable%s");
+  const int sms = device_sm_count();
+  if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  const int32_t bs = cache->block_size;
+  const SuffixLayout l = suffix_layout(cache, batch, num_q_heads);
+  *sp = pa::SuffixParams{};
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim, (cuuint64_t)num_q_heads,
+                                (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)cache->head_dim * 2,
+                                   (cuuint64_t)num_q_heads * cache->head_dim * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)group, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&sp->tmap_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
+  }
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim,
+                                (cuuint64_t)cache->num_blocks * (cuuint64_t)bs,
+                                (cuuint64_t)cache->num_kv_heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)cache->num_kv_heads * cache->head_dim * 2,
+                                   (cuuint64_t)cache->head_dim * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)bs, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    for (int which = 0; which < 2; ++which) {
+      if (fn(which ? &sp->tmap_v : &sp->tmap_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(which ? value_cache : key_cache), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return fail(PA_ERR_CUDA, "cannot describe the caches for the tensor copies%s");
+    }
+  }
+  // fp32 rows of D (seq_o, part_o) for the epilogue's tiled stores
+  auto encode_rows = [&](CUtensorMap *map, char *base, size_t rows) -> bool {
+    const cuuint64_t dims[2] = {(cuuint64_t)cache->head_dim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cache->head_dim * 4};
+    const cuuint32_t box[2] = {32, (cuuint32_t)group};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  if (!encode_rows(&sp->tmap_seq_o, ws + l.seq_o, (size_t)batch * num_q_heads) ||
+      !encode_rows(&sp->tmap_part_o, ws + l.part_o,
+                   (size_t)pa::stream::kMaxGrid * 2 * num_q_heads))
+    return fail(PA_ERR_CUDA, "cannot describe the suffix results for the tensor copies%s");
+  sp->block_tables = block_tables;
+  sp->context_lens = context_lens;
+  sp->seq_ml = reinterpret_cast<float *>(ws + l.seq_ml);
+  sp->seq_o = reinterpret_cast<float *>(ws + l.seq_o);
+  sp->part_ml = reinterpret_cast<float *>(ws + l.part_ml);
+  sp->part_o = reinterpret_cast<float *>(ws + l.part_o);
+  sp->merge = reinterpret_cast<int32_t *>(ws + l.merge);
+  sp->slot_mapping = nullptr;
+  sp->err_word = err_word;
+  sp->batch = batch;
+  sp->num_q_heads = num_q_heads;
+  sp->num_kv_heads = cache->num_kv_heads;
+  sp->group = group;
+  sp->block_size = bs;
+  sp->table_stride = max_blocks_per_seq;
+  sp->prefix_blocks = prefix_blocks;
+  sp->num_blocks = cache->num_blocks;
+  sp->grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
+  sp->scale_log2 = scale * 1.4426950408889634f;
+  return PA_OK;
 }
 
 }  // namespace
@@ -309,7 +399,7 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
                       int32_t max_blocks_per_seq, float scale, void *workspace,
                       size_t workspace_bytes, int32_t *err_word, pa_stream_t stream,
                       int32_t prefix_blocks = 0, float *seq_ml = nullptr,
-                      float *seq_o = nullptr) {
+                      float *seq_o = nullptr, bool allow_tensor = true) {
   pa_status s = check_decode_common(cache, q, key_cache, value_cache, block_tables,
                                     context_lens, batch, num_q_heads,
                                     max_blocks_per_seq, scale);
@@ -321,13 +411,40 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
   }
   if (batch == 0) return PA_OK;
   if ((s = check_ptr(out, "out")) != PA_OK) return s;
-  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq,
+                                          allow_tensor && prefix_blocks == 0);
   if (workspace_bytes < w.total)
     return fail(PA_ERR_INVALID_ARG, "workspace too small%s: need %lld bytes", "",
                 (long long)w.total);
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
     return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned%s");
   char *ws = static_cast<char *>(workspace);
+  if (w.tensor) {
+    // groups of 64 or 128 query heads per KV head: the tensor-core kernel
+    // over 128-token tiles of every (sequence, KV head) pair, then one pass
+    // that merges pairs cut between CTAs and writes bf16 out
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (fused) {
+      const int64_t row_bytes =
+          (int64_t)cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype);
+      const cudaError_t e = pa::launch_write_kv(cache->dtype, cache->block_size,
+                                                cache->num_blocks, row_bytes, key_cache,
+                                                value_cache, k_new, v_new, slot_mapping, batch,
+                                                err_word, st, block_tables, context_lens,
+                                                max_blocks_per_seq);
+      if (e != cudaSuccess) return fail(PA_ERR_CUDA, "write_kv launch: %s", cudaGetErrorString(e));
+    }
+    pa::SuffixParams sp;
+    s = make_suffix_params(cache, q, key_cache, value_cache, block_tables, context_lens, batch,
+                           num_q_heads, max_blocks_per_seq, 0, scale, ws, err_word, &sp);
+    if (s != PA_OK) return s;
+    sp.slot_mapping = slot_mapping;
+    cudaError_t e = pa::launch_suffix(sp, cache->head_dim, st);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    e = pa::launch_finish(sp, out, cache->head_dim, st);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+  }
   if (prefix_blocks > 0 && !w.stream)
     return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs the persistent kernel's shapes%s");
   if (w.stream) {
@@ -434,6 +551,31 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
   return PA_OK;
 }
 
+namespace pa {
+// pa_decode restricted to the page-stream and partition kernels, and its
+// workspace size: the tensor-core path's workspace (per-row results and
+// per-CTA partials of 64 or 128 query heads) outgrows pa_decode_noalloc's
+// fixed scratch.
+size_t decode_workspace_bytes_streamed(const pa_cache_desc *cache, int32_t batch,
+                                       int32_t num_q_heads, int32_t max_blocks_per_seq) {
+  if (check_cache(cache) != PA_OK || batch < 0 || num_q_heads <= 0 ||
+      num_q_heads % cache->num_kv_heads != 0 || max_blocks_per_seq < 0)
+    return 0;
+  return decode_layout(cache, batch, num_q_heads, max_blocks_per_seq, false).total;
+}
+pa_status decode_streamed(const pa_cache_desc *cache, void *out, const void *q,
+                          const void *key_cache, const void *value_cache,
+                          const int32_t *block_tables, const int32_t *context_lens,
+                          int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                          float scale, void *workspace, size_t workspace_bytes,
+                          int32_t *err_word, pa_stream_t stream) {
+  return decode_impl(cache, out, q, const_cast<void *>(key_cache),
+                     const_cast<void *>(value_cache), nullptr, nullptr, nullptr, block_tables,
+                     context_lens, batch, num_q_heads, max_blocks_per_seq, scale, workspace,
+                     workspace_bytes, err_word, stream, 0, nullptr, nullptr, false);
+}
+}  // namespace pa
+
 extern "C" {
 
 int32_t pa_version(void) { return 100; }
@@ -498,6 +640,7 @@ pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
                      workspace_bytes, err_word, stream);
 }
 
+
 pa_status pa_forward_decode(const pa_cache_desc *cache, void *out, const void *q,
                             void *key_cache, void *value_cache, const void *k_new,
                             const void *v_new, const int64_t *slot_mapping,
@@ -519,7 +662,8 @@ size_t pa_decode_shared_prefix_workspace_bytes(const pa_cache_desc *cache, int32
       num_q_heads % cache->num_kv_heads != 0 || prefix_blocks < 0 ||
       max_blocks_per_seq < prefix_blocks)
     return 0;
-  const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+  const WorkspaceLayout w =
+      decode_layout(cache, batch, num_q_heads, max_blocks_per_seq, /*allow_tensor=*/false);
   const size_t rows = (size_t)batch * num_q_heads;
   const size_t stream_path = w.total + round_up(rows * 2 * sizeof(float)) +
                              round_up(rows * (size_t)cache->head_dim * sizeof(float));
@@ -606,46 +750,11 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
   //    groups of 64 or 128 query heads, else on the page-stream kernel; one
   //    (max, normaliser, normalised output) per row, or partials of cut pairs
   if (suffix_kernel_serves(cache, group)) {
-    const SuffixLayout l = suffix_layout(cache, batch, num_q_heads);
-    const int sms = device_sm_count();
-    if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
-    pa::SuffixParams sp{};
-    if (!encode_q(&sp.tmap_q, (cuuint32_t)group, 1))
-      return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
-    sp.tmap_k = pp.tmap_k;
-    sp.tmap_v = pp.tmap_v;
-    // fp32 rows of D (seq_o, part_o) for the epilogue's tiled stores
-    auto encode_rows = [&](CUtensorMap *map, char *base, size_t rows) -> bool {
-      const cuuint64_t dims[2] = {(cuuint64_t)cache->head_dim, (cuuint64_t)rows};
-      const cuuint64_t strides[1] = {(cuuint64_t)cache->head_dim * 4};
-      const cuuint32_t box[2] = {32, (cuuint32_t)group};
-      const cuuint32_t estr[2] = {1, 1};
-      return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-    };
-    if (!encode_rows(&sp.tmap_seq_o, ws + l.seq_o, (size_t)batch * num_q_heads) ||
-        !encode_rows(&sp.tmap_part_o, ws + l.part_o,
-                     (size_t)pa::stream::kMaxGrid * 2 * num_q_heads))
-      return fail(PA_ERR_CUDA, "cannot describe the suffix results for the tensor copies%s");
-    sp.block_tables = block_tables;
-    sp.context_lens = context_lens;
-    sp.seq_ml = reinterpret_cast<float *>(ws + l.seq_ml);
-    sp.seq_o = reinterpret_cast<float *>(ws + l.seq_o);
-    sp.part_ml = reinterpret_cast<float *>(ws + l.part_ml);
-    sp.part_o = reinterpret_cast<float *>(ws + l.part_o);
-    sp.merge = reinterpret_cast<int32_t *>(ws + l.merge);
-    sp.err_word = err_word;
-    sp.batch = batch;
-    sp.num_q_heads = num_q_heads;
-    sp.num_kv_heads = cache->num_kv_heads;
-    sp.group = group;
-    sp.block_size = bs;
-    sp.table_stride = max_blocks_per_seq;
-    sp.prefix_blocks = prefix_blocks;
-    sp.num_blocks = cache->num_blocks;
-    sp.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
-    sp.scale_log2 = scale_log2;
+    pa::SuffixParams sp;
+    s = make_suffix_params(cache, q, key_cache, value_cache, block_tables, context_lens, batch,
+                           num_q_heads, max_blocks_per_seq, prefix_blocks, scale, ws, err_word,
+                           &sp);
+    if (s != PA_OK) return s;
     const cudaError_t e = pa::launch_suffix(sp, cache->head_dim, st);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "suffix launch: %s", cudaGetErrorString(e));
     pp.seq_ml = sp.seq_ml;
@@ -654,7 +763,8 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
     pp.part_ml = sp.part_ml;
     pp.part_o = sp.part_o;
   } else {
-    const WorkspaceLayout w = decode_layout(cache, batch, num_q_heads, max_blocks_per_seq);
+    const WorkspaceLayout w =
+        decode_layout(cache, batch, num_q_heads, max_blocks_per_seq, /*allow_tensor=*/false);
     const size_t rows = (size_t)batch * num_q_heads;
     float *seq_ml = reinterpret_cast<float *>(ws + w.total);
     float *seq_o = reinterpret_cast<float *>(ws + w.total + round_up(rows * 2 * sizeof(float)));

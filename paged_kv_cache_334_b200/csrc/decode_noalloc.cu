@@ -17,6 +17,19 @@
 #include "../../include/pa.h"
 #include "pa_launch.h"
 
+namespace pa {
+// api.cu: pa_decode on the page-stream / partition kernels only (the
+// tensor-core path for groups of 64 or 128 heads needs more scratch).
+size_t decode_workspace_bytes_streamed(const pa_cache_desc *cache, int32_t batch,
+                                       int32_t num_q_heads, int32_t max_blocks_per_seq);
+pa_status decode_streamed(const pa_cache_desc *cache, void *out, const void *q,
+                          const void *key_cache, const void *value_cache,
+                          const int32_t *block_tables, const int32_t *context_lens,
+                          int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                          float scale, void *workspace, size_t workspace_bytes,
+                          int32_t *err_word, pa_stream_t stream);
+}  // namespace pa
+
 namespace {
 
 constexpr size_t kScratchBytes = PA_DECODE_NOALLOC_SCRATCH_BYTES;
@@ -72,7 +85,7 @@ extern "C" pa_status pa_decode_noalloc(const pa_cache_desc *cache, void *out,
                                        int32_t max_blocks_per_seq, float scale,
                                        int32_t *err_word, pa_stream_t stream) {
   const size_t need =
-      pa_decode_workspace_bytes(cache, batch, num_q_heads, max_blocks_per_seq);
+      pa::decode_workspace_bytes_streamed(cache, batch, num_q_heads, max_blocks_per_seq);
   if (need > kScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof msg,
@@ -84,9 +97,9 @@ extern "C" pa_status pa_decode_noalloc(const pa_cache_desc *cache, void *out,
   }
   if (need == 0 || batch == 0) {
     // Invalid arguments or an empty batch: pa_decode reports / does nothing.
-    return pa_decode(cache, out, q, key_cache, value_cache, block_tables,
-                     context_lens, batch, num_q_heads, max_blocks_per_seq, scale,
-                     nullptr, 0, err_word, stream);
+    return pa::decode_streamed(cache, out, q, key_cache, value_cache, block_tables,
+                               context_lens, batch, num_q_heads, max_blocks_per_seq, scale,
+                               nullptr, 0, err_word, stream);
   }
   void *scratch = nullptr;
   pa_status s = scratch_address(&scratch);
@@ -100,7 +113,7 @@ extern "C" pa_status pa_decode_noalloc(const pa_cache_desc *cache, void *out,
     pa::set_last_error_message(msg);
     return PA_ERR_CUDA;
   }
-  return pa_decode(cache, out, q, key_cache, value_cache, block_tables,
-                   context_lens, batch, num_q_heads, max_blocks_per_seq, scale,
-                   scratch, kScratchBytes, err_word, stream);
+  return pa::decode_streamed(cache, out, q, key_cache, value_cache, block_tables,
+                             context_lens, batch, num_q_heads, max_blocks_per_seq, scale,
+                             scratch, kScratchBytes, err_word, stream);
 }

@@ -143,6 +143,10 @@ struct SuffixParams {
   float *seq_ml, *seq_o;    // pairs inside one CTA's range: [batch][Hq][2], [batch][Hq][D]
   float *part_ml, *part_o;  // cut pairs: [grid * 2][Hq][2], [grid * 2][Hq][D]
   int32_t *merge;           // [batch * Hkv][4], as read by the prefix kernel
+  // pa_forward_decode: sequence b's newest token must sit in slot_mapping[b]
+  // as the table gives position ctx - 1, else PA_DEVERR_SLOT and its output
+  // is zeroed (NULL: no check)
+  const int64_t *slot_mapping;
   int32_t *err_word;
   int32_t batch, num_q_heads, num_kv_heads, group, block_size, table_stride, prefix_blocks,
       num_blocks, grid;
@@ -150,6 +154,9 @@ struct SuffixParams {
 };
 size_t suffix_smem_bytes(int head_dim, int group);
 cudaError_t launch_suffix(const SuffixParams &p, int head_dim, cudaStream_t stream);
+// pa_decode on the tensor-core path (no prefix): each (sequence, KV head)
+// pair's rows from its result or its partials, as bf16 `out` rows.
+cudaError_t launch_finish(const SuffixParams &p, void *out, int head_dim, cudaStream_t stream);
 
 // Query heads handled together by one CTA for a GQA group of `group` heads.
 int decode_head_tile(int group);

@@ -62,7 +62,7 @@ constexpr int kTileBox = kTok * 128;  // bytes of one 64-wide half of a K or V t
 constexpr int kRing = 8;              // tile descriptors in flight
 constexpr int kMaxPPT = 16;           // pages per tile (block_size >= 8)
 constexpr int kQStages = 2, kVStages = 2, kMaxKStages = 3;
-constexpr int kFirst = 1, kLast = 2, kBad = 4, kDirect = 8;
+constexpr int kFirst = 1, kLast = 2, kBad = 4, kDirect = 8, kPairEnd = 16;
 // At least this much shared memory per CTA keeps one CTA per SM: tensor
 // memory is allocated whole (512 columns) and is not shared.
 constexpr size_t kMinSmem = 120 * 1024;
@@ -96,6 +96,7 @@ struct alignas(16) Shared {
   uint32_t tmem_base;
   Desc desc[kRing];
   int32_t pids[kRing][kMaxPPT];  // page ids of a tile, written by asynchronous copies
+  int64_t slots[kRing];          // new-token slot of the pair ending in the tile
   float xm[2][2][128];           // [tile parity][column half][row] partial row maxima
   float xl[2][128];              // [column half][row] partial normalisers
   float2 mlst[128];              // epilogue staging of (max, normaliser) per row
@@ -352,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool pair_end = wk.j == wk.n - 1;
       const bool last = pair_end || u == n_units - 1;
       const bool direct = wk.P >= start && wk.P + wk.n <= end;
-      x.flags = (first ? kFirst : 0) | (last ? kLast : 0) | (direct ? kDirect : 0);
+      x.flags = (first ? kFirst : 0) | (last ? kLast : 0) | (direct ? kDirect : 0) |
+                (pair_end ? kPairEnd : 0);
       const int slot = (start < wk.P) ? 1 : 0;
       x.row = direct ? wk.s * Hq + wk.h * G : (c * 2 + slot) * Hq + wk.h * G;
       if (pair_end && lane == 0) {
@@ -366,6 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t *trow =
           p.block_tables + (int64_t)wk.s * p.table_stride + p.prefix_blocks + wk.j * ppt;
       if (lane < x.npg) cp_async_4(&sh.pids[u % kRing][lane], trow + lane);
+      if (pair_end && p.slot_mapping != nullptr && lane == 0)
+        cp_async_8(&sh.slots[u % kRing], p.slot_mapping + wk.s);
       cp_async_commit();
       if (u + 1 < n_units) wk.advance(p, lane);
       return x;
@@ -389,8 +393,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         pb = in ? sh.pids[u % kRing][lane] : 0;
         const bool bad_pb = in && (pb < 0 || pb >= p.num_blocks);
         if (bad_pb) pb = 0;  // any valid page: the pair's output is flagged
-        const bool bad = __any_sync(0xffffffffu, bad_pb);
+        bool bad = __any_sync(0xffffffffu, bad_pb);
         if (bad && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
+        if ((t0.flags & kPairEnd) && p.slot_mapping != nullptr) {
+          // the pair's newest token (its last tile's last token) must have
+          // been written to the slot the table gives it
+          const int64_t slot = __shfl_sync(0xffffffffu, sh.slots[u % kRing], 0);
+          const int32_t pb_last = __shfl_sync(0xffffffffu, pb, t0.npg - 1);
+          const int64_t want = (int64_t)pb_last * bs + (t0.ntok - 1) % bs;
+          if (slot >= 0 && (bad || slot != want)) {
+            bad = true;
+            if (lane == 0) set_error(p.err_word, PA_DEVERR_SLOT);
+          }
+        }
         if (u >= kRing && !wait_all(&sh.dempty[u % kRing], ((u / kRing) - 1) & 1, sh, p, lane)) {
           ok = false;
           break;
@@ -820,6 +835,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// pa_decode on this path (no prefix): each (sequence, KV head) pair's G rows
+// from its one result or from the partials of the CTAs that cut it (the
+// running-max merge), as bf16; zeros for an empty pair, a bad page, a bad
+// new-token slot or a length outside the table.  One block per pair.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) finish_kernel(const __grid_constant__ SuffixParams p,
+                                                     __nv_bfloat16 *out) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int pair = blockIdx.x;
+  const int s = pair / p.num_kv_heads, h = pair - s * p.num_kv_heads;
+  const int4 md = __ldcg(reinterpret_cast<const int4 *>(p.merge) + pair);
+  const int n = md.w != 0 ? 0 : md.y;
+  const float2 *mls = reinterpret_cast<const float2 *>(n == 1 ? p.seq_ml : p.part_ml);
+  const float *obase = n == 1 ? p.seq_o : p.part_o;
+  for (int f = threadIdx.x * 4; f < p.group * D; f += blockDim.x * 4) {
+    const int hh = f / D, d0 = f - hh * D;
+    const int64_t row = (int64_t)s * p.num_q_heads + (int64_t)h * p.group + hh;
+    auto crow = [&](int x) -> int64_t {
+      return n == 1 ? row
+                    : ((int64_t)(md.x + x) * 2 + (x == 0 ? md.z : 0)) * p.num_q_heads +
+                          (int64_t)h * p.group + hh;
+    };
+    float M = -INFINITY;
+    bool bad = false;
+    for (int x = 0; x < n; ++x) {
+      const float2 ml = __ldcg(mls + crow(x));
+      bad |= ml.y < 0.f;
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float W = 0.f;
+    if (!bad) {
+      for (int x = 0; x < n; ++x) {
+        const int64_t cr = crow(x);
+        const float2 ml = __ldcg(mls + cr);
+        if (!(ml.y > 0.f)) continue;
+        const float w = ml.y * ex2(ml.x - M);
+        const float4 o = __ldcg(reinterpret_cast<const float4 *>(obase + cr * D + d0));
+        W += w;
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
+      }
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    Elem<__nv_bfloat16>::store4(out, row * D + d0,
+                                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
+  }
+}
+
 template <int D, int M>
 size_t smem_bytes() {
   using C = Cfg<D, M>;
@@ -861,6 +929,25 @@ cudaError_t launch_dm(const SuffixParams &p, cudaStream_t stream) {
 size_t suffix_smem_bytes(int head_dim, int group) {
   if (head_dim == 64) return group == 64 ? suffix::smem_bytes<64, 64>() : suffix::smem_bytes<64, 128>();
   return group == 64 ? suffix::smem_bytes<128, 64>() : suffix::smem_bytes<128, 128>();
+}
+
+cudaError_t launch_finish(const SuffixParams &p, void *out, int head_dim, cudaStream_t stream) {
+  const int64_t blocks = (int64_t)p.batch * p.num_kv_heads;
+  if (blocks == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+  if (head_dim == 64) return cudaLaunchKernelEx(&cfg, suffix::finish_kernel<64>, p, o);
+  if (head_dim == 128) return cudaLaunchKernelEx(&cfg, suffix::finish_kernel<128>, p, o);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_suffix(const SuffixParams &p, int head_dim, cudaStream_t stream) {

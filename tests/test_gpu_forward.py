@@ -122,6 +122,8 @@ def _slot_case(dtype, Hq, Hkv, D, bs):
     (wl.DTYPE_BF16, 32, 8, 128, 16),   # persistent kernel, tensor-core consumers
     (wl.DTYPE_F32, 8, 4, 64, 8),       # persistent kernel, CUDA-core consumers
     (wl.DTYPE_BF16, 6, 2, 128, 16),    # group 3: partition kernel after a checked write
+    (wl.DTYPE_BF16, 64, 1, 128, 32),   # group 64: tensor-core tiles after a checked write
+    (wl.DTYPE_BF16, 128, 1, 64, 16),   # group 128, head_dim 64
 ])
 def test_forward_decode_slot_checks(dtype, Hq, Hkv, D, bs):
     w, kn, vn, sm, bad_slot, own0 = _slot_case(dtype, Hq, Hkv, D, bs)

@@ -176,7 +176,7 @@ def test_boundary_context_lengths(dtype, Hq, Hkv, D, bs):
     assert np.all(got[np.asarray(lens) == 0] == 0)
 
 
-@pytest.mark.parametrize("group", [1, 2, 3, 4, 5, 8, 12, 16, 64])
+@pytest.mark.parametrize("group", [1, 2, 3, 4, 5, 8, 12, 16, 64, 128])
 def test_group_sizes(group):
     Hkv = 2 if group < 64 else 1
     w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=5, num_q_heads=group * Hkv,
@@ -442,3 +442,31 @@ def test_stream_repeated_calls_keep_workspace_clean():
         assert torch.equal(o.view(torch.uint16), outs[0].view(torch.uint16))
     ref, _, _, _ = oracle_after_write(w)
     assert_close(to_f64(outs[0]), ref, w.dtype, "long split")
+
+
+# Groups of 64 or 128 query heads per KV head decode on the tensor cores:
+# 128-token tiles of every (sequence, KV head) pair split evenly over one CTA
+# per SM; pairs cut between CTAs are merged by a second pass.
+@pytest.mark.parametrize("Hq,Hkv,D,bs,lens", [
+    (128, 2, 128, 16, [40000, 1, 0, 7000]),          # pairs spanning dozens of CTAs
+    (64, 1, 128, 64, [129, 128, 127, 1, 2, 3, 4096]),
+    (256, 2, 64, 32, [1000, 0, 33, 2500, 1]),         # 128 heads per KV head
+])
+def test_tensor_decode_long_and_ragged(Hq, Hkv, D, bs, lens):
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=len(lens), num_q_heads=Hq,
+                           num_kv_heads=Hkv, head_dim=D, block_size=bs, context_lens=lens,
+                           seed=Hq + bs, new_tokens=True)
+    d = upload(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gpu_write_and_decode(w, d, err)
+    again = torch.empty_like(out)
+    pa.pa_decode(again, d["q"], d["key_cache"], d["value_cache"], d["block_tables"],
+                 d["context_lens"], err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref, _, _, _ = oracle_after_write(w)
+    assert_close(to_f64(out), ref, w.dtype, f"tensor decode {Hq}/{Hkv} D{D} bs{bs}")
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert not to_f64(out)[b].any()
