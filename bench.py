@@ -412,14 +412,14 @@ def run_ours(args):
     if prefix and not w.shared_prefix_blocks:
         raise SystemExit(f"--step prefix needs a workload with a shared prefix, not {w.name}")
     # libpa kernels per step.  Groups of 64 or 128 query heads (tensor-core
-    # path): the checked write (inside pa_forward_decode or as its own call),
-    # the tile kernel and its finishing pass; with a shared prefix the tile
-    # kernel and the prefix kernel.  Other groups: the persistent decode
+    # path): the write (inside pa_forward_decode or as its own call), the
+    # tile kernel, and its finishing pass or, with a shared prefix, the
+    # prefix kernel.  Other groups: the persistent decode
     # kernel and its merge kernel, plus the write kernel when the write is a
     # separate call, plus the prefix kernel of the shared-prefix path.
     tensor = tensor_path(w)
     if tensor:
-        launches_per_step = 2 if prefix else 2 + (1 if has_new else 0)
+        launches_per_step = 2 + (1 if has_new else 0)
     else:
         launches_per_step = 2 + (1 if has_new and not fused else 0) + (1 if prefix else 0)
 
