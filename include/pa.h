@@ -148,7 +148,11 @@ size_t pa_decode_workspace_bytes(const pa_cache_desc *cache, int32_t batch,
  * buffer serves any number of stream-ordered calls.  Calls that overlap on
  * the GPU must not share a workspace.  A call may run as more than one
  * kernel; the later ones are launched with programmatic stream
- * serialisation and wait for the earlier ones.
+ * serialisation and wait for the earlier ones.  bf16 caches with 64 or 128
+ * query heads per KV head (head_dim 64 or 128, block_size 8..128) are
+ * computed on the tensor cores in tiles of 128 tokens (the serving page's
+ * section 4.1: many queries per KV page make the work a dense
+ * contraction); the result is the same up to rounding.
  */
 pa_status pa_decode(const pa_cache_desc *cache, void *out, const void *q,
                     const void *key_cache, const void *value_cache,
@@ -217,8 +221,10 @@ pa_status pa_forward_decode(const pa_cache_desc *cache, void *out, const void *q
  * PA_DEVERR_PREFIX and its output is zeroed; a bad prefix block id sets
  * PA_DEVERR_BLOCK_ID and zeroes every output.  Shapes: bf16, head_dim 64
  * or 128, query heads per KV head dividing 128, block_size 8..128 (a power
- * of two), prefix_blocks <= 2048, and a shape pa_decode serves with its
- * persistent kernel (else PA_ERR_UNSUPPORTED).  prefix_blocks == 0 is
+ * of two), prefix_blocks <= 2048; with fewer than 64 query heads per KV
+ * head also a shape pa_decode serves with its persistent page-stream kernel
+ * (else PA_ERR_UNSUPPORTED).  With 64 or 128 heads per KV head the suffix
+ * runs on the tensor cores too.  prefix_blocks == 0 is
  * pa_decode.  workspace: at least pa_decode_shared_prefix_workspace_bytes
  * bytes, 256-byte aligned, zero-filled before first use (as pa_decode's).
  */
