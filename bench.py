@@ -66,6 +66,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="gqa_bf16", choices=wl.WORKLOADS)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--block-size", type=int, default=None,
+                    help="page size override for gqa_bf16 / mixed_bf16 / long_bf16 (a sweep)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -344,7 +346,7 @@ def run_reference(args):
     world, rank, local = dist_env()
     if rank != 0:
         return 0
-    w = wl.make_workload(args.workload, seed=args.seed)
+    w = wl.make_workload(args.workload, seed=args.seed, block_size=args.block_size)
     nbytes_full = wl.roofline_bytes(w)
     budget = max(2.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     per_step, sample, cores, desc = time_oracle(w, budget, max_reps=1)
@@ -383,7 +385,8 @@ def run_ours(args):
     dist = init_dist(world, local)
     pa.load()
 
-    w = wl.make_workload(args.workload, seed=rank_seed(args.seed, rank))
+    w = wl.make_workload(args.workload, seed=rank_seed(args.seed, rank),
+                         block_size=args.block_size)
     tdt = torch.float32 if w.dtype == wl.DTYPE_F32 else torch.bfloat16
 
     def dev_t(a):
@@ -570,7 +573,8 @@ def run_ours(args):
         "hbm_frac_step": (bytes_all / (t_step_max * 1e-3) / 1e9) / (peak * world),
         "roofline": roofline_tensor if roofline_tensor is not None else {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+            "frac": achieved / peak,
+            "traffic": recorded_traffic(args.workload) if args.block_size is None else None,
             "kernel": ("pa_forward_decode" if fused else
                        "pa_decode_shared_prefix" if prefix else "pa_decode"),
             "algorithmic_bytes_per_launch": dec_bytes,

@@ -180,9 +180,18 @@ def _scattered_tables(rng, ctx, bs, MB, slack=0.2, prefix_blocks=0):
     return tables, NB
 
 
-def make_workload(name: str, seed: int = 0, batch: Optional[int] = None) -> Workload:
+def make_workload(name: str, seed: int = 0, batch: Optional[int] = None,
+                  block_size: Optional[int] = None) -> Workload:
     """Build one of the named workloads.  `batch` overrides the batch size
-    (used for reduced-size variants of the large workloads)."""
+    (used for reduced-size variants of the large workloads); `block_size`
+    (a power of two) overrides the page size of gqa_bf16, mixed_bf16 and
+    long_bf16 (the same lengths and values, paged differently: a page-size
+    sweep)."""
+    if block_size is not None:
+        if name not in ("gqa_bf16", "mixed_bf16", "long_bf16"):
+            raise ValueError(f"block_size override is for gqa_bf16, mixed_bf16, long_bf16, not {name}")
+        if block_size < 1 or block_size & (block_size - 1):
+            raise ValueError(f"block_size must be a power of two, not {block_size}")
     rng = np.random.Generator(np.random.PCG64(seed))
     if name == "tiny_fp32":
         B, Hq, Hkv, D, bs, NB = 3, 4, 4, 64, 4, 16
@@ -199,16 +208,16 @@ def make_workload(name: str, seed: int = 0, batch: Optional[int] = None) -> Work
                        description="B3 Hq4/Hkv4 D64 bs4 NB16 ctx[5,9,12] fp32")
     if name == "gqa_bf16":
         B = batch or 32
-        Hq, Hkv, D, bs = 32, 8, 128, 16
+        Hq, Hkv, D, bs = 32, 8, 128, block_size or 16
         ctx = rng.integers(128, 2048, size=B, endpoint=True).astype(np.int32)
         MB = _pages(2048, bs)
         tables, NB = _scattered_tables(rng, ctx, bs, MB)
         return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
                        tables, new_tokens=True, seed=seed,
-                       description=f"B{B} Hq32/Hkv8 D128 bs16 ctx~U[128,2048] bf16")
+                       description=f"B{B} Hq32/Hkv8 D128 bs{bs} ctx~U[128,2048] bf16")
     if name == "mixed_bf16":
         B = batch or 128
-        Hq, Hkv, D, bs = 32, 8, 128, 16
+        Hq, Hkv, D, bs = 32, 8, 128, block_size or 16
         base = rng.choice(np.array([128, 4096, 16000]), size=B, p=[0.5, 0.35, 0.15])
         jitter = rng.integers(0, 15, size=B, endpoint=True)
         ctx = (base + jitter).astype(np.int32)
@@ -216,16 +225,16 @@ def make_workload(name: str, seed: int = 0, batch: Optional[int] = None) -> Work
         tables, NB = _scattered_tables(rng, ctx, bs, MB)
         return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
                        tables, new_tokens=True, seed=seed,
-                       description=f"B{B} Hq32/Hkv8 D128 bs16 ctx {{128,4096,16000}}+U[0,15] bf16")
+                       description=f"B{B} Hq32/Hkv8 D128 bs{bs} ctx {{128,4096,16000}}+U[0,15] bf16")
     if name == "long_bf16":
         B = batch or 4
-        Hq, Hkv, D, bs, L = 32, 8, 128, 16, 131072
+        Hq, Hkv, D, bs, L = 32, 8, 128, block_size or 16, 131072
         ctx = np.full(B, L, dtype=np.int32)
         MB = _pages(L, bs)
         tables, NB = _scattered_tables(rng, ctx, bs, MB, slack=0.0)
         return _finish(name, DTYPE_BF16, rng, B, Hq, Hkv, D, bs, NB, MB, ctx,
                        tables, new_tokens=True, partition_tokens=512, seed=seed,
-                       description=f"B{B} ctx131072 Hq32/Hkv8 D128 bs16 bf16, 512-token partitions")
+                       description=f"B{B} ctx131072 Hq32/Hkv8 D128 bs{bs} bf16, 512-token partitions")
     if name == "mqa_prefix_bf16":
         B = batch or 256
         Hq, Hkv, D, bs, prefix = 64, 1, 128, 32, 2048

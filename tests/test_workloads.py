@@ -85,3 +85,28 @@ def test_roofline_bytes_counts_shared_prefix_once():
     write = 2 * (w.k_new.nbytes + w.v_new.nbytes) + w.slot_mapping.nbytes
     assert wl.roofline_bytes(w) == kv_unique + qo + meta + write
     assert wl.roofline_bytes(w, include_write=False) == kv_unique + qo + meta
+
+
+def test_block_size_override_keeps_lengths_and_pages_them_anew():
+    """A page-size sweep: the same context lengths, paged with another block
+    size, still a consistent allocator (every visible token in its own slot)."""
+    base = wl.make_workload("gqa_bf16", seed=2)
+    assert base.block_size == 16
+    assert wl.make_workload("gqa_bf16", seed=2, block_size=16).block_tables.tolist() == \
+        base.block_tables.tolist()
+    for bs in (8, 64, 256):
+        w = wl.make_workload("gqa_bf16", seed=2, block_size=bs)
+        assert w.block_size == bs
+        assert w.context_lens.tolist() == base.context_lens.tolist()
+        seen = set()
+        for b, ctx in enumerate(w.context_lens):
+            for t in range(0, int(ctx), 97):
+                pb = int(w.block_tables[b, t // bs])
+                assert 0 <= pb < w.num_blocks
+                key = (pb, t % bs)
+                assert key not in seen
+                seen.add(key)
+    with pytest.raises(ValueError):
+        wl.make_workload("gqa_bf16", block_size=48)
+    with pytest.raises(ValueError):
+        wl.make_workload("mqa_prefix_bf16", block_size=16)
