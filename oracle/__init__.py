@@ -65,6 +65,11 @@ def _load():
         lib.orc_merge.restype = None
         lib.orc_write_kv_cache.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32]
         lib.orc_write_kv_cache.restype = ctypes.c_int
+        f32 = ctypes.c_float
+        lib.orc_e4m3_encode_array.argtypes = [P, i64, P]
+        lib.orc_e4m3_encode_array.restype = None
+        lib.orc_write_kv_cache_fp8.argtypes = [P, P, P, P, P, i32, f32, f32, i32, i32, i32, i32]
+        lib.orc_write_kv_cache_fp8.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -79,7 +84,64 @@ def _dtype_code(a: np.ndarray) -> int:
         return 0
     if a.dtype == np.uint16:
         return 1
-    raise TypeError(f"storage dtype must be float32 or uint16 (bf16 bits), got {a.dtype}")
+    if a.dtype == np.uint8:
+        return 2  # E4M3 codes
+    if a.dtype == np.float64:
+        return 3
+    raise TypeError("storage dtype must be float32, uint16 (bf16 bits), uint8 (E4M3 codes) "
+                    f"or float64, got {a.dtype}")
+
+
+def e4m3_value(codes: np.ndarray) -> np.ndarray:
+    """E4M3 codes (uint8) -> their exact values as float64 (OCP 8-bit
+    floating point E4M3, "fn" form: bias 7, subnormals at exponent 0, no
+    infinities, S.1111.111 is NaN; largest finite 448)."""
+    return widen(np.ascontiguousarray(codes, dtype=np.uint8))
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """The E4M3 code nearest to each value (ties to the even mantissa,
+    magnitudes >= 448 saturate to 448, NaN -> 0x7F)."""
+    xs = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(xs.shape, dtype=np.uint8)
+    _load().orc_e4m3_encode_array(_ptr(xs), xs.size, _ptr(out))
+    return out
+
+
+def dequantize(codes: np.ndarray, scale: float) -> np.ndarray:
+    """FP8 pages as the values they stand for: code value * scale, in
+    float64 (exact: a code has at most 4 significant bits, a float32 scale
+    24)."""
+    return e4m3_value(codes) * np.float64(np.float32(scale))
+
+
+def write_kv_cache_fp8(key_cache: np.ndarray, value_cache: np.ndarray, k_new: np.ndarray,
+                       v_new: np.ndarray, slot_mapping: np.ndarray, k_scale: float,
+                       v_scale: float) -> int:
+    """Cache write into FP8 pages, in place: each element of the bf16 rows
+    k_new / v_new [N, Hkv, D] (uint16 bits) is divided by its scale in IEEE
+    single precision and rounded to the nearest E4M3 code, then stored at
+    its slot as in write_kv_cache (teaching page, "Writing slots and reading
+    the block table must agree").  Returns flags."""
+    NB, bs, Hkv, D = key_cache.shape
+    assert key_cache.dtype == np.uint8 and value_cache.dtype == np.uint8
+    assert k_new.dtype == np.uint16 and v_new.dtype == np.uint16
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    kn = np.ascontiguousarray(k_new)
+    vn = np.ascontiguousarray(v_new)
+    return _load().orc_write_kv_cache_fp8(_ptr(key_cache), _ptr(value_cache), _ptr(kn), _ptr(vn),
+                                          _ptr(sm), sm.size, np.float32(k_scale),
+                                          np.float32(v_scale), NB, bs, Hkv, D)
+
+
+def decode_fp8(q, key_cache, value_cache, k_scale: float, v_scale: float, block_tables,
+               context_lens, scale: Optional[float] = None):
+    """decode() over FP8 pages: the pages stand for code * scale (per
+    tensor) and q is bf16 (uint16 bits); every value is widened exactly to
+    float64 first.  Returns (out [B, Hq, D] float64, flags [B])."""
+    assert key_cache.dtype == np.uint8 and q.dtype == np.uint16
+    return decode(widen(q), dequantize(key_cache, k_scale), dequantize(value_cache, v_scale),
+                  block_tables, context_lens, scale)
 
 
 def map_token(block_table, token_index: int, block_size: int, num_blocks: int

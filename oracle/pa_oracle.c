@@ -50,15 +50,65 @@
 
 #define ORC_DTYPE_F32 0
 #define ORC_DTYPE_BF16 1
+#define ORC_DTYPE_FP8_E4M3 2 /* cache codes; see orc_e4m3_value */
+#define ORC_DTYPE_F64 3      /* already-widened values (e.g. dequantised pages) */
 
 #define ORC_FLAG_BLOCK_ID 1
 #define ORC_FLAG_CONTEXT_LEN 2
 #define ORC_FLAG_SLOT 4
 
+/* FP8 KV pages (a reading: the pages name quantised KV only as a later
+ * addition).  Codes follow the OCP 8-bit floating point format E4M3 in its
+ * "fn" form: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+ * exponent 0 holds the subnormals m/8 * 2^-6; there are no infinities and
+ * S.1111.111 is NaN, so the largest finite magnitude is 1.75 * 2^8 = 448.
+ * A cache entry stands for code value * scale (one scale per tensor). */
+static double orc_e4m3_value(uint8_t c) {
+  const int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double v = (e == 0) ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10);
+  return sgn ? -v : v;
+}
+
+/* The E4M3 code nearest to x: ties go to the even mantissa, magnitudes at
+ * or above 448 saturate to 448, NaN stays NaN (0x7F), the sign of zero is
+ * kept.  Uses the default round-to-nearest-even mode of nearbyint. */
+uint8_t orc_e4m3_encode(double x) {
+  if (isnan(x)) return 0x7F;
+  const uint8_t sgn = signbit(x) ? 0x80 : 0;
+  const double a = fabs(x);
+  if (a >= 448.0) return sgn | 0x7E;
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal range, quantum 2^-9; n == 8 is the smallest normal (0x08) */
+    const double n = nearbyint(ldexp(a, 9));
+    return sgn | (uint8_t)n;
+  }
+  int k;
+  frexp(a, &k); /* a in [2^(k-1), 2^k) */
+  int E = k - 1; /* -6 .. 8 */
+  double n = nearbyint(ldexp(a, 3 - E)); /* a / 2^(E-3), in [8, 16] */
+  if (n == 16.0) {
+    E += 1;
+    n = 8.0;
+  }
+  if (E > 8) return sgn | 0x7E;
+  return sgn | (uint8_t)(((E + 7) << 3) | ((int)n - 8));
+}
+
+void orc_e4m3_encode_array(const double *x, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_encode(x[i]);
+}
+
 /* Read element idx of a stored array and widen it exactly to double. */
 static double orc_load(const void *base, int64_t idx, int dtype) {
   if (dtype == ORC_DTYPE_F32) {
     return (double)((const float *)base)[idx];
+  }
+  if (dtype == ORC_DTYPE_FP8_E4M3) {
+    return orc_e4m3_value(((const uint8_t *)base)[idx]);
+  }
+  if (dtype == ORC_DTYPE_F64) {
+    return ((const double *)base)[idx];
   }
   uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;
   float f;
@@ -328,6 +378,35 @@ void orc_merge(const double *part_max, const double *part_sum,
     }
     for (int32_t d = 0; d < head_dim; ++d) o[d] /= wsum;
   }
+}
+
+/* Cache write into FP8 pages: the new rows arrive as bf16 (widened
+ * exactly), each element is divided by its tensor's scale in IEEE single
+ * precision and rounded to the nearest E4M3 code (orc_e4m3_encode) -- the
+ * quantisation decision is taken in the precision the kernel takes it in.
+ * Slots as in orc_write_kv_cache. */
+int orc_write_kv_cache_fp8(uint8_t *key_cache, uint8_t *value_cache, const uint16_t *k_new,
+                           const uint16_t *v_new, const int64_t *slot_mapping,
+                           int32_t num_tokens, float k_scale, float v_scale,
+                           int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                           int32_t head_dim) {
+  const int64_t row = (int64_t)num_kv_heads * head_dim;
+  int flags = 0;
+  for (int32_t i = 0; i < num_tokens; ++i) {
+    const int64_t s = slot_mapping[i];
+    if (s < 0) continue;
+    if (s >= (int64_t)num_blocks * block_size) {
+      flags |= ORC_FLAG_SLOT;
+      continue;
+    }
+    for (int64_t e = 0; e < row; ++e) {
+      const volatile float kq = (float)orc_load(k_new, i * row + e, ORC_DTYPE_BF16) / k_scale;
+      const volatile float vq = (float)orc_load(v_new, i * row + e, ORC_DTYPE_BF16) / v_scale;
+      key_cache[s * row + e] = orc_e4m3_encode((double)kq);
+      value_cache[s * row + e] = orc_e4m3_encode((double)vq);
+    }
+  }
+  return flags;
 }
 
 /* Cache write by slot mapping: for each new token i with slot s >= 0 copy

@@ -369,3 +369,79 @@ def test_bad_metadata_is_flagged_and_zeroed():
                               np.array([-1, w.num_blocks * w.block_size]))
     assert f == oracle.FLAG_SLOT
     assert np.array_equal(kc, w.key_cache, equal_nan=True)
+
+
+# ---------------------------------------------------------------------------
+# FP8 KV pages (E4M3, OCP 8-bit floating point, "fn" form).  The oracle's
+# codec is pinned against torch's float8_e4m3fn (a library decoder), against
+# a brute-force nearest-code search, and against values of the format's
+# definition; the quantising write against a hand-worked example.
+# ---------------------------------------------------------------------------
+def test_e4m3_values_of_the_definition():
+    v = oracle.e4m3_value(np.array([0x00, 0x01, 0x07, 0x08, 0x38, 0x3F, 0x40, 0x7E, 0x80,
+                                    0xB8, 0xFE], dtype=np.uint8))
+    assert v.tolist() == [0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, 1.875, 2.0, 448.0,
+                          -0.0, -1.0, -448.0]
+    assert np.isnan(oracle.e4m3_value(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+    pos = oracle.e4m3_value(np.arange(0x7F, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0), "codes 0x00..0x7E increase"
+
+
+def test_e4m3_values_match_torch_float8():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_value(codes)
+    theirs = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(theirs))
+    ok = ~np.isnan(ours)
+    assert np.array_equal(ours[ok], theirs[ok])
+    assert np.array_equal(np.signbit(ours[ok]), np.signbit(theirs[ok]))
+
+
+def _nearest_code_brute(x: float) -> int:
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle.e4m3_value(codes)
+    finite = ~np.isnan(vals)
+    if abs(x) >= 448.0:
+        return 0x7E | (0x80 if np.signbit(x) else 0)
+    d = np.where(finite, np.abs(vals - x), np.inf)
+    best = np.flatnonzero(d == d.min())
+    # equal distance: the code whose mantissa (its last bit) is even; the
+    # two zeros are equally near only to 0 itself: keep x's sign
+    best = [int(c) for c in best if not (vals[c] == 0 and np.signbit(vals[c]) != np.signbit(x))]
+    even = [c for c in best if c % 2 == 0]
+    return (even or best)[0]
+
+
+def test_e4m3_encode_is_the_nearest_code():
+    rng = np.random.default_rng(7)
+    xs = np.concatenate([rng.normal(0, 4, 300), rng.normal(0, 0.01, 200),
+                         rng.uniform(-500, 500, 100), [0.0, -0.0, 447.9, 448.0, 449.0, 479.9]])
+    # every midpoint between neighbouring codes (ties)
+    pos = oracle.e4m3_value(np.arange(0x7F, dtype=np.uint8))
+    mids = (pos[1:] + pos[:-1]) / 2
+    xs = np.concatenate([xs, mids, -mids])
+    got = oracle.e4m3_encode(xs)
+    want = np.array([_nearest_code_brute(float(x)) for x in xs], dtype=np.uint8)
+    assert np.array_equal(got, want)
+    assert oracle.e4m3_encode(np.array([np.nan]))[0] == 0x7F
+
+
+def test_write_kv_cache_fp8_worked_example():
+    """Two tokens into a 2-block pool of 2-token pages, 1 KV head, head_dim 4:
+    bf16 1.0, -3.0, 0.25, 1000.0 divided by k_scale 0.5 are 2, -6, 0.5 and
+    2000 -> codes 0x40, 0xCC (-1.5 * 2^2: exponent field 9, mantissa 4),
+    0x30, 0x7E (saturated); V by v_scale 2.0."""
+    def bf16(xs):
+        return (np.array(xs, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    kc = np.zeros((2, 2, 1, 4), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    k_new = bf16([[1.0, -3.0, 0.25, 1000.0], [0.0, 0.0, 0.0, 0.0]]).reshape(2, 1, 4)
+    v_new = bf16([[1.0, 2.0, 3.0, 4.0], [0.5, 0.5, 0.5, 0.5]]).reshape(2, 1, 4)
+    f = oracle.write_kv_cache_fp8(kc, vc, k_new, v_new, np.array([3, -1]), 0.5, 2.0)
+    assert f == 0
+    assert kc[1, 1, 0].tolist() == [0x40, 0xCC, 0x30, 0x7E]
+    # 0.5, 1, 1.5, 2 -> 0x30, 0x38, 0x3C, 0x40
+    assert vc[1, 1, 0].tolist() == [0x30, 0x38, 0x3C, 0x40]
+    assert not kc[0].any() and not kc[1, 0].any()
+    assert oracle.write_kv_cache_fp8(kc, vc, k_new, v_new, np.array([4, 0]), 0.5, 2.0) == \
+        oracle.FLAG_SLOT
