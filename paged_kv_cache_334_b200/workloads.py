@@ -37,6 +37,12 @@ rounded to nearest-even by torch's cast; every array is host memory):
     followed by a private suffix of uniform [1, 1024] tokens in scattered
     blocks (20 % slack).
 
+``gqa_fp8``
+    gqa_bf16's shape and lengths with FP8 pages: caches of E4M3 codes
+    (uint8) standing for code * 0.25 (K) and code * 0.5 (V), the codes drawn
+    directly (sign, exponent field 3..9, mantissa uniform), NaN code 0x7F
+    in unused slots; q and the new rows in bf16.
+
 In every workload but ``tiny_fp32`` the last token of each sequence is the
 token of the current decode step: its K/V rows are returned in
 ``k_new``/``v_new`` with the slot reserved for it in ``slot_mapping``, and
@@ -54,8 +60,11 @@ import numpy as np
 
 DTYPE_F32 = "f32"
 DTYPE_BF16 = "bf16"
+DTYPE_FP8 = "fp8_e4m3"
+FP8_K_SCALE = 0.25  # the fp8 workloads' per-tensor scales
+FP8_V_SCALE = 0.5
 
-WORKLOADS = ("tiny_fp32", "gqa_bf16", "mixed_bf16", "long_bf16", "mqa_prefix_bf16")
+WORKLOADS = ("tiny_fp32", "gqa_bf16", "mixed_bf16", "long_bf16", "mqa_prefix_bf16", "gqa_fp8")
 
 _BF16_NAN = np.uint16(0x7FC0)
 
@@ -63,7 +72,10 @@ _BF16_NAN = np.uint16(0x7FC0)
 @dataclasses.dataclass
 class Workload:
     name: str
-    dtype: str  # "f32" (float32 arrays) or "bf16" (uint16 arrays of bf16 bits)
+    # "f32" (float32 arrays), "bf16" (uint16 arrays of bf16 bits) or
+    # "fp8_e4m3": caches of E4M3 codes (uint8) standing for code * k_scale /
+    # code * v_scale, with q and the new rows in bf16
+    dtype: str
     batch: int
     num_q_heads: int
     num_kv_heads: int
@@ -83,9 +95,17 @@ class Workload:
     seed: int = 0
     description: str = ""
     shared_prefix_blocks: int = 0  # leading table entries every sequence shares
+    k_scale: float = 1.0  # fp8_e4m3 caches: value = code * scale
+    v_scale: float = 1.0
 
     @property
     def elem_bytes(self) -> int:
+        """Bytes of one cache element."""
+        return 4 if self.dtype == DTYPE_F32 else 1 if self.dtype == DTYPE_FP8 else 2
+
+    @property
+    def act_bytes(self) -> int:
+        """Bytes of one element of q, out and the new rows."""
         return 4 if self.dtype == DTYPE_F32 else 2
 
     @property
@@ -122,13 +142,36 @@ def _pages(ctx: int, bs: int) -> int:
     return (ctx + bs - 1) // bs
 
 
+def _e4m3_codes(rng: np.random.Generator, shape, chunk: int = 1 << 26) -> np.ndarray:
+    """Random E4M3 codes (uint8): sign, exponent field 3..9 (magnitudes
+    2^-4 .. 1.875 * 2^2) and mantissa drawn uniformly; no value is computed."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint8)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        sign = rng.integers(0, 2, size=e - s, dtype=np.uint8) << 7
+        expo = rng.integers(3, 10, size=e - s, dtype=np.uint8) << 3
+        mant = rng.integers(0, 8, size=e - s, dtype=np.uint8)
+        out[s:e] = sign | expo | mant
+    return out.reshape(shape)
+
+
+_E4M3_NAN = np.uint8(0x7F)
+
+
 def _finish(name, dtype, rng, B, Hq, Hkv, D, bs, NB, MB, ctx, tables,
             new_tokens: bool, partition_tokens=None, seed=0, description=""):
     """Draw q and cache contents, poison unused slots, peel off new tokens."""
-    q = _normal_storage(rng, (B, Hq, D), dtype)
-    kc = _normal_storage(rng, (NB, bs, Hkv, D), dtype)
-    vc = _normal_storage(rng, (NB, bs, Hkv, D), dtype)
-    nan = _nan_value(dtype)
+    fp8 = dtype == DTYPE_FP8
+    q = _normal_storage(rng, (B, Hq, D), DTYPE_BF16 if fp8 else dtype)
+    if fp8:
+        kc = _e4m3_codes(rng, (NB, bs, Hkv, D))
+        vc = _e4m3_codes(rng, (NB, bs, Hkv, D))
+        nan = _E4M3_NAN
+    else:
+        kc = _normal_storage(rng, (NB, bs, Hkv, D), dtype)
+        vc = _normal_storage(rng, (NB, bs, Hkv, D), dtype)
+        nan = _nan_value(dtype)
     # Slots that hold a visible token of some sequence.
     live = np.zeros((NB, bs), dtype=bool)
     for b in range(B):
@@ -140,14 +183,20 @@ def _finish(name, dtype, rng, B, Hq, Hkv, D, bs, NB, MB, ctx, tables,
     k_new = v_new = slots = None
     if new_tokens:
         rows = [b for b in range(B) if ctx[b] > 0]
-        k_new = np.empty((len(rows), Hkv, D), dtype=kc.dtype)
-        v_new = np.empty_like(k_new)
+        if fp8:
+            # the new rows arrive in bf16; the write quantises them
+            k_new = _normal_storage(rng, (len(rows), Hkv, D), DTYPE_BF16)
+            v_new = _normal_storage(rng, (len(rows), Hkv, D), DTYPE_BF16)
+        else:
+            k_new = np.empty((len(rows), Hkv, D), dtype=kc.dtype)
+            v_new = np.empty_like(k_new)
         slots = np.empty(len(rows), dtype=np.int64)
         for i, b in enumerate(rows):
             t = int(ctx[b]) - 1
             pb, off = int(tables[b, t // bs]), t % bs  # where the allocator put it
-            k_new[i] = kc[pb, off]
-            v_new[i] = vc[pb, off]
+            if not fp8:
+                k_new[i] = kc[pb, off]
+                v_new[i] = vc[pb, off]
             kc[pb, off] = nan
             vc[pb, off] = nan
             slots[i] = pb * bs + off
@@ -188,8 +237,9 @@ def make_workload(name: str, seed: int = 0, batch: Optional[int] = None,
     long_bf16 (the same lengths and values, paged differently: a page-size
     sweep)."""
     if block_size is not None:
-        if name not in ("gqa_bf16", "mixed_bf16", "long_bf16"):
-            raise ValueError(f"block_size override is for gqa_bf16, mixed_bf16, long_bf16, not {name}")
+        if name not in ("gqa_bf16", "mixed_bf16", "long_bf16", "gqa_fp8"):
+            raise ValueError("block_size override is for gqa_bf16, mixed_bf16, long_bf16, "
+                             f"gqa_fp8, not {name}")
         if block_size < 1 or block_size & (block_size - 1):
             raise ValueError(f"block_size must be a power of two, not {block_size}")
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -247,16 +297,30 @@ def make_workload(name: str, seed: int = 0, batch: Optional[int] = None,
                     description=f"B{B} Hq64/Hkv1 D128 bs32, 2048 shared prefix + U[1,1024] suffix, bf16")
         w.shared_prefix_blocks = prefix // bs
         return w
+    if name == "gqa_fp8":
+        # gqa_bf16's shape and lengths with FP8 (E4M3) pages
+        B = batch or 32
+        Hq, Hkv, D, bs = 32, 8, 128, block_size or 16
+        ctx = rng.integers(128, 2048, size=B, endpoint=True).astype(np.int32)
+        MB = _pages(2048, bs)
+        tables, NB = _scattered_tables(rng, ctx, bs, MB)
+        w = _finish(name, DTYPE_FP8, rng, B, Hq, Hkv, D, bs, NB, MB, ctx, tables,
+                    new_tokens=True, seed=seed,
+                    description=f"B{B} Hq32/Hkv8 D128 bs{bs} ctx~U[128,2048] fp8_e4m3 pages")
+        w.k_scale, w.v_scale = FP8_K_SCALE, FP8_V_SCALE
+        return w
     raise ValueError(f"unknown workload {name!r}; known: {WORKLOADS}")
 
 
 def custom_workload(*, dtype: str, batch: int, num_q_heads: int, num_kv_heads: int,
                     head_dim: int, block_size: int, context_lens, seed: int = 0,
                     slack: float = 0.2, max_blocks: Optional[int] = None,
-                    new_tokens: bool = False, prefix_blocks: int = 0) -> Workload:
+                    new_tokens: bool = False, prefix_blocks: int = 0,
+                    k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE) -> Workload:
     """A workload with explicit context lengths (edge cases, sweeps).  With
     prefix_blocks > 0 every table starts with the same physical blocks (a
-    shared prompt prefix); every context must cover them."""
+    shared prompt prefix); every context must cover them.  k_scale / v_scale
+    are the per-tensor scales of fp8_e4m3 caches."""
     rng = np.random.Generator(np.random.PCG64(seed))
     ctx = np.asarray(context_lens, dtype=np.int32)
     need = max([_pages(int(c), block_size) for c in ctx] + [1])
@@ -271,6 +335,8 @@ def custom_workload(*, dtype: str, batch: int, num_q_heads: int, num_kv_heads: i
                 new_tokens=new_tokens, seed=seed,
                 description=f"custom ctx={list(map(int, ctx))[:8]}...")
     w.shared_prefix_blocks = prefix_blocks
+    if dtype == DTYPE_FP8:
+        w.k_scale, w.v_scale = k_scale, v_scale
     return w
 
 
@@ -290,10 +356,12 @@ def roofline_bytes(w: Workload, include_write: bool = True) -> int:
                 continue
             seen.add(pb)
             kv += 2 * n_valid * row
-    qo = 2 * w.batch * w.num_q_heads * w.head_dim * w.elem_bytes
+    qo = 2 * w.batch * w.num_q_heads * w.head_dim * w.act_bytes
     meta = w.block_tables.size * 4 + w.context_lens.size * 4
     extra = 0
     if include_write and w.slot_mapping is not None:
-        # new rows read once and stored once, for K and for V
-        extra = 2 * (w.k_new.nbytes + w.v_new.nbytes) + w.slot_mapping.nbytes
+        # new rows read once and stored once (as cache elements), K and V
+        n_new = w.slot_mapping.size
+        extra = (w.k_new.nbytes + w.v_new.nbytes + 2 * n_new * row +
+                 w.slot_mapping.nbytes)
     return int(kv + qo + meta + extra)
