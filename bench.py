@@ -309,10 +309,18 @@ def time_oracle(w, target_seconds: float, max_reps: int = 1000):
 def _oracle_step(w) -> float:
     import oracle
     kc, vc = w.key_cache, w.value_cache
+    scale = 1.0 / math.sqrt(w.head_dim)
     t0 = time.perf_counter()
+    if w.dtype == wl.DTYPE_FP8:
+        if w.slot_mapping is not None:
+            oracle.write_kv_cache_fp8(kc, vc, w.k_new, w.v_new, w.slot_mapping, w.k_scale,
+                                      w.v_scale)
+        oracle.decode_fp8(w.q, kc, vc, w.k_scale, w.v_scale, w.block_tables, w.context_lens,
+                          scale)
+        return time.perf_counter() - t0
     if w.slot_mapping is not None:
         oracle.write_kv_cache(kc, vc, w.k_new, w.v_new, w.slot_mapping)
-    oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, 1.0 / math.sqrt(w.head_dim))
+    oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, scale)
     return time.perf_counter() - t0
 
 
@@ -391,7 +399,11 @@ def run_ours(args):
 
     def dev_t(a):
         t = torch.from_numpy(np.ascontiguousarray(a))
-        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).to(dev)
+        if a.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+        elif a.dtype == np.uint8:  # E4M3 codes
+            t = t.view(torch.float8_e4m3fn)
+        return t.to(dev)
 
     q, kc, vc = dev_t(w.q), dev_t(w.key_cache), dev_t(w.value_cache)
     bt = torch.from_numpy(w.block_tables).to(dev)
@@ -402,7 +414,8 @@ def run_ours(args):
     sm = torch.from_numpy(w.slot_mapping).to(dev) if has_new else None
     out = torch.empty_like(q)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws = pa.decode_workspace(kc, w.batch, w.num_q_heads, w.max_blocks)
+    sc = dict(k_scale=w.k_scale, v_scale=w.v_scale)  # FP8 pages: code * scale
+    ws = pa.decode_workspace(kc, w.batch, w.num_q_heads, w.max_blocks, **sc)
     scale = 1.0 / math.sqrt(w.head_dim)
     stream = torch.cuda.current_stream(dev)
 
@@ -435,18 +448,18 @@ def run_ours(args):
 
     def write():
         if has_new and not fused:
-            pa.pa_write_kv_cache(kc, vc, kn, vn, sm, err_word=err, stream=stream)
+            pa.pa_write_kv_cache(kc, vc, kn, vn, sm, err_word=err, stream=stream, **sc)
 
     def decode():
         if prefix:
             pa.pa_decode_shared_prefix(out, q, kc, vc, bt, cl, w.shared_prefix_blocks, scale=scale,
-                                       err_word=err, stream=stream)
+                                       err_word=err, stream=stream, **sc)
         elif fused:
             pa.pa_forward_decode(out, q, kc, vc, kn, vn, sm, bt, cl, scale=scale, workspace=ws,
-                                 err_word=err, stream=stream)
+                                 err_word=err, stream=stream, **sc)
         else:
             pa.pa_decode(out, q, kc, vc, bt, cl, scale=scale, workspace=ws, err_word=err,
-                         stream=stream)
+                         stream=stream, **sc)
 
     for _ in range(max(args.warmup, 3)):
         flush_l2()

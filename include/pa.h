@@ -63,7 +63,23 @@ typedef enum pa_status {
   PA_ERR_CUDA = 3
 } pa_status;
 
-typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1, PA_DTYPE_FP8_E4M3 = 2 } pa_dtype;
+
+/*
+ * FP8 pages (PA_DTYPE_FP8_E4M3).  The pages name quantised KV only as a
+ * later addition; the reading taken: the caches hold codes of the OCP 8-bit
+ * floating point format E4M3 in its "fn" form (1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits, subnormals at exponent 0, no infinities,
+ * S.1111.111 is NaN, largest finite magnitude 448), and a key_cache entry
+ * stands for code * k_scale, a value_cache entry for code * v_scale (one
+ * scale per tensor, pa_cache_desc).  q, out, k_new and v_new are bf16.
+ * pa_write_kv_cache stores the code nearest to x / scale (the division in
+ * IEEE single precision, ties to the even mantissa, magnitudes at or above
+ * 448 saturating to 448).  Served by pa_write_kv_cache, pa_decode,
+ * pa_forward_decode and pa_decode_noalloc for head_dim 128, block_size >=
+ * 16, at most 8 KV heads, and at most 8 or exactly 16 query heads per KV
+ * head; other calls and shapes return PA_ERR_UNSUPPORTED.
+ */
 
 /* Bits OR'd into *err_word by kernels that meet bad device data. */
 #define PA_DEVERR_BLOCK_ID 1
@@ -85,9 +101,15 @@ typedef struct pa_cache_desc {
   int32_t num_kv_heads;
   int32_t head_dim;
   int32_t dtype; /* pa_dtype */
+  /* PA_DTYPE_FP8_E4M3 only (ignored for the other dtypes): the values the
+   * codes of key_cache / value_cache stand for are code * k_scale and
+   * code * v_scale; both finite and > 0. */
+  float k_scale;
+  float v_scale;
 } pa_cache_desc;
 
-/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+/* Version of this ABI (major * 10000 + minor * 100 + patch); 200 added the
+ * scales of pa_cache_desc and PA_DTYPE_FP8_E4M3. */
 int32_t pa_version(void);
 
 /* Static text for a status code. */

@@ -34,12 +34,22 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool is_pow2(int32_t x) { return x > 0 && (x & (x - 1)) == 0; }
 
-int32_t elem_bytes(int32_t dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
+// Bytes of one cache element, and of one element of q / out / the new rows.
+int32_t elem_bytes(int32_t dtype) {
+  return dtype == PA_DTYPE_F32 ? 4 : dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2;
+}
+int32_t act_bytes(int32_t dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
 
 pa_status check_cache(const pa_cache_desc *c) {
   if (c == nullptr) return fail(PA_ERR_INVALID_ARG, "cache descriptor is NULL%s");
-  if (c->dtype != PA_DTYPE_F32 && c->dtype != PA_DTYPE_BF16)
-    return fail(PA_ERR_INVALID_ARG, "dtype %s%lld is neither F32 nor BF16", "", c->dtype);
+  if (c->dtype != PA_DTYPE_F32 && c->dtype != PA_DTYPE_BF16 && c->dtype != PA_DTYPE_FP8_E4M3)
+    return fail(PA_ERR_INVALID_ARG, "dtype %s%lld is not F32, BF16 or FP8_E4M3", "", c->dtype);
+  if (c->dtype == PA_DTYPE_FP8_E4M3) {
+    if (!(c->k_scale > 0.f && c->k_scale <= 3.4e38f && c->v_scale > 0.f && c->v_scale <= 3.4e38f))
+      return fail(PA_ERR_INVALID_ARG, "FP8 pages need finite scales > 0%s");
+    if (c->head_dim != 128)
+      return fail(PA_ERR_UNSUPPORTED, "FP8 pages need head_dim 128%s (got %lld)", "", c->head_dim);
+  }
   if (c->num_blocks <= 0)
     return fail(PA_ERR_INVALID_ARG, "num_blocks must be > 0%s (got %lld)", "", c->num_blocks);
   if (c->num_kv_heads <= 0)
@@ -102,6 +112,8 @@ struct StreamPlan {
   int32_t vbs, log2_vbs, log2_vpp, row_bytes, row_pitch, vpage_stride, q_bytes, pps, stages,
       stage_bytes, box_bytes, n_dhalf;
   int32_t heads_per_warp, warps_per_kv;
+  bool fp8;               // E4M3 pages, converted to bf16 by the consumers
+  int32_t scratch_bytes;  // fp8: the bf16 page the consumers convert into
   size_t smem;
 };
 
@@ -117,7 +129,10 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   s.ok = false;
   const int32_t hkv = c->num_kv_heads;
   const int32_t group = num_q_heads / hkv;
-  const bool bf16 = c->dtype == PA_DTYPE_BF16;
+  // fp8 pages take the bf16 tensor-core consumers after a conversion
+  const bool fp8 = c->dtype == PA_DTYPE_FP8_E4M3;
+  const bool bf16 = c->dtype == PA_DTYPE_BF16 || fp8;
+  s.fp8 = fp8;
   if (bf16) {
     // tensor-core consumers: one warp per (KV head, 16 query heads) when the
     // group is a multiple of 16, else per (KV head, up to 8 query heads)
@@ -144,7 +159,13 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   const int32_t elt = elem_bytes(c->dtype);
   s.row_bytes = hkv * c->head_dim * elt;
   if (s.row_bytes + 16 > st::kVPageBytes) return s;
-  const int32_t rows = st::kVPageBytes / s.row_bytes;  // power of two
+  int32_t rows = st::kVPageBytes / s.row_bytes;  // power of two
+  if (fp8) {
+    // 16-token virtual pages (one MMA tile), each warp alone on its KV
+    // head's rows of the converted page (a warp never shares them)
+    if (c->block_size < 16 || hkv > 8 || s.warps_per_kv != 1) return s;
+    rows = 16;
+  }
   s.vbs = c->block_size < rows ? c->block_size : rows;
   s.log2_vbs = ilog2(s.vbs);
   s.log2_vpp = ilog2(c->block_size / s.vbs);
@@ -163,11 +184,15 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
     s.row_pitch = s.row_bytes;
     s.vpage_stride = s.vbs * s.row_bytes;
   }
-  s.q_bytes = num_q_heads * c->head_dim * elt;
+  s.q_bytes = num_q_heads * c->head_dim * act_bytes(c->dtype);
   s.pps = st::kVPageBytes / s.vpage_stride;
   if (s.pps > st::kMaxPPS) s.pps = st::kMaxPPS;
   if (s.pps < 1) s.pps = 1;
-  const int32_t avail = st::kSmemLimit - st::kHdrBytes - 1024;  // 1 KB alignment slack
+  if (fp8 && !s.tile) return s;
+  // fp8: a bf16 page (K and V, every 64-wide half of D) to convert into
+  s.scratch_bytes = fp8 ? 2 * s.n_dhalf * s.box_bytes : 0;
+  const int32_t avail =
+      st::kSmemLimit - st::kHdrBytes - 1024 - s.scratch_bytes;  // 1 KB alignment slack
   for (;;) {
     s.stage_bytes = (int32_t)(((size_t)2 * s.pps * s.vpage_stride + (size_t)s.pps * s.q_bytes +
                                1023) / 1024 * 1024);
@@ -177,7 +202,7 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
     --s.pps;
   }
   if (s.stages < 2) return s;
-  s.smem = (size_t)st::kHdrBytes + 1024 + (size_t)s.stages * s.stage_bytes;
+  s.smem = (size_t)st::kHdrBytes + 1024 + (size_t)s.stages * s.stage_bytes + s.scratch_bytes;
   s.ok = true;
   return s;
 }
@@ -198,22 +223,25 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 3-D view (head_dim, token row of the pool, KV head) of a bf16 cache with
-// boxes of 64 x vbs x Hkv and 128-byte swizzle.
+// 3-D view (head_dim, token row of the pool, KV head) of a cache with boxes
+// of 128 bytes x vbs x Hkv and 128-byte swizzle: 64 bf16 elements (one box
+// per 64-wide half of head_dim) or 128 E4M3 codes (one box per row).
 bool encode_cache_map(CUtensorMap *map, const void *base, const pa_cache_desc *c, int32_t vbs) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (fn == nullptr) return false;
+  const bool fp8 = c->dtype == PA_DTYPE_FP8_E4M3;
+  const cuuint64_t elt = fp8 ? 1 : 2;
   const cuuint64_t dims[3] = {(cuuint64_t)c->head_dim,
                               (cuuint64_t)c->num_blocks * (cuuint64_t)c->block_size,
                               (cuuint64_t)c->num_kv_heads};
-  const cuuint64_t strides[2] = {(cuuint64_t)c->num_kv_heads * c->head_dim * 2,
-                                 (cuuint64_t)c->head_dim * 2};
-  const cuuint32_t box[3] = {64, (cuuint32_t)vbs, (cuuint32_t)c->num_kv_heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)c->num_kv_heads * c->head_dim * elt,
+                                 (cuuint64_t)c->head_dim * elt};
+  const cuuint32_t box[3] = {(cuuint32_t)(128 / elt), (cuuint32_t)vbs, (cuuint32_t)c->num_kv_heads};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        3, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -431,7 +459,8 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
                                                 cache->num_blocks, row_bytes, key_cache,
                                                 value_cache, k_new, v_new, slot_mapping, batch,
                                                 err_word, st, block_tables, context_lens,
-                                                max_blocks_per_seq);
+                                                max_blocks_per_seq, cache->k_scale,
+                                                cache->v_scale);
       if (e != cudaSuccess) return fail(PA_ERR_CUDA, "write_kv launch: %s", cudaGetErrorString(e));
     }
     pa::SuffixParams sp;
@@ -447,14 +476,21 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
   }
   if (prefix_blocks > 0 && !w.stream)
     return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs the persistent kernel's shapes%s");
+  const bool fp8 = cache->dtype == PA_DTYPE_FP8_E4M3;
+  if (fp8 && (!w.stream || prefix_blocks > 0))
+    return fail(PA_ERR_UNSUPPORTED,
+                "FP8 pages: head_dim 128, block_size >= 16, at most 8 KV heads and at most 8 or "
+                "exactly 16 query heads per KV head%s");
   if (w.stream) {
     StreamPlan sp = plan_stream(cache, num_q_heads);
     const int sms = device_sm_count();
     if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
     pa::stream::Params p{};
     if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, sp.vbs) &&
-                     encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs)))
+                     encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs))) {
+      if (fp8) return fail(PA_ERR_CUDA, "cannot describe the FP8 caches for the tensor copies%s");
       sp = plan_stream(cache, num_q_heads, /*allow_tile=*/false);
+    }
     p.q = q;
     p.out = out;
     p.key_cache = key_cache;
@@ -491,6 +527,16 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
     p.hdr_bytes = pa::stream::kHdrBytes;
     p.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.fp8 = fp8 ? 1 : 0;
+    p.out_scale = 1.f;
+    p.k_scale = cache->k_scale;
+    p.v_scale = cache->v_scale;
+    if (fp8) {
+      // the consumers see the codes' values (exact in bf16): K's scale goes
+      // into the score scale, V's into the output
+      p.scale_log2 *= cache->k_scale;
+      p.out_scale = cache->v_scale;
+    }
     const int group = num_q_heads / cache->num_kv_heads;
     p.group = group;
     p.heads_per_warp = sp.heads_per_warp;
@@ -498,14 +544,14 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
     p.tile = sp.tile ? 1 : 0;
     p.box_bytes = sp.box_bytes;
     p.n_dhalf = sp.n_dhalf;
-    cudaError_t e = (cache->dtype == PA_DTYPE_BF16)
+    const bool mma = cache->dtype != PA_DTYPE_F32;
+    cudaError_t e = mma
                         ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
                                                   sp.smem, static_cast<cudaStream_t>(stream))
                         : pa::stream::launch_f32(p, cache->head_dim, group, cache->num_kv_heads,
                                                  sp.smem, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    e = (cache->dtype == PA_DTYPE_BF16)
-            ? pa::stream::launch_merge_bf16(p, cache->head_dim, static_cast<cudaStream_t>(stream))
+    e = mma ? pa::stream::launch_merge_bf16(p, cache->head_dim, static_cast<cudaStream_t>(stream))
             : pa::stream::launch_merge_f32(p, cache->head_dim, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
     return PA_OK;
@@ -518,7 +564,8 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
                                         row_bytes, key_cache, value_cache, k_new, v_new,
                                         slot_mapping, batch, err_word,
                                         static_cast<cudaStream_t>(stream), block_tables,
-                                        context_lens, max_blocks_per_seq);
+                                        context_lens, max_blocks_per_seq, cache->k_scale,
+                                        cache->v_scale);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "write_kv launch: %s", cudaGetErrorString(e));
   }
   pa::DecodeArgs a{};
@@ -578,7 +625,7 @@ pa_status decode_streamed(const pa_cache_desc *cache, void *out, const void *q,
 
 extern "C" {
 
-int32_t pa_version(void) { return 100; }
+int32_t pa_version(void) { return 200; }
 
 const char *pa_status_string(int32_t status) {
   switch (status) {
@@ -613,7 +660,8 @@ pa_status pa_write_kv_cache(const pa_cache_desc *cache, void *key_cache,
                                       cache->num_blocks, row_bytes, key_cache,
                                       value_cache, k_new, v_new, slot_mapping,
                                       num_tokens, err_word,
-                                      static_cast<cudaStream_t>(stream));
+                                      static_cast<cudaStream_t>(stream), nullptr, nullptr, 0,
+                                      cache->k_scale, cache->v_scale);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "write_kv launch: %s", cudaGetErrorString(e));
   return PA_OK;
 }

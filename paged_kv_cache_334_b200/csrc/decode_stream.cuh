@@ -335,7 +335,8 @@ struct MmaConsumer {
     const bool odd = g & 1;
     const int q = g & 3;
     const int hh = 2 * t + (odd ? 1 : 0);  // head of this lane's values
-    const float inv = seg_bad ? 0.f : 1.f / (odd ? L1 : L0);
+    // out_scale: 1, or V's scale for FP8 pages (the products saw the codes)
+    const float inv = seg_bad ? 0.f : p.out_scale / (odd ? L1 : L0);
     const int dcol = (g - q) + (q < 2 ? 0 : 8);
     float4 v[KS];
 #pragma unroll
@@ -577,7 +578,7 @@ struct HeadRowConsumer {
       L0 += __shfl_xor_sync(0xffffffffu, L0, mask);
       L1 += __shfl_xor_sync(0xffffffffu, L1, mask);
     }
-    const float i0 = seg_bad ? 0.f : 1.f / L0, i1 = seg_bad ? 0.f : 1.f / L1;
+    const float i0 = seg_bad ? 0.f : p.out_scale / L0, i1 = seg_bad ? 0.f : p.out_scale / L1;
     if (d.n_contrib == 1 && p.seq_o != nullptr) {
       // suffix mode: the sequence's result as a partial for the prefix pass
       const int64_t row = (int64_t)d.seq * p.num_q_heads + hq0 + r;
@@ -841,9 +842,10 @@ struct PageWalker {
   // the new token's rows towards L2 now; they are copied at that page.
   __device__ __forceinline__ void prefetch_new_rows(const Params &p, int64_t end, int lane) {
     if (p.slot_mapping != nullptr && lane == 0 && slot_s >= 0 && P_s + pages_s <= end) {
-      const int64_t off = (int64_t)s * p.row_bytes;
-      prefetch_l2(static_cast<const unsigned char *>(p.k_new) + off, (uint32_t)p.row_bytes);
-      prefetch_l2(static_cast<const unsigned char *>(p.v_new) + off, (uint32_t)p.row_bytes);
+      const int64_t in_row = (p.fp8 ? 2 : 1) * (int64_t)p.row_bytes;  // fp8: bf16 rows
+      const int64_t off = (int64_t)s * in_row;
+      prefetch_l2(static_cast<const unsigned char *>(p.k_new) + off, (uint32_t)in_row);
+      prefetch_l2(static_cast<const unsigned char *>(p.v_new) + off, (uint32_t)in_row);
     }
   }
   __device__ __forceinline__ void init(const Params &p, const Shared *cache, int32_t s0,
@@ -984,6 +986,55 @@ __device__ __forceinline__ void write_new_rows(const Params &p, int32_t s, int64
   fence_proxy_async_global();
 }
 
+// FP8 pages: the new token's bf16 rows (2 * row_bytes bytes each) divided
+// by the tensors' scales and quantised to E4M3 codes in its slot (row_bytes
+// codes), 16 elements per lane step; then the same fence.
+__device__ __forceinline__ void write_new_rows_fp8(const Params &p, int32_t s, int64_t slot,
+                                                   int lane) {
+  const int groups = p.row_bytes >> 4;
+  const uint4 *ks = reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.k_new) +
+                                                    (int64_t)s * 2 * p.row_bytes);
+  const uint4 *vs = reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(p.v_new) +
+                                                    (int64_t)s * 2 * p.row_bytes);
+  uint4 *kd = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.key_cache) +
+                                        slot * p.row_bytes);
+  uint4 *vd = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.value_cache) +
+                                        slot * p.row_bytes);
+  for (int x = lane; x < groups; x += 32) {
+    const uint4 k0 = __ldg(ks + 2 * x), k1 = __ldg(ks + 2 * x + 1);
+    const uint4 v0 = __ldg(vs + 2 * x), v1 = __ldg(vs + 2 * x + 1);
+    kd[x] = bf16x16_to_e4m3(k0, k1, p.k_scale);
+    vd[x] = bf16x16_to_e4m3(v0, v1, p.v_scale);
+  }
+  fence_proxy_async_global();
+}
+
+// FP8 pages: this warp's KV-head rows (h * 16 .. + 15) of one staged page,
+// stored as one box of 128 codes per row with the 128-byte swizzle (16-byte
+// chunk c of row r at chunk c ^ (r % 8)), converted exactly into the bf16
+// tile layout the tensor-core consumers read: 64-wide halves of head_dim in
+// boxes box_bytes apart, 8 elements per 16-byte chunk, the same swizzle.
+__device__ __forceinline__ void fp8_rows_to_bf16(const unsigned char *src, unsigned char *dst,
+                                                 int h, const Params &p, int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = lane + 32 * i;       // 16 rows x 8 chunks
+    const int r = h * 16 + (k & 15);   // row in the page's box
+    const int c = k >> 4;              // chunk of 16 codes: elements 16c .. 16c + 15
+    const uint4 x = *reinterpret_cast<const uint4 *>(src + r * 128 + ((c ^ (r & 7)) << 4));
+    uint32_t y[8];
+    e4m3x4_to_bf16x4(x.x, y[0], y[1]);
+    e4m3x4_to_bf16x4(x.y, y[2], y[3]);
+    e4m3x4_to_bf16x4(x.z, y[4], y[5]);
+    e4m3x4_to_bf16x4(x.w, y[6], y[7]);
+    unsigned char *row = dst + (c >> 2) * p.box_bytes + r * 128;
+    const int j0 = 2 * (c & 3);  // first of the two bf16 chunks in its half
+    *reinterpret_cast<uint4 *>(row + ((j0 ^ (r & 7)) << 4)) = make_uint4(y[0], y[1], y[2], y[3]);
+    *reinterpret_cast<uint4 *>(row + (((j0 + 1) ^ (r & 7)) << 4)) =
+        make_uint4(y[4], y[5], y[6], y[7]);
+  }
+}
+
 // ===========================================================================
 // The kernel.  T = element type; D = head_dim; G = query heads per KV head
 // for the fp32 consumer; for bf16, G = 16 selects the head-row consumer (16
@@ -1012,6 +1063,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   // stages start 1024-byte aligned (the 128-byte swizzle repeats every 1 KB)
   unsigned char *stages =
       smem_raw + (((smem_u32(smem_raw) + p.hdr_bytes + 1023u) & ~1023u) - smem_u32(smem_raw));
+  // FP8 pages: the bf16 page the consumers convert into (K, then V)
+  unsigned char *scratch = stages + (size_t)p.stages * p.stage_bytes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
@@ -1121,6 +1174,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     const int n_stages = (int)((end - start + p.pps - 1) / p.pps);
     if (warp == 0) {
       // ===================== producer =====================
+      const int nbox = p.fp8 ? 1 : p.n_dhalf;  // tensor copies per page and tensor
       PageWalker wk;
       wk.init(p, cached ? &sh : nullptr, sh.s_begin, sh.vlb_begin, sh.P_begin, start, end,
               lane);
@@ -1152,7 +1206,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             const int32_t pos = wk.ctx_s - 1;
             const int64_t want = (int64_t)pb * p.block_size + (pos & (p.block_size - 1));
             if (!bad_block && wk.slot_s == want) {
-              write_new_rows(p, wk.s, want, lane);
+              if (p.fp8)
+                write_new_rows_fp8(p, wk.s, want, lane);
+              else
+                write_new_rows(p, wk.s, want, lane);
               wrote = true;
             } else {
               bad = true;
@@ -1186,7 +1243,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             descs[slot * kMaxPPS + k] = d;
           }
           if (!bad)
-            bytes += p.tile ? 2u * (uint32_t)p.n_dhalf * (uint32_t)p.box_bytes
+            bytes += p.tile ? 2u * (uint32_t)nbox * (uint32_t)p.box_bytes
                             : 2u * (uint32_t)ntok * (uint32_t)p.row_bytes;
           if (first) bytes += (uint32_t)p.q_bytes;
           wk.advance(p, end, lane);
@@ -1204,9 +1261,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           const PageDesc d = descs[slot * kMaxPPS + k];
           if (!(d.flags & kBad) && p.tile) {
             // one box per (tensor, 64-wide d half), one lane each
-            if (lane < 2 * p.n_dhalf) {
-              const int dh = lane % p.n_dhalf;
-              const bool isv = lane >= p.n_dhalf;
+            if (lane < 2 * nbox) {
+              const int dh = lane % nbox;
+              const bool isv = lane >= nbox;
               tma_load_3d((isv ? vst : kst) + (size_t)k * p.vpage_stride + (size_t)dh * p.box_bytes,
                           isv ? &p.tmap_v : &p.tmap_k, dh * 64, d.pb * p.block_size + d.toff, 0,
                           &sh.full[slot]);
@@ -1293,6 +1350,15 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             const unsigned char *kp = kst + (size_t)k * p.vpage_stride;
             const unsigned char *vp = vst + (size_t)k * p.vpage_stride;
             if constexpr (kMma) {
+              if (p.fp8) {
+                // one warp per KV head: its rows of the converted page are its own
+                unsigned char *sk = scratch, *sv = scratch + (size_t)p.n_dhalf * p.box_bytes;
+                fp8_rows_to_bf16(kp, sk, h, p, lane);
+                fp8_rows_to_bf16(vp, sv, h, p, lane);
+                __syncwarp();
+                kp = sk;
+                vp = sv;
+              }
               cs.page(kp, vp, d.ntok, p, h, col_bytes, lane);
             } else {
               cs.page(kp, vp, d.ntok, p.row_pitch, col_bytes, sc_buf, lane);

@@ -85,6 +85,12 @@ struct Params {
   int32_t tile;                     // 1: tensor copies of swizzled boxes, else row copies
   int32_t box_bytes;                // bytes of one box (64 x vbs x Hkv bf16)
   int32_t n_dhalf;                  // boxes per page per tensor (head_dim / 64)
+  // FP8 pages: one box of 128 codes x vbs x Hkv per page and tensor, which
+  // the consumers convert into a bf16 page (the tile layout) after the
+  // stages; scale_log2 then includes k_scale and out_scale is v_scale
+  int32_t fp8;
+  float out_scale;
+  float k_scale, v_scale;  // FP8 pages: the fused write's quantisation scales
   float scale_log2;
 };
 
@@ -164,6 +170,8 @@ int decode_head_tile(int group);
 // With block_tables / context_lens set (num_tokens = batch, token b = the
 // newest token of sequence b), a token is written only when its slot is the
 // one the table gives position context_lens[b] - 1; others are flagged.
+// FP8 pages (dtype PA_DTYPE_FP8_E4M3): row_bytes is a cache row of codes,
+// the new rows are bf16 and are quantised with k_scale / v_scale.
 cudaError_t launch_write_kv(int32_t dtype, int32_t block_size,
                             int32_t num_blocks, int64_t row_bytes,
                             void *key_cache, void *value_cache,
@@ -171,7 +179,8 @@ cudaError_t launch_write_kv(int32_t dtype, int32_t block_size,
                             const int64_t *slot_mapping, int32_t num_tokens,
                             int32_t *err_word, cudaStream_t stream,
                             const int32_t *block_tables = nullptr,
-                            const int32_t *context_lens = nullptr, int32_t max_blocks = 0);
+                            const int32_t *context_lens = nullptr, int32_t max_blocks = 0,
+                            float k_scale = 1.f, float v_scale = 1.f);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 

@@ -32,6 +32,7 @@ PA_ERR_UNSUPPORTED = 2
 PA_ERR_CUDA = 3
 PA_DTYPE_F32 = 0
 PA_DTYPE_BF16 = 1
+PA_DTYPE_FP8_E4M3 = 2  # E4M3 codes; q, out and new rows bf16
 PA_DEVERR_BLOCK_ID = 1
 PA_DEVERR_CONTEXT_LEN = 2
 PA_DEVERR_SLOT = 4
@@ -60,7 +61,8 @@ class PaError(RuntimeError):
 class CacheDesc(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("k_scale", ctypes.c_float),
+                ("v_scale", ctypes.c_float)]
 
 
 _lib = None
@@ -119,7 +121,10 @@ def _dtype_code(dtype: torch.dtype) -> int:
         return PA_DTYPE_F32
     if dtype == torch.bfloat16:
         return PA_DTYPE_BF16
-    raise TypeError(f"unsupported dtype {dtype}: libpa takes float32 or bfloat16")
+    if dtype == torch.float8_e4m3fn:
+        return PA_DTYPE_FP8_E4M3
+    raise TypeError(f"unsupported dtype {dtype}: libpa takes float32, bfloat16 or "
+                    "float8_e4m3fn (caches)")
 
 
 def _dev(t: Optional[torch.Tensor], name: str, dtype: Optional[torch.dtype] = None):
@@ -135,11 +140,17 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype: Optional[torch.dtype] = No
     return ctypes.c_void_p(t.data_ptr()) if t.numel() else None
 
 
-def cache_desc(key_cache: torch.Tensor) -> CacheDesc:
+def _act(key_cache: torch.Tensor) -> torch.dtype:
+    """dtype of q, out and the new rows for this cache (bf16 for FP8 pages)."""
+    return torch.bfloat16 if key_cache.dtype == torch.float8_e4m3fn else key_cache.dtype
+
+
+def cache_desc(key_cache: torch.Tensor, k_scale: float = 1.0, v_scale: float = 1.0) -> CacheDesc:
+    """The pool's shape; k_scale / v_scale: FP8 pages stand for code * scale."""
     if key_cache.dim() != 4:
         raise ValueError("key_cache must be [num_blocks, block_size, num_kv_heads, head_dim]")
     nb, bs, hkv, d = key_cache.shape
-    return CacheDesc(nb, bs, hkv, d, _dtype_code(key_cache.dtype))
+    return CacheDesc(nb, bs, hkv, d, _dtype_code(key_cache.dtype), float(k_scale), float(v_scale))
 
 
 def _stream(stream: Optional[torch.cuda.Stream]):
@@ -152,22 +163,24 @@ def pa_version() -> int:
 
 
 def pa_write_kv_cache(key_cache, value_cache, k_new, v_new, slot_mapping,
-                      err_word: Optional[torch.Tensor] = None, stream=None) -> None:
+                      err_word: Optional[torch.Tensor] = None, stream=None,
+                      k_scale: float = 1.0, v_scale: float = 1.0) -> None:
     """Store each new token's K/V row at its slot (see include/pa.h)."""
     lib = load()
-    desc = cache_desc(key_cache)
+    desc = cache_desc(key_cache, k_scale, v_scale)
     if value_cache.shape != key_cache.shape or value_cache.dtype != key_cache.dtype:
         raise ValueError("value_cache must match key_cache")
     _check(lib.pa_write_kv_cache(
         ctypes.byref(desc), _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache"),
-        _dev(k_new, "k_new", key_cache.dtype), _dev(v_new, "v_new", key_cache.dtype),
+        _dev(k_new, "k_new", _act(key_cache)), _dev(v_new, "v_new", _act(key_cache)),
         _dev(slot_mapping, "slot_mapping", torch.int64), int(slot_mapping.numel()),
         _dev(err_word, "err_word", torch.int32), _stream(stream)))
 
 
 def pa_decode_workspace_bytes(key_cache, batch: int, num_q_heads: int,
-                              max_blocks_per_seq: int) -> int:
-    desc = cache_desc(key_cache)
+                              max_blocks_per_seq: int,
+                              k_scale: float = 1.0, v_scale: float = 1.0) -> int:
+    desc = cache_desc(key_cache, k_scale, v_scale)
     return int(load().pa_decode_workspace_bytes(ctypes.byref(desc), batch, num_q_heads,
                                                 max_blocks_per_seq))
 
@@ -175,12 +188,13 @@ def pa_decode_workspace_bytes(key_cache, batch: int, num_q_heads: int,
 _workspaces = {}
 
 
-def decode_workspace(key_cache, batch: int, num_q_heads: int, max_blocks_per_seq: int
-                     ) -> torch.Tensor:
+def decode_workspace(key_cache, batch: int, num_q_heads: int, max_blocks_per_seq: int,
+                     k_scale: float = 1.0, v_scale: float = 1.0) -> torch.Tensor:
     """A zero-filled workspace for pa_decode, cached per device and size
     (pa_decode leaves it zero-filled, so it can be reused by stream-ordered
     calls)."""
-    n = pa_decode_workspace_bytes(key_cache, batch, num_q_heads, max_blocks_per_seq)
+    n = pa_decode_workspace_bytes(key_cache, batch, num_q_heads, max_blocks_per_seq,
+                                  k_scale=k_scale, v_scale=v_scale)
     key = (key_cache.device, n)
     ws = _workspaces.get(key)
     if ws is None:
@@ -191,18 +205,19 @@ def decode_workspace(key_cache, batch: int, num_q_heads: int, max_blocks_per_seq
 
 def pa_decode(out, q, key_cache, value_cache, block_tables, context_lens,
               scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
-              err_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+              err_word: Optional[torch.Tensor] = None, stream=None,
+              k_scale: float = 1.0, v_scale: float = 1.0) -> torch.Tensor:
     """Fused paged decode attention into `out` (see include/pa.h)."""
     lib = load()
-    desc = cache_desc(key_cache)
+    desc = cache_desc(key_cache, k_scale, v_scale)
     B, Hq, Dq = q.shape
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
     if scale is None:
         scale = 1.0 / math.sqrt(Dq)
     if workspace is None:
-        workspace = decode_workspace(key_cache, B, Hq, MB)
+        workspace = decode_workspace(key_cache, B, Hq, MB, k_scale=k_scale, v_scale=v_scale)
     _check(lib.pa_decode(
-        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        ctypes.byref(desc), _dev(out, "out", _act(key_cache)), _dev(q, "q", _act(key_cache)),
         _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
@@ -214,11 +229,12 @@ def pa_decode(out, q, key_cache, value_cache, block_tables, context_lens,
 def pa_forward_decode(out, q, key_cache, value_cache, k_new, v_new, slot_mapping,
                       block_tables, context_lens, scale: Optional[float] = None,
                       workspace: Optional[torch.Tensor] = None,
-                      err_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                      err_word: Optional[torch.Tensor] = None, stream=None,
+                      k_scale: float = 1.0, v_scale: float = 1.0) -> torch.Tensor:
     """One decode step: store each sequence's newest K/V row at its slot, then
     decode over the whole history into `out` (see include/pa.h)."""
     lib = load()
-    desc = cache_desc(key_cache)
+    desc = cache_desc(key_cache, k_scale, v_scale)
     B, Hq, Dq = q.shape
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
     if slot_mapping.numel() != B:
@@ -226,11 +242,11 @@ def pa_forward_decode(out, q, key_cache, value_cache, k_new, v_new, slot_mapping
     if scale is None:
         scale = 1.0 / math.sqrt(Dq)
     if workspace is None:
-        workspace = decode_workspace(key_cache, B, Hq, MB)
+        workspace = decode_workspace(key_cache, B, Hq, MB, k_scale=k_scale, v_scale=v_scale)
     _check(lib.pa_forward_decode(
-        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        ctypes.byref(desc), _dev(out, "out", _act(key_cache)), _dev(q, "q", _act(key_cache)),
         _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
-        _dev(k_new, "k_new", key_cache.dtype), _dev(v_new, "v_new", key_cache.dtype),
+        _dev(k_new, "k_new", _act(key_cache)), _dev(v_new, "v_new", _act(key_cache)),
         _dev(slot_mapping, "slot_mapping", torch.int64),
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
@@ -242,11 +258,12 @@ def pa_forward_decode(out, q, key_cache, value_cache, k_new, v_new, slot_mapping
 def pa_decode_shared_prefix(out, q, key_cache, value_cache, block_tables, context_lens,
                             prefix_blocks: int, scale: Optional[float] = None,
                             workspace: Optional[torch.Tensor] = None,
-                            err_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                            err_word: Optional[torch.Tensor] = None, stream=None,
+                            k_scale: float = 1.0, v_scale: float = 1.0) -> torch.Tensor:
     """pa_decode for a batch whose tables all start with the same
     prefix_blocks pages (see include/pa.h)."""
     lib = load()
-    desc = cache_desc(key_cache)
+    desc = cache_desc(key_cache, k_scale, v_scale)
     B, Hq, Dq = q.shape
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
     if scale is None:
@@ -260,7 +277,7 @@ def pa_decode_shared_prefix(out, q, key_cache, value_cache, block_tables, contex
             workspace = torch.zeros(max(n, 256), dtype=torch.uint8, device=key_cache.device)
             _workspaces[key] = workspace
     _check(lib.pa_decode_shared_prefix(
-        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        ctypes.byref(desc), _dev(out, "out", _act(key_cache)), _dev(q, "q", _act(key_cache)),
         _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, int(prefix_blocks),
@@ -273,18 +290,19 @@ def pa_decode_shared_prefix(out, q, key_cache, value_cache, block_tables, contex
 def pa_decode_splitk(q, key_cache, value_cache, block_tables, context_lens,
                      partition_tokens: int, part_max, part_sum, part_out,
                      scale: Optional[float] = None, err_word: Optional[torch.Tensor] = None,
-                     stream=None) -> None:
+                     stream=None,
+                     k_scale: float = 1.0, v_scale: float = 1.0) -> None:
     """Per-partition (max, sum, normalised output) partials (see include/pa.h).
     part_max/part_sum: [B, Hq, P] float32; part_out: [B, Hq, P, D] float32."""
     lib = load()
-    desc = cache_desc(key_cache)
+    desc = cache_desc(key_cache, k_scale, v_scale)
     B, Hq, Dq = q.shape
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
     P = part_max.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(Dq)
     _check(lib.pa_decode_splitk(
-        ctypes.byref(desc), _dev(q, "q", key_cache.dtype), _dev(key_cache, "key_cache"),
+        ctypes.byref(desc), _dev(q, "q", _act(key_cache)), _dev(key_cache, "key_cache"),
         _dev(value_cache, "value_cache", key_cache.dtype),
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
@@ -309,20 +327,21 @@ def pa_reduce(out, part_max, part_sum, part_out, context_lens, partition_tokens:
 
 def pa_decode_noalloc(out, q, key_cache, value_cache, block_tables, context_lens,
                       scale: Optional[float] = None, err_word: Optional[torch.Tensor] = None,
-                      stream=None) -> torch.Tensor:
+                      stream=None,
+                      k_scale: float = 1.0, v_scale: float = 1.0) -> torch.Tensor:
     """pa_decode without a workspace, for callers that may not allocate device
     memory: the library's own fixed scratch array (NOALLOC_SCRATCH_BYTES per
     GPU) stands in for it.  Sizes whose workspace would not fit raise
     PaError(PA_ERR_UNSUPPORTED).  Calls that overlap on the GPU share that
     array and race; keep them on one stream (see include/pa.h)."""
     lib = load()
-    desc = cache_desc(key_cache)
+    desc = cache_desc(key_cache, k_scale, v_scale)
     B, Hq, Dq = q.shape
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
     if scale is None:
         scale = 1.0 / math.sqrt(Dq)
     _check(lib.pa_decode_noalloc(
-        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        ctypes.byref(desc), _dev(out, "out", _act(key_cache)), _dev(q, "q", _act(key_cache)),
         _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
