@@ -77,8 +77,10 @@ typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1, PA_DTYPE_FP8_E4M3 =
  * IEEE single precision, ties to the even mantissa, magnitudes at or above
  * 448 saturating to 448).  Served by pa_write_kv_cache, pa_decode,
  * pa_forward_decode and pa_decode_noalloc for head_dim 128, block_size >=
- * 16, at most 8 KV heads, and at most 8 or exactly 16 query heads per KV
- * head; other calls and shapes return PA_ERR_UNSUPPORTED.
+ * 16, 4 or 8 KV heads and at most 8 query heads per KV head; other calls
+ * and shapes return PA_ERR_UNSUPPORTED.  Decode converts the codes exactly
+ * and multiplies them in fp16 tiles (fp32 accumulation), so q must lie
+ * within fp16's range (|q| < 65504).
  */
 
 /* Bits OR'd into *err_word by kernels that meet bad device data. */

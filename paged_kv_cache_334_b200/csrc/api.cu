@@ -163,7 +163,9 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   if (fp8) {
     // 16-token virtual pages (one MMA tile), each warp alone on its KV
     // head's rows of the converted page (a warp never shares them)
-    if (c->block_size < 16 || hkv > 8 || s.warps_per_kv != 1) return s;
+    if (c->block_size < 16 || (hkv != 4 && hkv != 8) || s.warps_per_kv != 1 ||
+        s.heads_per_warp > 8)
+      return s;
     rows = 16;
   }
   s.vbs = c->block_size < rows ? c->block_size : rows;
@@ -479,8 +481,8 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
   const bool fp8 = cache->dtype == PA_DTYPE_FP8_E4M3;
   if (fp8 && (!w.stream || prefix_blocks > 0))
     return fail(PA_ERR_UNSUPPORTED,
-                "FP8 pages: head_dim 128, block_size >= 16, at most 8 KV heads and at most 8 or "
-                "exactly 16 query heads per KV head%s");
+                "FP8 pages: head_dim 128, block_size >= 16, 4 or 8 KV heads and at most 8 "
+                "query heads per KV head%s");
   if (w.stream) {
     StreamPlan sp = plan_stream(cache, num_q_heads);
     const int sms = device_sm_count();
@@ -532,10 +534,10 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
     p.k_scale = cache->k_scale;
     p.v_scale = cache->v_scale;
     if (fp8) {
-      // the consumers see the codes' values (exact in bf16): K's scale goes
-      // into the score scale, V's into the output
-      p.scale_log2 *= cache->k_scale;
-      p.out_scale = cache->v_scale;
+      // the consumers see code value * 2^-8 (exact in fp16): 256 k_scale
+      // goes into the score scale, 256 v_scale into the output
+      p.scale_log2 *= 256.f * cache->k_scale;
+      p.out_scale = 256.f * cache->v_scale;
     }
     const int group = num_q_heads / cache->num_kv_heads;
     p.group = group;
@@ -545,7 +547,9 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
     p.box_bytes = sp.box_bytes;
     p.n_dhalf = sp.n_dhalf;
     const bool mma = cache->dtype != PA_DTYPE_F32;
-    cudaError_t e = mma
+    cudaError_t e = fp8 ? pa::stream::launch_fp8(p, cache->num_kv_heads, sp.smem,
+                                                 static_cast<cudaStream_t>(stream))
+                    : mma
                         ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
                                                   sp.smem, static_cast<cudaStream_t>(stream))
                         : pa::stream::launch_f32(p, cache->head_dim, group, cache->num_kv_heads,

@@ -64,6 +64,10 @@ constexpr int kFirst = 1, kLast = 2, kBad = 4;
 constexpr uint64_t kTablePrefetchMax = 16ull << 20;
 constexpr int kSeqCache = 256;
 
+// Element-type tag of FP8 (E4M3) pages: q and out are bf16, the pages hold
+// codes standing for code * scale.
+struct Fp8E4M3 {};
+
 struct alignas(16) PageDesc {
   int32_t seq, ntok, flags, n_contrib;
   int32_t c_first, slot_bits, pb, toff;
@@ -144,9 +148,28 @@ struct alignas(16) Shared {
 // of tokens g and g + 8 for query heads 2t and 2t + 1, and for each 16-wide
 // d tile the output accumulator of d = 16 dt + g (+8) for the same two heads.
 // ===========================================================================
-template <int D>
+// F16: fp16 tiles (FP8 pages, converted to fp16 by the consumers), with q
+// and P in fp16; else bf16.
+template <int D, bool F16 = false>
 struct MmaConsumer {
   static constexpr int KS = D / 16;  // k steps of QK, d tiles of PV
+  __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    if constexpr (F16)
+      mma_16816_f16(d, a, b0, b1);
+    else
+      mma_16816(d, a, b0, b1);
+  }
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+  }
+  // bf16 pair -> the tile type (fp16 conversion of exact fp32 widening)
+  __device__ __forceinline__ static uint32_t q_pair(uint32_t w) {
+    if constexpr (F16)
+      return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    else
+      return w;
+  }
   uint32_t qb[KS][2];                // Q^T as B operand (d x head), one pair per k step
   float o[KS][4];                    // O^T accumulators
   float m0_, m1_, l0, l1;            // running max / partial normaliser, heads 2t, 2t+1
@@ -170,8 +193,8 @@ struct MmaConsumer {
     for (int k = 0; k < KS; ++k) {
       if (g < nh) {
         const uint32_t *row = reinterpret_cast<const uint32_t *>(qs + (size_t)(hq0 + g) * D);
-        qb[k][0] = row[(k * 16 + t * 2) >> 1];
-        qb[k][1] = row[(k * 16 + t * 2 + 8) >> 1];
+        qb[k][0] = q_pair(row[(k * 16 + t * 2) >> 1]);
+        qb[k][1] = q_pair(row[(k * 16 + t * 2 + 8) >> 1]);
       } else {
         qb[k][0] = qb[k][1] = 0u;
       }
@@ -219,8 +242,8 @@ struct MmaConsumer {
           ldsm_x4(a, smem_u32(kr + k * 32));
           ldsm_x4(b, smem_u32(kr + (k + 1) * 32));
         }
-        mma_16816(sa, a, qb[k][0], qb[k][1]);
-        mma_16816(sb, b, qb[k + 1][0], qb[k + 1][1]);
+        mma(sa, a, qb[k][0], qb[k][1]);
+        mma(sb, b, qb[k + 1][0], qb[k + 1][1]);
       }
       const int r0 = m0 + 16 * u + g;
       const bool v0 = r0 < ntok, v1 = r0 + 8 < ntok;
@@ -253,8 +276,8 @@ struct MmaConsumer {
       add0 += p0 + p2;
       add1 += p1 + p3;
       // P^T (16 tokens x 8 heads) as the B operand: transpose the two 8x8 tiles
-      pb[u][0] = movmatrix_trans(pack_bf16x2(p0, p1));
-      pb[u][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+      pb[u][0] = movmatrix_trans(pack(p0, p1));
+      pb[u][1] = movmatrix_trans(pack(p2, p3));
     }
     l0 = l0 * a0 + add0;
     l1 = l1 * a1 + add1;
@@ -293,7 +316,7 @@ struct MmaConsumer {
         a[1] &= mlo;
         a[2] &= mhi;
         a[3] &= mhi;
-        mma_16816(o[k], a, pb[u][0], pb[u][1]);
+        mma(o[k], a, pb[u][0], pb[u][1]);
       }
     }
   }
@@ -1011,11 +1034,21 @@ __device__ __forceinline__ void write_new_rows_fp8(const Params &p, int32_t s, i
 
 // FP8 pages: this warp's KV-head rows (h * 16 .. + 15) of one staged page,
 // stored as one box of 128 codes per row with the 128-byte swizzle (16-byte
-// chunk c of row r at chunk c ^ (r % 8)), converted exactly into the bf16
-// tile layout the tensor-core consumers read: 64-wide halves of head_dim in
-// boxes box_bytes apart, 8 elements per 16-byte chunk, the same swizzle.
-__device__ __forceinline__ void fp8_rows_to_bf16(const unsigned char *src, unsigned char *dst,
-                                                 int h, const Params &p, int lane) {
+// chunk c of row r at chunk c ^ (r % 8)), converted into the tile layout the
+// tensor-core consumer reads (64-wide halves of head_dim in boxes box_bytes
+// apart, 8 elements per 16-byte chunk, the same swizzle) as fp16 holding
+// code value * 2^-8: the code's sign bit becomes bit 15 and its 7 other bits
+// bits 7..13 -- exact for every code, subnormals included, by integer
+// operations only (no conversion instructions).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t &lo, uint32_t &hi) {
+  const uint32_t a = __byte_perm(x, 0u, 0x1404);  // codes 0, 1 in the high byte of each half
+  const uint32_t b = __byte_perm(x, 0u, 0x3424);  // codes 2, 3
+  lo = (a & 0x80008000u) | ((a >> 1) & 0x3f803f80u);
+  hi = (b & 0x80008000u) | ((b >> 1) & 0x3f803f80u);
+}
+
+__device__ __forceinline__ void fp8_rows_to_f16(const unsigned char *src, unsigned char *dst,
+                                                int h, const Params &p, int lane) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int k = lane + 32 * i;       // 16 rows x 8 chunks
@@ -1023,12 +1056,12 @@ __device__ __forceinline__ void fp8_rows_to_bf16(const unsigned char *src, unsig
     const int c = k >> 4;              // chunk of 16 codes: elements 16c .. 16c + 15
     const uint4 x = *reinterpret_cast<const uint4 *>(src + r * 128 + ((c ^ (r & 7)) << 4));
     uint32_t y[8];
-    e4m3x4_to_bf16x4(x.x, y[0], y[1]);
-    e4m3x4_to_bf16x4(x.y, y[2], y[3]);
-    e4m3x4_to_bf16x4(x.z, y[4], y[5]);
-    e4m3x4_to_bf16x4(x.w, y[6], y[7]);
+    e4m3x4_to_f16x4(x.x, y[0], y[1]);
+    e4m3x4_to_f16x4(x.y, y[2], y[3]);
+    e4m3x4_to_f16x4(x.z, y[4], y[5]);
+    e4m3x4_to_f16x4(x.w, y[6], y[7]);
     unsigned char *row = dst + (c >> 2) * p.box_bytes + r * 128;
-    const int j0 = 2 * (c & 3);  // first of the two bf16 chunks in its half
+    const int j0 = 2 * (c & 3);  // first of the two 16-byte chunks in its half
     *reinterpret_cast<uint4 *>(row + ((j0 ^ (r & 7)) << 4)) = make_uint4(y[0], y[1], y[2], y[3]);
     *reinterpret_cast<uint4 *>(row + (((j0 + 1) ^ (r & 7)) << 4)) =
         make_uint4(y[4], y[5], y[6], y[7]);
@@ -1044,17 +1077,20 @@ __device__ __forceinline__ void fp8_rows_to_bf16(const unsigned char *src, unsig
 template <typename T, int D, int G, int NCW>
 __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     decode_stream_kernel(const __grid_constant__ Params p) {
-  constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value;
+  // T: __nv_bfloat16, float, or Fp8E4M3 (FP8 pages; q and out bf16)
+  constexpr bool kFp8 = std::is_same<T, Fp8E4M3>::value;
+  constexpr bool kMma = std::is_same<T, __nv_bfloat16>::value || kFp8;
+  using TA = typename std::conditional<kFp8, __nv_bfloat16, T>::type;  // q, out
   constexpr int kFmaG = kMma ? 1 : (G > 0 ? G : 1);  // fp32 consumer's group
-  constexpr int kScoreFloats = kMma ? 1 : FmaConsumer<T, D, kFmaG>::E;
+  constexpr int kScoreFloats = kMma ? 1 : FmaConsumer<TA, D, kFmaG>::E;
   static_assert(sizeof(Shared) + sizeof(PageDesc) * kMaxStages * kMaxPPS +
                         sizeof(float) * NCW * kScoreFloats <= kHdrBytes,
                 "header region");
   static_assert(sizeof(Shared) % 16 == 0 && sizeof(PageDesc) % 16 == 0,
                 "descriptors and score buffers need 16-byte alignment");
   using MmaCons =
-      typename std::conditional<G == 16, HeadRowConsumer<D>, MmaConsumer<D>>::type;
-  using Cons = typename std::conditional<kMma, MmaCons, FmaConsumer<T, D, kFmaG>>::type;
+      typename std::conditional<G == 16, HeadRowConsumer<D>, MmaConsumer<D, kFp8>>::type;
+  using Cons = typename std::conditional<kMma, MmaCons, FmaConsumer<TA, D, kFmaG>>::type;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Shared &sh = *reinterpret_cast<Shared *>(smem_raw);
   PageDesc *descs = reinterpret_cast<PageDesc *>(smem_raw + sizeof(Shared));
@@ -1063,7 +1099,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   // stages start 1024-byte aligned (the 128-byte swizzle repeats every 1 KB)
   unsigned char *stages =
       smem_raw + (((smem_u32(smem_raw) + p.hdr_bytes + 1023u) & ~1023u) - smem_u32(smem_raw));
-  // FP8 pages: the bf16 page the consumers convert into (K, then V)
+  // FP8 pages: the fp16 page the consumers convert into (K, then V)
   unsigned char *scratch = stages + (size_t)p.stages * p.stage_bytes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1337,7 +1373,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           const PageDesc d = descs[slot * kMaxPPS + k];
           if (d.flags & kFirst) {
             cs.reset();
-            const T *qs = reinterpret_cast<const T *>(qst + (size_t)k * p.q_bytes);
+            const TA *qs = reinterpret_cast<const TA *>(qst + (size_t)k * p.q_bytes);
             if constexpr (kMma) {
               cs.load_q(qs, hq0, p.heads_per_warp, lane);
             } else {
@@ -1350,12 +1386,19 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             const unsigned char *kp = kst + (size_t)k * p.vpage_stride;
             const unsigned char *vp = vst + (size_t)k * p.vpage_stride;
             if constexpr (kMma) {
-              if (p.fp8) {
+              if constexpr (kFp8) {
                 // one warp per KV head: its rows of the converted page are its own
                 unsigned char *sk = scratch, *sv = scratch + (size_t)p.n_dhalf * p.box_bytes;
-                fp8_rows_to_bf16(kp, sk, h, p, lane);
-                fp8_rows_to_bf16(vp, sv, h, p, lane);
+                fp8_rows_to_f16(kp, sk, h, p, lane);
+                fp8_rows_to_f16(vp, sv, h, p, lane);
                 __syncwarp();
+                // the products read the converted copy: the stage can go back
+                // to the producer after its last page is converted (q, read
+                // at the sequence's first page, is in registers already)
+                if (k == npg - 1) {
+                  if (lane == 0) mbar_arrive(&sh.empty[slot]);
+                  released = true;
+                }
                 kp = sk;
                 vp = sv;
               }
@@ -1367,13 +1410,13 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           if (d.flags & kLast) {
             // The flush works on registers only: hand the stage back first
             // when this was its last page, so the producer is not held up.
-            if (k == npg - 1) {
+            if (k == npg - 1 && !released) {
               __syncwarp();
               if (lane == 0) mbar_arrive(&sh.empty[slot]);
               released = true;
             }
             if constexpr (kMma) {
-              cs.template flush<T>(p, d, hq0, p.heads_per_warp, c, lane);
+              cs.template flush<TA>(p, d, hq0, p.heads_per_warp, c, lane);
             } else {
               cs.flush(p, d, hq0, c, lane);
             }
@@ -1411,7 +1454,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             make_float2(-INFINITY, 0.f);
     } else {
       for (int64_t x = tid; x < n; x += blockDim.x)
-        Elem<T>::store1(p.out, (int64_t)s * n + x, 0.f);
+        Elem<TA>::store1(p.out, (int64_t)s * n + x, 0.f);
     }
   }
 }

@@ -86,8 +86,9 @@ struct Params {
   int32_t box_bytes;                // bytes of one box (64 x vbs x Hkv bf16)
   int32_t n_dhalf;                  // boxes per page per tensor (head_dim / 64)
   // FP8 pages: one box of 128 codes x vbs x Hkv per page and tensor, which
-  // the consumers convert into a bf16 page (the tile layout) after the
-  // stages; scale_log2 then includes k_scale and out_scale is v_scale
+  // the consumers convert into an fp16 page (the tile layout, code value *
+  // 2^-8) after the stages; scale_log2 then includes 256 k_scale and
+  // out_scale is 256 v_scale
   int32_t fp8;
   float out_scale;
   float k_scale, v_scale;  // FP8 pages: the fused write's quantisation scales
@@ -96,6 +97,8 @@ struct Params {
 
 cudaError_t launch_bf16(const Params &p, int head_dim, int group, int hkv, size_t smem,
                         cudaStream_t stream);
+// FP8 pages (head_dim 128, up to 8 query heads per KV head, 4 or 8 KV heads).
+cudaError_t launch_fp8(const Params &p, int hkv, size_t smem, cudaStream_t stream);
 // Second kernel of pa_decode: merge the partials of sequences split across CTAs.
 cudaError_t launch_merge_bf16(const Params &p, int head_dim, cudaStream_t stream);
 cudaError_t launch_merge_f32(const Params &p, int head_dim, cudaStream_t stream);

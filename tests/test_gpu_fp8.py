@@ -4,7 +4,7 @@ The write (bf16 rows divided by the tensor's scale in IEEE single precision,
 rounded to the nearest E4M3 code, saturating at 448) is bit-exact; decode
 over the pages (values code * scale, q bf16) is held to the bf16 tolerance
 (<= 2e-2 max-abs, <= 1e-2 mean-abs): the kernel converts the codes exactly
-and computes as on bf16 pages.  Unused slots hold the NaN code 0x7F, so an
+to fp16 and computes in fp16 tiles with fp32 accumulation.  Unused slots hold the NaN code 0x7F, so an
 over-read shows as NaN.
 """
 import math
@@ -115,7 +115,7 @@ FP8_SHAPES = [
     (8, 8, 16),    # 1
     (16, 8, 256),  # 256-token pages in 16-token virtual pages
     (16, 4, 32),
-    (64, 4, 16),   # 16 heads per KV head: the head-row consumer
+    (8, 4, 64),    # 2
     (32, 4, 128),  # 8
 ]
 
@@ -171,10 +171,11 @@ def test_fp8_unsupported_shapes_are_refused():
         return torch.zeros(nb, bs, hkv, d, dtype=torch.uint8, device="cuda").view(
             torch.float8_e4m3fn)
 
+    big = torch.zeros(2, 64, 128, dtype=torch.bfloat16, device="cuda")
     for kc, qq in [(cache(8, 8, 8, 128), q),                 # 8-token pages
-                   (cache(8, 16, 16, 128), q[:, :, :]),      # 16 KV heads (group 2)
-                   (cache(8, 16, 4, 128), torch.zeros(2, 128, 128, dtype=torch.bfloat16,
-                                                      device="cuda"))]:  # group 32
+                   (cache(8, 16, 16, 128), q),               # 16 KV heads (group 2)
+                   (cache(8, 16, 2, 128), q),                # 2 KV heads (group 16)
+                   (cache(8, 16, 4, 128), big)]:             # group 16
         out = torch.empty_like(qq)
         with pytest.raises(pa.PaError) as e:
             pa.pa_decode(out, qq, kc, kc.clone(), bt, cl, k_scale=1.0, v_scale=1.0)
