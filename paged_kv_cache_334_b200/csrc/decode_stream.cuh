@@ -1210,7 +1210,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     const int n_stages = (int)((end - start + p.pps - 1) / p.pps);
     if (warp == 0) {
       // ===================== producer =====================
-      const int nbox = p.fp8 ? 1 : p.n_dhalf;  // tensor copies per page and tensor
+      const int nbox = kFp8 ? 1 : p.n_dhalf;  // tensor copies per page and tensor
       PageWalker wk;
       wk.init(p, cached ? &sh : nullptr, sh.s_begin, sh.vlb_begin, sh.P_begin, start, end,
               lane);
@@ -1242,7 +1242,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             const int32_t pos = wk.ctx_s - 1;
             const int64_t want = (int64_t)pb * p.block_size + (pos & (p.block_size - 1));
             if (!bad_block && wk.slot_s == want) {
-              if (p.fp8)
+              if constexpr (kFp8)
                 write_new_rows_fp8(p, wk.s, want, lane);
               else
                 write_new_rows(p, wk.s, want, lane);
