@@ -861,6 +861,8 @@ pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
                                     context_lens, batch, num_q_heads,
                                     max_blocks_per_seq, scale);
   if (s != PA_OK) return s;
+  if (cache->dtype == PA_DTYPE_FP8_E4M3)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode_splitk takes F32 or BF16 pages, not FP8%s");
   if (partition_tokens <= 0 || partition_tokens % cache->block_size != 0)
     return fail(PA_ERR_INVALID_ARG,
                 "partition_tokens must be a positive multiple of block_size%s (got %lld)", "",

@@ -443,6 +443,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   if (a.batch == 0 || a.max_parts == 0) return cudaSuccess;
   dim3 grid((unsigned)a.max_parts, (unsigned)(a.num_kv_heads * kp.head_tiles),
             (unsigned)a.batch);
+  if (a.dtype != PA_DTYPE_BF16 && a.dtype != PA_DTYPE_F32) return cudaErrorInvalidValue;
   const bool bf16 = a.dtype == PA_DTYPE_BF16;
   if (a.head_dim == 64)
     return bf16 ? launch_dtype_dim<__nv_bfloat16, 64>(kp, gt, grid, stream)

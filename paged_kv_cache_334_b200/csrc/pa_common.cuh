@@ -168,25 +168,4 @@ __device__ __forceinline__ uint4 bf16x16_to_e4m3(const uint4 &a, const uint4 &b,
   return make_uint4(c[0], c[1], c[2], c[3]);
 }
 
-// Four codes (code 0 in the low byte) -> four bf16 values, exactly (every
-// E4M3 value is an fp16 and a bf16 value; NaN stays NaN): lo holds elements
-// 0 and 1, hi elements 2 and 3, the lower element in the low half.
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t x, uint32_t &lo, uint32_t &hi) {
-  float f[4];
-  asm("{ .reg .b16 a, b, c0, c1, c2, c3; .reg .b32 h01, h23;\n\t"
-      "mov.b32 {a, b}, %4;\n\t"
-      "cvt.rn.f16x2.e4m3x2 h01, a;\n\t"
-      "cvt.rn.f16x2.e4m3x2 h23, b;\n\t"
-      "mov.b32 {c0, c1}, h01;\n\t"
-      "mov.b32 {c2, c3}, h23;\n\t"
-      "cvt.f32.f16 %0, c0;\n\t"
-      "cvt.f32.f16 %1, c1;\n\t"
-      "cvt.f32.f16 %2, c2;\n\t"
-      "cvt.f32.f16 %3, c3; }"
-      : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3])
-      : "r"(x));
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(f[1]), "f"(f[0]));
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(f[3]), "f"(f[2]));
-}
-
 }  // namespace pa

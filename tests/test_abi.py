@@ -165,3 +165,36 @@ def test_forward_decode_argument_checks(lib):
     assert call(Hq=30) == pa.PA_ERR_INVALID_ARG
     assert call(dsc=_desc(d=96)) == pa.PA_ERR_UNSUPPORTED
     assert call(B=0, sm=None, k_new=None, v_new=None) == pa.PA_OK
+
+
+def _fp8(nb=16, bs=16, hkv=8, d=128, ks=0.25, vs=0.5):
+    return pa.CacheDesc(nb, bs, hkv, d, pa.PA_DTYPE_FP8_E4M3, ks, vs)
+
+
+def test_fp8_argument_checks_need_no_device(lib):
+    """FP8 pages: scales and shapes are checked on the host, before any
+    device work (every pointer here is fake)."""
+    # scales must be finite and > 0
+    for ks, vs in [(0.0, 1.0), (1.0, -1.0), (float("nan"), 1.0), (float("inf"), 1.0)]:
+        assert _decode(lib, _fp8(ks=ks, vs=vs)) == pa.PA_ERR_INVALID_ARG
+    assert b"scales" in lib.pa_last_error_message()
+    # head_dim 128 only
+    assert _decode(lib, _fp8(d=64)) == pa.PA_ERR_UNSUPPORTED
+    # the page-stream shapes: block_size >= 16, 4 or 8 KV heads, <= 8 heads per KV head
+    assert _decode(lib, _fp8(bs=8)) == pa.PA_ERR_UNSUPPORTED
+    assert _decode(lib, _fp8(hkv=2), Hq=4) == pa.PA_ERR_UNSUPPORTED
+    assert _decode(lib, _fp8(hkv=4), Hq=64) == pa.PA_ERR_UNSUPPORTED
+    assert b"FP8" in lib.pa_last_error_message()
+    # split-K partials and the shared-prefix call take bf16 / fp32 pages only
+    P = 8
+    assert lib.pa_decode_splitk(ctypes.byref(_fp8()), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4,
+                                0.1, 16, P, FAKE, FAKE, FAKE, None, None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_decode_shared_prefix(ctypes.byref(_fp8()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                       2, 32, 4, 1, 0.1, FAKE, 1 << 30, None,
+                                       None) == pa.PA_ERR_UNSUPPORTED
+    # the write: the same descriptor checks
+    assert lib.pa_write_kv_cache(ctypes.byref(_fp8(d=64)), FAKE, FAKE, FAKE, FAKE, FAKE, 2, None,
+                                 None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_write_kv_cache(ctypes.byref(_fp8(ks=0.0)), FAKE, FAKE, FAKE, FAKE, FAKE, 2,
+                                 None, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_version() == 200
