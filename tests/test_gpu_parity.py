@@ -470,3 +470,20 @@ def test_tensor_decode_long_and_ragged(Hq, Hkv, D, bs, lens):
     for b, n in enumerate(lens):
         if n == 0:
             assert not to_f64(out)[b].any()
+
+
+def test_tensor_decode_batch_above_one_scan_pass():
+    """400 sequences of 64 query heads on one KV head: the tile kernel's
+    prologue scans the context lengths in several passes of its threads."""
+    rng = np.random.default_rng(12)
+    lens = [int(x) for x in rng.integers(0, 300, size=400)]
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=len(lens), num_q_heads=64, num_kv_heads=1,
+                           head_dim=128, block_size=32, context_lens=lens, seed=12,
+                           new_tokens=True)
+    d = upload(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gpu_write_and_decode(w, d, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref, _, _, _ = oracle_after_write(w)
+    assert_close(to_f64(out), ref, w.dtype, "tensor decode, 400 sequences")

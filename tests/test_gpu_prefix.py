@@ -200,3 +200,20 @@ def test_tensor_suffix_bad_page_and_length():
     ref = _decode_ref(w)
     keep = [0, 3, 4]
     assert_close(got[keep], ref[keep], w.dtype, "unaffected sequences")
+
+
+def test_tensor_suffix_batch_above_one_scan_pass():
+    """400 sequences: the suffix kernel's prologue takes several scan passes
+    and the prefix kernel two waves of CTAs."""
+    npre, bs = 3, 32
+    rng = np.random.default_rng(13)
+    lens = [npre * bs + int(x) for x in rng.integers(0, 200, size=400)]
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=len(lens), num_q_heads=64,
+                           num_kv_heads=1, head_dim=128, block_size=bs, context_lens=lens,
+                           seed=13, prefix_blocks=npre)
+    d = upload(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = shared_prefix(d, npre, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert_close(to_f64(out), _decode_ref(w), w.dtype, "tensor suffix, 400 sequences")
