@@ -66,6 +66,9 @@ def _load():
         lib.orc_write_kv_cache.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32]
         lib.orc_write_kv_cache.restype = ctypes.c_int
         f32 = ctypes.c_float
+        lib.orc_prefill.argtypes = [P, P, P, ctypes.c_int, i32, i32, i32, i32, P, P, P, i32, i32,
+                                    i32, dbl, P, P]
+        lib.orc_prefill.restype = ctypes.c_int
         lib.orc_e4m3_encode_array.argtypes = [P, i64, P]
         lib.orc_e4m3_encode_array.restype = None
         lib.orc_write_kv_cache_fp8.argtypes = [P, P, P, P, P, i32, f32, f32, i32, i32, i32, i32]
@@ -262,3 +265,33 @@ def write_kv_cache(key_cache, value_cache, k_new, v_new, slot_mapping) -> int:
     vn = np.ascontiguousarray(v_new, dtype=key_cache.dtype)
     return _load().orc_write_kv_cache(_ptr(key_cache), _ptr(value_cache), _ptr(kn), _ptr(vn),
                                       _ptr(sm), sm.size, key_cache.itemsize, NB, bs, Hkv, D)
+
+
+def prefill(q, key_cache, value_cache, block_tables, context_lens, query_start,
+            scale: Optional[float] = None):
+    """Paged (chunked) prefill with the causal mask (teaching page, "Where is
+    the attention mask"; route page, "decode attention and prefill attention
+    are different").  Sequence b's new tokens are rows query_start[b] ..
+    query_start[b+1]-1 of q [T, Hq, D]; their K/V are already stored at their
+    slots, its history holds context_lens[b] tokens including them, and new
+    token j (position context_lens[b] - n_b + j) attends to positions 0..that
+    position through the block table.  Returns (out [T, Hq, D] float64,
+    flags [B])."""
+    NB, bs, Hkv, D = key_cache.shape
+    T, Hq, Dq = q.shape
+    assert Dq == D and q.dtype == key_cache.dtype
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    B = cl.size
+    assert qs.size == B + 1 and qs[-1] == T
+    qq = np.ascontiguousarray(q)
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    flags = np.zeros(B, dtype=np.int32)
+    _load().orc_prefill(_ptr(qq), _ptr(key_cache), _ptr(value_cache), _dtype_code(key_cache),
+                        NB, bs, Hkv, D, _ptr(bt), _ptr(cl), _ptr(qs), B, Hq, bt.shape[1],
+                        float(scale), _ptr(out), _ptr(flags))
+    return out, flags
+

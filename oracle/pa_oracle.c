@@ -290,6 +290,68 @@ int orc_decode(const void *q, const void *key_cache, const void *value_cache,
   return all;
 }
 
+/* Paged (chunked) prefill with the causal mask.  Teaching page, section
+ * "Where is the attention mask": in prefill every prompt token sees only
+ * itself and the tokens before it; route page, section "decode attention
+ * and prefill attention are different": prefill processes a whole prompt
+ * (or a chunk of it) at once.  Sequence b brings n_b = qstart[b+1] -
+ * qstart[b] new tokens whose K/V rows are already stored at their slots;
+ * its history is context_lens[b] tokens including them, so new token j sits
+ * at position p = context_lens[b] - n_b + j and attends to positions
+ * [0, p], read through the block table (gather first, then attention, as in
+ * orc_decode).  q, out: [qstart[batch], Hq, D] (q stored in dtype, out
+ * double).  n_b < 0 or n_b > context_lens[b], or bad metadata, flags the
+ * sequence and its rows are zero.  Returns the OR of all flags. */
+int orc_prefill(const void *q, const void *key_cache, const void *value_cache, int dtype,
+                int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                int32_t head_dim, const int32_t *block_tables, const int32_t *context_lens,
+                const int32_t *qstart, int32_t batch, int32_t num_q_heads, int32_t max_blocks,
+                double scale, double *out, int32_t *seq_flags) {
+  const int64_t qrow = (int64_t)num_q_heads * head_dim;
+  const int64_t kvrow = (int64_t)num_kv_heads * head_dim;
+  const int32_t group = num_q_heads / num_kv_heads;
+  int all = 0;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t n = qstart[b + 1] - qstart[b];
+    const int32_t ctx = context_lens[b];
+    double *rows = out + (int64_t)qstart[b] * qrow;
+    double *keys = NULL, *values = NULL;
+    int flags = 0;
+    if (n < 0 || n > ctx) {
+      flags = ORC_FLAG_CONTEXT_LEN;
+    } else {
+      flags = orc_gather_seq(key_cache, value_cache, dtype, num_blocks, block_size,
+                             num_kv_heads, head_dim, block_tables + (int64_t)b * max_blocks,
+                             max_blocks, ctx, &keys, &values);
+    }
+    if (flags || n <= 0) {
+      for (int64_t e = 0; n > 0 && e < (int64_t)n * qrow; ++e) rows[e] = 0.0;
+    } else {
+      double *scores = (double *)malloc(sizeof(double) * ctx);
+      double *qh = (double *)malloc(sizeof(double) * head_dim);
+      for (int32_t j = 0; j < n; ++j) {
+        const int64_t pos = (int64_t)ctx - n + j;
+        for (int32_t hq = 0; hq < num_q_heads; ++hq) {
+          const int32_t h = hq / group;
+          const int64_t qi = ((int64_t)qstart[b] + j) * qrow + (int64_t)hq * head_dim;
+          for (int32_t d = 0; d < head_dim; ++d) qh[d] = orc_load(q, qi + d, dtype);
+          double m, l;
+          orc_attend_range(qh, keys + (int64_t)h * head_dim, values + (int64_t)h * head_dim,
+                           kvrow, 0, pos + 1, head_dim, scale, scores, &m, &l,
+                           rows + (int64_t)j * qrow + (int64_t)hq * head_dim);
+        }
+      }
+      free(scores);
+      free(qh);
+    }
+    free(keys);
+    free(values);
+    if (seq_flags) seq_flags[b] = flags;
+    all |= flags;
+  }
+  return all;
+}
+
 /* Per-partition partials.  Partition p of sequence b covers tokens
  * [p*P, min((p+1)*P, ctx)).  For every non-empty partition:
  *   part_max[b,hq,p] = max_t s_t,  part_sum[b,hq,p] = sum_t exp(s_t - max),

@@ -445,3 +445,104 @@ def test_write_kv_cache_fp8_worked_example():
     assert not kc[0].any() and not kc[1, 0].any()
     assert oracle.write_kv_cache_fp8(kc, vc, k_new, v_new, np.array([4, 0]), 0.5, 2.0) == \
         oracle.FLAG_SLOT
+
+
+# ---------------------------------------------------------------------------
+# Paged (chunked) prefill with the causal mask (next-row groundwork: the
+# oracle comes before any kernel).  Pinned against torch's causal SDPA on
+# K/V gathered here by plain indexing, and by invariants.
+# ---------------------------------------------------------------------------
+def _prompt_case(lens, seed, Hq=8, Hkv=2, D=32, bs=4):
+    w = wl.custom_workload(dtype=wl.DTYPE_F32, batch=len(lens), num_q_heads=Hq,
+                           num_kv_heads=Hkv, head_dim=D, block_size=bs, context_lens=lens,
+                           seed=seed)
+    rng = np.random.default_rng(seed + 100)
+    q = rng.standard_normal((int(sum(lens)), Hq, D)).astype(np.float32)
+    qs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return w, q, qs
+
+
+def _rows_by_table(cache, table, n, bs):
+    return np.stack([cache[table[t // bs], t % bs] for t in range(n)]).astype(np.float64)
+
+
+def test_prefill_matches_torch_causal_sdpa():
+    lens = [11, 7, 1]
+    w, q, qs = _prompt_case(lens, seed=3)
+    out, fl = oracle.prefill(q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, qs)
+    assert not fl.any()
+    D = w.head_dim
+    for b, n in enumerate(lens):
+        K = _rows_by_table(w.key_cache, w.block_tables[b], n, w.block_size)
+        V = _rows_by_table(w.value_cache, w.block_tables[b], n, w.block_size)
+        qt = torch.from_numpy(q[qs[b]:qs[b + 1]].astype(np.float64)).permute(1, 0, 2)[None]
+        kt = torch.from_numpy(K).permute(1, 0, 2)[None]
+        vt = torch.from_numpy(V).permute(1, 0, 2)[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qt, kt, vt, is_causal=True, scale=1.0 / math.sqrt(D), enable_gqa=True)
+        ref = ref[0].permute(1, 0, 2).numpy()
+        assert np.allclose(out[qs[b]:qs[b + 1]], ref, rtol=0, atol=1e-12)
+
+
+def test_prefill_in_chunks_equals_one_shot():
+    lens = [13, 9]
+    w, q, qs = _prompt_case(lens, seed=4)
+    full, _ = oracle.prefill(q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, qs)
+    cut = [5, 9]  # the second sequence has nothing left for chunk 2
+    q1 = np.concatenate([q[qs[b]:qs[b] + cut[b]] for b in range(2)])
+    q2 = np.concatenate([q[qs[b] + cut[b]:qs[b + 1]] for b in range(2)])
+    qs1 = np.array([0, cut[0], cut[0] + cut[1]], dtype=np.int32)
+    rest = [lens[b] - cut[b] for b in range(2)]
+    qs2 = np.array([0, rest[0], rest[0] + rest[1]], dtype=np.int32)
+    o1, f1 = oracle.prefill(q1, w.key_cache, w.value_cache, w.block_tables,
+                            np.array(cut, dtype=np.int32), qs1)
+    o2, f2 = oracle.prefill(q2, w.key_cache, w.value_cache, w.block_tables, w.context_lens, qs2)
+    assert not f1.any() and not f2.any()
+    for b in range(2):
+        assert np.array_equal(o1[qs1[b]:qs1[b + 1]], full[qs[b]:qs[b] + cut[b]])
+        assert np.array_equal(o2[qs2[b]:qs2[b + 1]], full[qs[b] + cut[b]:qs[b + 1]])
+
+
+def test_prefill_last_token_is_decode_and_first_is_v0():
+    lens = [10, 6]
+    w, q, qs = _prompt_case(lens, seed=5)
+    out, _ = oracle.prefill(q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, qs)
+    last = np.stack([q[qs[b + 1] - 1] for b in range(2)])
+    dec, _ = oracle.decode(last, w.key_cache, w.value_cache, w.block_tables, w.context_lens,
+                           1.0 / math.sqrt(w.head_dim))
+    group = w.num_q_heads // w.num_kv_heads
+    for b in range(2):
+        assert np.array_equal(out[qs[b + 1] - 1], dec[b])
+        # the first prompt token sees only itself: out = V_0 of its KV head
+        v0 = w.value_cache[w.block_tables[b, 0], 0].astype(np.float64)
+        for hq in range(w.num_q_heads):
+            assert np.array_equal(out[qs[b], hq], v0[hq // group])
+
+
+def test_prefill_is_causal():
+    """NaN in every slot after position p leaves the rows up to p unchanged."""
+    lens = [12]
+    w, q, qs = _prompt_case(lens, seed=6)
+    out, _ = oracle.prefill(q, w.key_cache, w.value_cache, w.block_tables, w.context_lens, qs)
+    p = 6
+    kc, vc = w.key_cache.copy(), w.value_cache.copy()
+    for t in range(p + 1, lens[0]):
+        pb, off = w.block_tables[0, t // w.block_size], t % w.block_size
+        kc[pb, off] = np.nan
+        vc[pb, off] = np.nan
+    out2, _ = oracle.prefill(q, kc, vc, w.block_tables, w.context_lens, qs)
+    assert np.array_equal(out2[:p + 1], out[:p + 1])
+    assert np.isnan(out2[p + 1:]).all()
+
+
+def test_prefill_flags():
+    lens = [8, 5]
+    w, q, qs = _prompt_case(lens, seed=7)
+    cl = np.array([8, 3], dtype=np.int32)  # sequence 1: 5 new tokens but a 3-token history
+    out, fl = oracle.prefill(q, w.key_cache, w.value_cache, w.block_tables, cl, qs)
+    assert fl.tolist() == [0, oracle.FLAG_CONTEXT_LEN]
+    assert not out[qs[1]:].any() and out[:qs[1]].any()
+    bt = w.block_tables.copy()
+    bt[0, 1] = w.num_blocks + 3
+    out, fl = oracle.prefill(q, w.key_cache, w.value_cache, bt, w.context_lens, qs)
+    assert fl[0] == oracle.FLAG_BLOCK_ID and not out[:qs[1]].any()
