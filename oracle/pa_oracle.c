@@ -35,6 +35,13 @@
  *     merge: the running-max / normaliser bookkeeping of the online softmax
  *     (optimisation-route page, section "What the attention kernel really
  *     does", blockwise softmax paragraph), applied to whole partitions.
+ *   - Paged (chunked) prefill with the causal mask (teaching page, section
+ *     "Where is the attention mask"): new token j of a chunk of n attends to
+ *     positions 0 .. context_len - n + j, gathered through the block table.
+ *   - FP8 pages (a reading: the pages name quantised KV as a later
+ *     addition): E4M3 codes of the OCP 8-bit floating point format, value =
+ *     code * per-tensor scale; the write rounds x / scale (IEEE single
+ *     precision division) to the nearest code, ties to even, saturating.
  *
  * Readings where the pages are silent: query head hq uses KV head
  * hq / (Hq / Hkv) (contiguous GQA groups); bf16 values are widened exactly
