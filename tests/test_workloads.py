@@ -110,3 +110,36 @@ def test_block_size_override_keeps_lengths_and_pages_them_anew():
         wl.make_workload("gqa_bf16", block_size=48)
     with pytest.raises(ValueError):
         wl.make_workload("mqa_prefix_bf16", block_size=16)
+
+
+def test_gqa_fp8_pages():
+    """gqa_fp8: gqa_bf16's lengths; E4M3 codes with exponent fields 3..9 in
+    visible slots, the NaN code everywhere else (the newest tokens' slots
+    too, until the write), bf16 q and new rows, and half the cache bytes."""
+    w = wl.make_workload("gqa_fp8", seed=1)
+    g = wl.make_workload("gqa_bf16", seed=1)
+    assert w.context_lens.tolist() == g.context_lens.tolist()
+    assert w.key_cache.dtype == np.uint8 and w.q.dtype == np.uint16
+    assert w.k_new.dtype == np.uint16 and w.k_new.shape == (w.batch, 8, 128)
+    assert (w.k_scale, w.v_scale) == (wl.FP8_K_SCALE, wl.FP8_V_SCALE)
+    bs = w.block_size
+    live = np.zeros((w.num_blocks, bs), dtype=bool)
+    for b, ctx in enumerate(w.context_lens):
+        for t in range(int(ctx) - 1):  # the newest token's slot is poisoned too
+            live[w.block_tables[b, t // bs], t % bs] = True
+    for cache in (w.key_cache, w.value_cache):
+        vis = cache[live]
+        assert not np.any(vis == 0x7F)
+        expo = (vis >> 3) & 15
+        assert expo.min() >= 3 and expo.max() <= 9
+        assert np.all(cache[~live] == 0x7F)
+    for b, ctx in enumerate(w.context_lens):
+        t = int(ctx) - 1
+        pb, off = w.block_tables[b, t // bs], t % bs
+        assert w.slot_mapping[b] == pb * bs + off
+    # the cache rows are half as wide as bf16 ones; q, out and new rows are not
+    kv_bf16 = wl.roofline_bytes(g, include_write=False)
+    kv_fp8 = wl.roofline_bytes(w, include_write=False)
+    qo = 2 * w.batch * w.num_q_heads * w.head_dim * 2
+    meta = w.block_tables.size * 4 + w.context_lens.size * 4
+    assert kv_fp8 - qo - meta == (kv_bf16 - qo - meta) // 2
