@@ -1,6 +1,7 @@
-// suffix.cu -- the private part of every sequence for pa_decode_shared_prefix
-// when one KV head serves 64 or 128 query heads, on the 5th-generation tensor
-// cores (tcgen05).
+// suffix.cu -- decode attention on the 5th-generation tensor cores (tcgen05)
+// when one KV head serves 64 or 128 query heads: the private part of every
+// sequence for pa_decode_shared_prefix, and with no prefix the whole of
+// pa_decode / pa_forward_decode (then finish_kernel merges and writes bf16).
 //
 // Page "Operators and compilers: inference attention and KV kernels",
 // section 4.1: with that many query heads per KV head, decode attention does
@@ -28,7 +29,8 @@
 //              copies into shared memory), one descriptor per tile, the Q
 //              tile of each pair it starts, K and V tiles into separate rings
 //              (tiled copies, no multicast);
-//   warp 1     tcgen05.mma: S_b = Q K^T, then O += P V of the previous tile;
+//   warp 1     tcgen05.mma: S_b = Q K^T of the next tile and O += P V of the
+//              previous one, whichever has its inputs first;
 //   warps 2-9  softmax, two warps per tensor-memory subpartition (each owns
 //              half of a tile's 128 columns and of O's), and the epilogue of
 //              every pair segment;
