@@ -198,3 +198,52 @@ def test_fp8_argument_checks_need_no_device(lib):
     assert lib.pa_write_kv_cache(ctypes.byref(_fp8(ks=0.0)), FAKE, FAKE, FAKE, FAKE, FAKE, 2,
                                  None, None) == pa.PA_ERR_INVALID_ARG
     assert lib.pa_version() == 200
+
+
+def _round256(x):
+    return (x + 255) // 256 * 256
+
+
+def test_workspace_sizes_of_the_tensor_core_path(lib):
+    """Groups of 64 or 128 query heads (bf16) decode on the tile kernel: the
+    workspace holds per-CTA partials for 192 CTAs x 2 slots, one 16-byte
+    record per (sequence, KV head) and each row's fp32 result, independent
+    of the table width; the shared-prefix call asks for at least as much."""
+    for hkv, hq, d in [(1, 64, 128), (2, 128, 128), (1, 128, 64)]:
+        desc = _desc(nb=1000, bs=32, hkv=hkv, d=d)
+        B = 300
+        slots = 192 * 2 * hq
+        rows = B * hq
+        want = _round256(slots * 2 * 4)
+        want = _round256(want + slots * d * 4)
+        want = _round256(want + B * hkv * 16)
+        want = _round256(want + rows * 2 * 4)
+        want = _round256(want + rows * d * 4)
+        for mb in (4, 500):
+            got = lib.pa_decode_workspace_bytes(ctypes.byref(desc), B, hq, mb)
+            assert got == want, (hkv, hq, d, mb, got, want)
+        assert lib.pa_decode_shared_prefix_workspace_bytes(ctypes.byref(desc), B, hq, 500,
+                                                           64) >= want
+    # a group of 32 stays on the page stream: partials for 192 CTAs x 2
+    # slots plus 16 bytes of counters per sequence, so the batch adds only
+    # the counters
+    desc = _desc(nb=1000, bs=32, hkv=2, d=128)
+    one = lib.pa_decode_workspace_bytes(ctypes.byref(desc), 1, 64, 500)
+    many = lib.pa_decode_workspace_bytes(ctypes.byref(desc), 300, 64, 500)
+    assert one >= 192 * 2 * 64 * 128 * 4
+    assert 0 <= many - one <= _round256(300 * 16)
+
+
+def test_noalloc_refuses_what_its_scratch_cannot_hold(lib):
+    """pa_decode_noalloc uses the page-stream layout in its 16 MiB scratch and
+    refuses, before touching the device, sizes whose layout is larger."""
+    f = lib.pa_decode_noalloc
+    desc = _desc(nb=1000, bs=32, hkv=1, d=128)
+    # 128 query heads: the partials alone take 192 x 2 x 128 x 128 x 4 bytes
+    assert f(ctypes.byref(desc), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 128, 4096, 0.1,
+             None, None) == pa.PA_ERR_UNSUPPORTED
+    assert b"scratch" in lib.pa_last_error_message()
+    # 64 query heads fit, but not with a million sequences' counters
+    assert f(ctypes.byref(desc), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, 64, 4096, 0.1,
+             None, None) == pa.PA_ERR_UNSUPPORTED
+    assert b"scratch" in lib.pa_last_error_message()
