@@ -364,12 +364,12 @@ struct MmaConsumer {
     float4 v[KS];
 #pragma unroll
     for (int k = 0; k < KS; ++k) {
-      // round 1 (lanes g, g ^ 1): pairs (d, d + 1) of one head, at +0 and +8
+      // first exchange (lanes g, g ^ 1): pairs (d, d + 1) of one head, at +0 and +8
       const float s0 = __shfl_xor_sync(0xffffffffu, odd ? o[k][0] : o[k][1], 4);
       const float s2 = __shfl_xor_sync(0xffffffffu, odd ? o[k][2] : o[k][3], 4);
       const float lo0 = odd ? s0 : o[k][0], lo1 = odd ? o[k][1] : s0;
       const float hi0 = odd ? s2 : o[k][2], hi1 = odd ? o[k][3] : s2;
-      // round 2 (lanes g, g ^ 2): q < 2 keeps the +0 pairs, q >= 2 the +8 pairs
+      // second exchange (lanes g, g ^ 2): q < 2 keeps the +0 pairs, q >= 2 the +8 pairs
       const float r0 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi0 : lo0, 8);
       const float r1 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi1 : lo1, 8);
       v[k] = q < 2 ? make_float4(lo0 * inv, lo1 * inv, r0 * inv, r1 * inv)
