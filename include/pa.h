@@ -111,7 +111,7 @@ typedef struct pa_cache_desc {
 } pa_cache_desc;
 
 /* Version of this ABI (major * 10000 + minor * 100 + patch); 200 added the
- * scales of pa_cache_desc and PA_DTYPE_FP8_E4M3. */
+ * scales of pa_cache_desc and PA_DTYPE_FP8_E4M3, 300 added pa_prefill. */
 int32_t pa_version(void);
 
 /* Static text for a status code. */
@@ -261,6 +261,51 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
                                   int32_t batch, int32_t num_q_heads, int32_t max_blocks_per_seq,
                                   int32_t prefix_blocks, float scale, void *workspace,
                                   size_t workspace_bytes, int32_t *err_word, pa_stream_t stream);
+
+/*
+ * pa_prefill -- paged (chunked) prefill attention with the causal mask.
+ *
+ * [teaching] section "Where is the attention mask": in prefill every prompt
+ * token sees itself and the tokens before it; [route] section "decode
+ * attention and prefill attention are different": prefill processes a whole
+ * prompt, or a chunk of it, at once.  Sequence b brings
+ * n_b = query_start[b+1] - query_start[b] new tokens, rows query_start[b] ..
+ * query_start[b+1]-1 of q and out.  Their K/V rows must already be stored at
+ * their slots (pa_write_kv_cache); the history of sequence b holds
+ * context_lens[b] tokens including them, so new token j sits at position
+ * p = context_lens[b] - n_b + j and
+ *   out[row, hq, :] = sum_{t <= p} softmax_t(scale * q[row, hq, :] . K_t) V_t
+ * with K_t, V_t read through row b of block_tables (KV head hq / G).  With
+ * context_lens[b] == n_b this is a plain causal prompt prefill; with more it
+ * is a later chunk of a chunked prefill.
+ *
+ * Arrays: q, out [num_tokens, num_q_heads, head_dim] bf16; query_start
+ * [batch + 1] int32, non-decreasing, query_start[batch] <= num_tokens;
+ * block_tables [batch, max_blocks_per_seq]; context_lens [batch].
+ * max_query_len must be >= every n_b: the grid covers that many tokens per
+ * sequence.  Rows of out outside every sequence's range are not written.
+ *
+ * Data errors (flagged in *err_word): a query_start range outside
+ * [0, num_tokens] or decreasing sets PA_DEVERR_CONTEXT_LEN and writes none
+ * of that sequence's rows; n_b > context_lens[b], n_b > max_query_len or
+ * context_lens[b] > max_blocks_per_seq * block_size sets
+ * PA_DEVERR_CONTEXT_LEN and zeroes the rows of the sequence that the grid
+ * covers; a block id outside [0, num_blocks) among the sequence's first
+ * ceil(context_lens[b] / block_size) entries sets PA_DEVERR_BLOCK_ID and
+ * zeroes its rows.  A sequence with n_b == 0 is not read.
+ *
+ * Shapes: bf16, head_dim 64 or 128, query heads per KV head dividing 128,
+ * block_size 8..128, max_blocks_per_seq <= 4096 (else PA_ERR_UNSUPPORTED).
+ * batch, num_tokens or max_query_len == 0 is a no-op.  The work runs as
+ * tcgen05 tiles of 128 (query token, query head) rows x 128 KV tokens with
+ * the online softmax; no workspace.
+ */
+pa_status pa_prefill(const pa_cache_desc *cache, void *out, const void *q,
+                     const void *key_cache, const void *value_cache,
+                     const int32_t *block_tables, const int32_t *context_lens,
+                     const int32_t *query_start, int32_t batch, int32_t num_tokens,
+                     int32_t num_q_heads, int32_t max_blocks_per_seq, int32_t max_query_len,
+                     float scale, int32_t *err_word, pa_stream_t stream);
 
 /*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device

@@ -629,7 +629,7 @@ pa_status decode_streamed(const pa_cache_desc *cache, void *out, const void *q,
 
 extern "C" {
 
-int32_t pa_version(void) { return 200; }
+int32_t pa_version(void) { return 300; }
 
 const char *pa_status_string(int32_t status) {
   switch (status) {
@@ -845,6 +845,105 @@ pa_status pa_decode_shared_prefix(const pa_cache_desc *cache, void *out, const v
   pp.scale_log2 = scale_log2;
   const cudaError_t e = pa::launch_prefix(pp, cache->head_dim, st);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+pa_status pa_prefill(const pa_cache_desc *cache, void *out, const void *q,
+                     const void *key_cache, const void *value_cache,
+                     const int32_t *block_tables, const int32_t *context_lens,
+                     const int32_t *query_start, int32_t batch, int32_t num_tokens,
+                     int32_t num_q_heads, int32_t max_blocks_per_seq, int32_t max_query_len,
+                     float scale, int32_t *err_word, pa_stream_t stream) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (batch < 0 || batch > 65535)
+    return fail(PA_ERR_INVALID_ARG, "batch must be in [0, 65535]%s (got %lld)", "", batch);
+  if (num_tokens < 0)
+    return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0%s (got %lld)", "", num_tokens);
+  if (max_query_len < 0)
+    return fail(PA_ERR_INVALID_ARG, "max_query_len must be >= 0%s (got %lld)", "", max_query_len);
+  if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "num_q_heads must be a positive multiple of num_kv_heads%s (got %lld)", "",
+                num_q_heads);
+  if (max_blocks_per_seq < 0 || (int64_t)max_blocks_per_seq * cache->block_size > 0x7fffffffLL)
+    return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq * block_size must fit int32%s (%lld)", "",
+                max_blocks_per_seq);
+  if (!isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite%s");
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  const int32_t bs = cache->block_size;
+  if (cache->dtype != PA_DTYPE_BF16) return fail(PA_ERR_UNSUPPORTED, "prefill is bf16 only%s");
+  if (group > 128 || 128 % group != 0)
+    return fail(PA_ERR_UNSUPPORTED, "prefill needs 128 %% (query heads per KV head) == 0%s (%lld)",
+                "", group);
+  if (bs < 8 || bs > 128)
+    return fail(PA_ERR_UNSUPPORTED, "prefill needs block_size in [8, 128]%s (%lld)", "", bs);
+  if (max_blocks_per_seq > pa::kMaxPrefillBlocks)
+    return fail(PA_ERR_UNSUPPORTED, "prefill reads at most 4096 table entries per sequence%s (%lld)",
+                "", max_blocks_per_seq);
+  if (cache->num_kv_heads > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "more than 65535 KV heads%s (%lld)", "", cache->num_kv_heads);
+  const int64_t tiles = ((int64_t)max_query_len * group + 127) / 128;
+  if (tiles > 0x7fffffffLL)
+    return fail(PA_ERR_INVALID_ARG, "max_query_len too large%s (%lld)", "", max_query_len);
+  if (batch == 0 || num_tokens == 0 || max_query_len == 0) return PA_OK;
+  if ((s = check_ptr(q, "q")) != PA_OK) return s;
+  if ((s = check_ptr(out, "out")) != PA_OK) return s;
+  if ((s = check_ptr(key_cache, "key_cache")) != PA_OK) return s;
+  if ((s = check_ptr(value_cache, "value_cache")) != PA_OK) return s;
+  if (context_lens == nullptr) return fail(PA_ERR_INVALID_ARG, "context_lens is NULL%s");
+  if (query_start == nullptr) return fail(PA_ERR_INVALID_ARG, "query_start is NULL%s");
+  if (block_tables == nullptr) return fail(PA_ERR_INVALID_ARG, "block_tables is NULL%s");
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return fail(PA_ERR_CUDA, "cannot describe tensors for the tensor copies%s");
+  pa::PrefillParams pp{};
+  {
+    // q (head_dim, query head, token) with boxes of 64 x group x 128 / group
+    const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim, (cuuint64_t)num_q_heads,
+                                (cuuint64_t)num_tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)cache->head_dim * 2,
+                                   (cuuint64_t)num_q_heads * cache->head_dim * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(128 / group)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&pp.tmap_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return fail(PA_ERR_CUDA, "cannot describe q for the tensor copies%s");
+  }
+  {
+    // caches (head_dim, token row of the pool, KV head), boxes of 64 x bs x 1
+    const cuuint64_t dims[3] = {(cuuint64_t)cache->head_dim,
+                                (cuuint64_t)cache->num_blocks * (cuuint64_t)bs,
+                                (cuuint64_t)cache->num_kv_heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)cache->num_kv_heads * cache->head_dim * 2,
+                                   (cuuint64_t)cache->head_dim * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)bs, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    for (int which = 0; which < 2; ++which) {
+      if (fn(which ? &pp.tmap_v : &pp.tmap_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(which ? value_cache : key_cache), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return fail(PA_ERR_CUDA, "cannot describe the caches for the tensor copies%s");
+    }
+  }
+  pp.block_tables = block_tables;
+  pp.context_lens = context_lens;
+  pp.query_start = query_start;
+  pp.out = out;
+  pp.err_word = err_word;
+  pp.batch = batch;
+  pp.num_tokens = num_tokens;
+  pp.num_q_heads = num_q_heads;
+  pp.num_kv_heads = cache->num_kv_heads;
+  pp.group = group;
+  pp.block_size = bs;
+  pp.table_stride = max_blocks_per_seq;
+  pp.num_blocks = cache->num_blocks;
+  pp.tiles_per_seq = (int32_t)tiles;
+  pp.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = pa::launch_prefill(pp, cache->head_dim, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
   return PA_OK;
 }
 

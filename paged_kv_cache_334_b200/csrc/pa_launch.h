@@ -167,6 +167,25 @@ cudaError_t launch_suffix(const SuffixParams &p, int head_dim, cudaStream_t stre
 // pair's rows from its result or its partials, as bf16 `out` rows.
 cudaError_t launch_finish(const SuffixParams &p, void *out, int head_dim, cudaStream_t stream);
 
+// Arguments of the paged prefill kernel (prefill.cu).
+constexpr int kMaxPrefillBlocks = 4096;  // table entries per sequence (max_blocks_per_seq)
+struct PrefillParams {
+  CUtensorMap tmap_q;  // q (head_dim, query head, token), boxes of 64 x group x 128 / group
+  CUtensorMap tmap_k;  // caches as in PrefixParams
+  CUtensorMap tmap_v;
+  const int32_t *block_tables;  // [batch][table_stride]
+  const int32_t *context_lens;  // [batch]: history including the new tokens
+  const int32_t *query_start;   // [batch + 1]: sequence b's new tokens are q rows [qs[b], qs[b+1])
+  void *out;                    // [num_tokens][Hq][D] bf16
+  int32_t *err_word;
+  int32_t batch, num_tokens, num_q_heads, num_kv_heads, group, block_size, table_stride,
+      num_blocks;
+  int32_t tiles_per_seq;  // ceil(max_query_len * group / 128): grid x
+  float scale_log2;
+};
+size_t prefill_smem_bytes(int head_dim);
+cudaError_t launch_prefill(const PrefillParams &p, int head_dim, cudaStream_t stream);
+
 // Query heads handled together by one CTA for a GQA group of `group` heads.
 int decode_head_tile(int group);
 

@@ -43,7 +43,7 @@ EXPORTED_SYMBOLS = (
     "pa_version", "pa_status_string", "pa_last_error_message", "pa_write_kv_cache",
     "pa_decode_workspace_bytes", "pa_decode", "pa_decode_splitk", "pa_reduce",
     "pa_decode_noalloc", "pa_forward_decode", "pa_decode_shared_prefix",
-    "pa_decode_shared_prefix_workspace_bytes",
+    "pa_decode_shared_prefix_workspace_bytes", "pa_prefill",
 )
 
 # Size of the fixed device scratch array pa_decode_noalloc uses.
@@ -105,6 +105,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_shared_prefix.argtypes = [D, P, P, P, P, P, P, i32, i32, i32, i32, f32, P, sz,
                                             P, P]
     lib.pa_decode_shared_prefix.restype = ctypes.c_int
+    lib.pa_prefill.argtypes = [D, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P]
+    lib.pa_prefill.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -346,4 +348,33 @@ def pa_decode_noalloc(out, q, key_cache, value_cache, block_tables, context_lens
         _dev(block_tables, "block_tables", torch.int32),
         _dev(context_lens, "context_lens", torch.int32), B, Hq, MB, float(scale),
         _dev(err_word, "err_word", torch.int32), _stream(stream)))
+    return out
+
+
+def pa_prefill(out, q, key_cache, value_cache, block_tables, context_lens, query_start,
+               max_query_len: Optional[int] = None, scale: Optional[float] = None,
+               err_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Paged (chunked) prefill with the causal mask into `out` [T, Hq, D]:
+    sequence b's new tokens are rows query_start[b] .. query_start[b+1]-1 of
+    q, their K/V already stored, context_lens[b] counting them (see
+    include/pa.h).  max_query_len (>= every chunk's length) defaults to the
+    longest chunk, which reads query_start back to the host."""
+    lib = load()
+    desc = cache_desc(key_cache)
+    T, Hq, Dq = q.shape
+    B = context_lens.numel()
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if query_start.numel() != B + 1:
+        raise ValueError("query_start must hold batch + 1 entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dq)
+    if max_query_len is None:
+        max_query_len = int((query_start[1:] - query_start[:-1]).max().item()) if B else 0
+    _check(lib.pa_prefill(
+        ctypes.byref(desc), _dev(out, "out", key_cache.dtype), _dev(q, "q", key_cache.dtype),
+        _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache", key_cache.dtype),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32), B, T, Hq, MB, int(max_query_len),
+        float(scale), _dev(err_word, "err_word", torch.int32), _stream(stream)))
     return out

@@ -197,7 +197,7 @@ def test_fp8_argument_checks_need_no_device(lib):
                                  None) == pa.PA_ERR_UNSUPPORTED
     assert lib.pa_write_kv_cache(ctypes.byref(_fp8(ks=0.0)), FAKE, FAKE, FAKE, FAKE, FAKE, 2,
                                  None, None) == pa.PA_ERR_INVALID_ARG
-    assert lib.pa_version() == 200
+    assert lib.pa_version() == 300
 
 
 def _round256(x):
@@ -247,3 +247,34 @@ def test_noalloc_refuses_what_its_scratch_cannot_hold(lib):
     assert f(ctypes.byref(desc), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, 64, 4096, 0.1,
              None, None) == pa.PA_ERR_UNSUPPORTED
     assert b"scratch" in lib.pa_last_error_message()
+
+
+def test_prefill_argument_checks(lib):
+    """pa_prefill refuses, before touching the device, what its tensor-core
+    tiles cannot serve, and does nothing for empty work."""
+    f = lib.pa_prefill
+
+    def call(desc, *, out=FAKE, q=FAKE, qs=FAKE, B=2, T=64, Hq=32, MB=16, mql=32, scale=0.1):
+        return f(ctypes.byref(desc), out, q, FAKE, FAKE, FAKE, FAKE, qs, B, T, Hq, MB, mql,
+                 scale, None, None)
+
+    bf = _desc(nb=64, bs=16, hkv=8, d=128)
+    assert call(_desc(nb=64, bs=16, hkv=8, d=128, dtype=0)) == pa.PA_ERR_UNSUPPORTED  # fp32
+    assert b"bf16" in lib.pa_last_error_message()
+    assert call(_fp8()) == pa.PA_ERR_UNSUPPORTED
+    assert call(bf, Hq=24) == pa.PA_ERR_UNSUPPORTED        # 3 heads per KV head
+    assert call(_desc(nb=64, bs=256, hkv=1, d=128), Hq=256) == pa.PA_ERR_UNSUPPORTED
+    assert call(_desc(nb=64, bs=4, hkv=8, d=128)) == pa.PA_ERR_UNSUPPORTED
+    assert call(bf, MB=4097) == pa.PA_ERR_UNSUPPORTED       # table slice past shared memory
+    assert call(bf, Hq=20) == pa.PA_ERR_INVALID_ARG         # not a multiple of Hkv
+    assert call(bf, T=-1) == pa.PA_ERR_INVALID_ARG
+    assert call(bf, mql=-1) == pa.PA_ERR_INVALID_ARG
+    assert call(bf, B=70000) == pa.PA_ERR_INVALID_ARG
+    assert call(bf, scale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    assert call(bf, q=MISALIGNED) == pa.PA_ERR_INVALID_ARG
+    assert call(bf, out=None) == pa.PA_ERR_INVALID_ARG
+    assert call(bf, qs=None) == pa.PA_ERR_INVALID_ARG
+    # empty work: nothing to launch
+    assert call(bf, B=0) == pa.PA_OK
+    assert call(bf, T=0) == pa.PA_OK
+    assert call(bf, mql=0) == pa.PA_OK
