@@ -1,6 +1,7 @@
 /*
- * pa.h -- C ABI of libpa: single-query decode attention over a paged KV
- * cache on NVIDIA B200 (sm_100a).
+ * pa.h -- C ABI of libpa: attention over a paged KV cache on NVIDIA B200
+ * (sm_100a): single-query decode (pa_decode and its variants) and chunked
+ * prefill with the causal mask (pa_prefill).
  *
  * The operations follow three public pages:
  *   [route]    "From correct to faster: the PagedAttention optimisation
@@ -20,7 +21,8 @@
  *   call.
  * - Arrays are dense, row-major, exactly as written:
  *     key_cache, value_cache  [num_blocks, block_size, num_kv_heads, head_dim]
- *     q, out                  [batch, num_q_heads, head_dim]
+ *     q, out                  [batch, num_q_heads, head_dim] (pa_prefill:
+ *                             [num_tokens, num_q_heads, head_dim])
  *     k_new, v_new            [num_tokens, num_kv_heads, head_dim]
  *     block_tables            [batch, max_blocks_per_seq] int32
  *     context_lens            [batch] int32
