@@ -26,6 +26,12 @@ barrier and max/sum reductions of the timings (weak scaling).
 
 ``--impl reference`` times the fp64 CPU oracle itself as the reference arm
 (rank 0 only; other ranks exit at once).
+
+``--step prefill`` measures pa_prefill instead: the workload's sequences as
+whole prompts (or, with ``--chunk C``, the last C tokens of each context as
+a later chunk), all their K/V in the pool, one call per step, reported in
+TFLOP/s of causal attention (QK and PV of every visible position) against
+the measured bf16 tensor peak.
 """
 from __future__ import annotations
 
@@ -72,11 +78,16 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--step", choices=("fused", "separate", "prefix"), default="fused",
+    ap.add_argument("--step", choices=("fused", "separate", "prefix", "prefill"),
+                    default="fused",
                     help="fused: one pa_forward_decode call per step (cache write inside the "
                          "decode kernel); separate: pa_write_kv_cache then pa_decode; prefix: "
                          "pa_write_kv_cache then pa_decode_shared_prefix (workloads with a "
-                         "shared prefix)")
+                         "shared prefix); prefill: one pa_prefill call over the workload's "
+                         "sequences as whole prompts (bf16 workloads), reported in TFLOP/s")
+    ap.add_argument("--chunk", type=int, default=None,
+                    help="--step prefill: the last CHUNK tokens of each context are the "
+                         "chunk (a later chunk of a chunked prefill) instead of whole prompts")
     return ap.parse_args(argv)
 
 
@@ -606,8 +617,220 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# --step prefill: one pa_prefill call per step
+# ---------------------------------------------------------------------------
+
+PREFILL_METRIC = "paged prefill attention (causal) TFLOP/s and fraction of the B200 bf16 peak"
+
+
+def prefill_sample(pw, m: int):
+    """The oracle's share of a prefill step: sequence 0's last m chunk tokens
+    (the same positions, so the same rows of the result)."""
+    import dataclasses
+    base = pw.base
+    n0 = int(pw.chunk_lens[0])
+    m = max(1, min(m, n0))
+    b1 = dataclasses.replace(base, batch=1, q=base.q[:1].copy(),
+                             block_tables=base.block_tables[:1].copy(),
+                             context_lens=base.context_lens[:1].copy())
+    q = pw.q[n0 - m:n0].copy()
+    return wl.PrefillWorkload(base=b1, q=q, query_start=np.array([0, m], dtype=np.int32),
+                              chunk_lens=np.array([m], dtype=np.int32),
+                              description=f"sequence 0's last {m} of {n0} chunk tokens")
+
+
+def time_oracle_prefill(pw, target_seconds: float):
+    """Time the fp64 oracle's prefill on a sample growing by 4x until one
+    pass takes about a quarter of target_seconds, then repeat it to about
+    target_seconds."""
+    import oracle
+    oracle.build()
+
+    def one(s):
+        b = s.base
+        t0 = time.perf_counter()
+        oracle.prefill(s.q, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
+                       s.query_start, 1.0 / math.sqrt(b.head_dim))
+        return time.perf_counter() - t0
+
+    m = 4
+    sample = prefill_sample(pw, m)
+    t = one(sample)
+    while t < target_seconds / 4 and m < int(pw.chunk_lens[0]):
+        m *= 4
+        sample = prefill_sample(pw, m)
+        t = one(sample)
+    total, reps = t, 1
+    while total < target_seconds:
+        total += one(sample)
+        reps += 1
+    # the oracle's prefill loops over rows on one thread
+    return total / reps, sample, 1, f"{sample.description}, {reps} repetition(s)"
+
+
+def run_prefill(args):
+    import torch
+    from paged_kv_cache_334_b200 import pa
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, local)
+    pa.load()
+
+    w = wl.make_workload(args.workload, seed=rank_seed(args.seed, rank),
+                         block_size=args.block_size)
+    pw = wl.prefill_workload(w, chunk=args.chunk, seed=rank_seed(args.seed, rank))
+    base = pw.base
+
+    def dev_t(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).to(dev)
+
+    q, kc, vc = dev_t(pw.q), dev_t(base.key_cache), dev_t(base.value_cache)
+    bt, cl, qs = dev_t(base.block_tables), dev_t(base.context_lens), dev_t(pw.query_start)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(base.head_dim)
+    mql = pw.max_query_len
+    stream = torch.cuda.current_stream(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    flush_f32 = flush_buf.view(torch.float32)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush_buf.zero_()
+        torch.amax(flush_f32, out=flush_sink)
+
+    def call():
+        pa.pa_prefill(out, q, kc, vc, bt, cl, qs, max_query_len=mql, scale=scale,
+                      err_word=err, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush_l2()
+        call()
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())} during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark("t0")
+    for k in range(K):
+        flush_l2()
+        ev[k][0].record(stream)
+        call()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark("t1")
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    t_call = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+
+    e2e = None
+    if not args.no_e2e:
+        host = [(q, q.cpu().pin_memory()), (bt, bt.cpu().pin_memory()),
+                (cl, cl.cpu().pin_memory()), (qs, qs.cpu().pin_memory())]
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(h.numel() * h.element_size() for _, h in host)
+        d2h = out_host.numel() * out_host.element_size()
+        Ke = max(3, min(K, 200))
+        eve = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+        for k in range(Ke + 3):
+            flush_l2()
+            if k >= 3:
+                eve[k - 3][0].record(stream)
+            for dst, src in host:
+                dst.copy_(src, non_blocking=True)
+            call()
+            out_host.copy_(out, non_blocking=True)
+            if k >= 3:
+                eve[k - 3][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e = (statistics.mean(e[0].elapsed_time(e[1]) for e in eve), h2d, d2h)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+
+    flops = wl.prefill_flops(pw)
+    t_max = reduce_scalar(t_call, "max", dist, dev)
+    flops_all = reduce_scalar(flops, "sum", dist, dev)
+    tokens_all = reduce_scalar(pw.num_tokens, "sum", dist, dev)
+    e2e_line = None
+    if e2e is not None:
+        t_e2e_max = reduce_scalar(e2e[0], "max", dist, dev)
+        e2e_line = {"value": flops_all / (t_e2e_max * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(e2e[1]), "d2h_bytes_per_step": int(e2e[2]),
+                    "ms_per_step": t_e2e_max}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_step, sample, cores, desc = time_oracle_prefill(pw, args.cpu_seconds)
+        cpu = {"value": wl.prefill_flops(sample) / per_step / 1e12, "unit": "TFLOP/s",
+               "cores": cores, "kind": "oracle", "sample": desc,
+               "ms_per_step": per_step * 1e3}
+    tpeak, tpeak_src = tensor_peak()
+    hpeak, _ = hbm_peak()
+    achieved = flops / (t_call * 1e-3) / 1e12
+    nbytes = wl.prefill_roofline_bytes(pw)
+    line = {
+        "metric": PREFILL_METRIC,
+        "value": flops_all / (t_max * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": t_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{args.workload} as prefill: {pw.description}",
+            "batch": base.batch, "num_q_heads": base.num_q_heads,
+            "num_kv_heads": base.num_kv_heads, "head_dim": base.head_dim,
+            "block_size": base.block_size, "query_tokens": pw.num_tokens,
+            "max_query_len": mql, "context_tokens": int(base.context_lens.sum()),
+            "seed": args.seed, "step": "pa_prefill (causal, K/V through the block table)",
+            "l2": "flushed before every timed step (zero-fill then read of 2x L2, outside "
+                  "the events)",
+            "parallelism": f"replicas: one independent batch per GPU x{args.gpus}",
+        },
+        "query_tokens_per_s": tokens_all / (t_max * 1e-3),
+        "roofline": {
+            "bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s",
+            "frac": achieved / tpeak, "traffic": None, "kernel": "pa_prefill",
+            "flops_per_launch": flops, "launch_us": t_call * 1e3, "peak_source": tpeak_src,
+            "algorithmic_bytes_per_launch": nbytes,
+            "hbm_frac": nbytes / (t_call * 1e-3) / 1e9 / hpeak,
+        },
+        "e2e": e2e_line,
+        "cpu_baseline": cpu,
+        "gpu_launches": K,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.step == "prefill":
+        if args.impl == "reference":
+            raise SystemExit("--step prefill has no reference arm; its cpu_baseline is the "
+                             "oracle")
+        return run_prefill(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

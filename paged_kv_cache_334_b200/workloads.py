@@ -365,3 +365,77 @@ def roofline_bytes(w: Workload, include_write: bool = True) -> int:
         extra = (w.k_new.nbytes + w.v_new.nbytes + 2 * n_new * row +
                  w.slot_mapping.nbytes)
     return int(kv + qo + meta + extra)
+
+
+# ---------------------------------------------------------------------------
+# paged (chunked) prefill inputs
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PrefillWorkload:
+    """Prefill inputs over a decode workload's pool: sequence b's chunk is
+    rows query_start[b] .. query_start[b+1]-1 of q, the last chunk_lens[b]
+    tokens of its context_lens[b]-token history, every token of which is
+    stored in the pool of `base`."""
+    base: Workload          # pool, tables and lengths; no pending new tokens
+    q: np.ndarray           # [T, Hq, D] bf16 storage
+    query_start: np.ndarray  # [B + 1] int32
+    chunk_lens: np.ndarray   # [B] int32
+    description: str = ""
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+    @property
+    def max_query_len(self) -> int:
+        return int(self.chunk_lens.max()) if self.chunk_lens.size else 0
+
+
+def prefill_workload(w: Workload, chunk: Optional[int] = None, seed: int = 0) -> PrefillWorkload:
+    """Prefill inputs over w's pool, tables and lengths: whole prompts (chunk
+    None: each context is one prompt, as the teaching page's prefill stores a
+    prompt's K/V and attends over it causally) or, with chunk = c, the last
+    min(c, ctx) tokens of each context as the chunk of a chunked prefill.
+    The newest tokens w held back for its decode step are put into their
+    slots, so every context token is stored; q is drawn afresh (N(0, 1),
+    rounded to bf16)."""
+    if w.dtype != DTYPE_BF16:
+        raise ValueError(f"prefill inputs are bf16, not {w.dtype}")
+    kc, vc = w.key_cache.copy(), w.value_cache.copy()
+    if w.slot_mapping is not None:
+        bs = w.block_size
+        for i, s in enumerate(w.slot_mapping.tolist()):
+            kc[s // bs, s % bs] = w.k_new[i]
+            vc[s // bs, s % bs] = w.v_new[i]
+    ctx = w.context_lens.astype(np.int64)
+    n = ctx if chunk is None else np.minimum(ctx, int(chunk))
+    qs = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    rng = np.random.Generator(np.random.PCG64(seed + 0x5EED))
+    q = _normal_storage(rng, (int(qs[-1]), w.num_q_heads, w.head_dim), DTYPE_BF16)
+    base = dataclasses.replace(w, key_cache=kc, value_cache=vc, k_new=None, v_new=None,
+                               slot_mapping=None)
+    what = "whole prompts" if chunk is None else f"last <= {chunk} tokens of each context"
+    return PrefillWorkload(base=base, q=q, query_start=qs, chunk_lens=n.astype(np.int32),
+                           description=f"{w.name} pool, {what}, {int(qs[-1])} query tokens")
+
+
+def prefill_flops(pw: PrefillWorkload) -> float:
+    """QK and PV of every (chunk token, query head, visible position): chunk
+    token j of a chunk of n at the end of a ctx-token history sees ctx - n +
+    j + 1 positions, 2 * 2 * head_dim flops each."""
+    w = pw.base
+    ctx = w.context_lens.astype(np.float64)
+    n = pw.chunk_lens.astype(np.float64)
+    pairs = float(np.sum(n * (ctx - n) + n * (n + 1) / 2))
+    return 4.0 * w.head_dim * w.num_q_heads * pairs
+
+
+def prefill_roofline_bytes(pw: PrefillWorkload) -> int:
+    """Algorithmic HBM bytes of one prefill call: unique K/V bytes of every
+    context token, tables, lengths, query_start, and q and out of the chunk
+    tokens (read and written once)."""
+    w = pw.base
+    decode_qo = 2 * w.batch * w.num_q_heads * w.head_dim * w.act_bytes
+    qo = 2 * pw.num_tokens * w.num_q_heads * w.head_dim * w.act_bytes
+    return int(roofline_bytes(w, include_write=False) - decode_qo + qo + pw.query_start.nbytes)

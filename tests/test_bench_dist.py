@@ -60,3 +60,34 @@ def test_rank_zero_alone_runs_the_reference_arm(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
     assert capsys.readouterr().out == ""     # non-zero ranks exit without work
+
+
+def test_prefill_step_arguments_and_oracle_sample():
+    """--step prefill: its arguments, the refusal of a reference arm, and the
+    oracle's sample (sequence 0's last m chunk rows at their own positions)."""
+    import pytest
+
+    import bench
+    from paged_kv_cache_334_b200 import workloads as wl
+
+    a = bench.parse_args(["--step", "prefill", "--chunk", "64"])
+    assert a.step == "prefill" and a.chunk == 64 and a.workload == "gqa_bf16"
+    with pytest.raises(SystemExit):
+        bench.main(["--step", "prefill", "--impl", "reference"])
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=3, num_q_heads=8, num_kv_heads=2,
+                           head_dim=64, block_size=4, context_lens=[9, 5, 3], seed=1,
+                           new_tokens=True)
+    pw = wl.prefill_workload(w, chunk=6, seed=1)
+    s = bench.prefill_sample(pw, 4)
+    assert s.base.batch == 1 and s.query_start.tolist() == [0, 4]
+    assert int(s.base.context_lens[0]) == 9 and s.chunk_lens.tolist() == [4]
+    assert np.array_equal(s.q, pw.q[2:6])  # chunk rows 2..5 of sequence 0: positions 5..8
+    assert bench.prefill_sample(pw, 100).chunk_lens.tolist() == [6]
+    # the sample's rows are the full call's rows at those positions
+    import oracle
+    b = pw.base
+    full, _ = oracle.prefill(pw.q, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
+                             pw.query_start)
+    part, _ = oracle.prefill(s.q, s.base.key_cache, s.base.value_cache, s.base.block_tables,
+                             s.base.context_lens, s.query_start)
+    assert np.isfinite(full).all() and np.array_equal(part, full[2:6])

@@ -143,3 +143,49 @@ def test_gqa_fp8_pages():
     qo = 2 * w.batch * w.num_q_heads * w.head_dim * 2
     meta = w.block_tables.size * 4 + w.context_lens.size * 4
     assert kv_fp8 - qo - meta == (kv_bf16 - qo - meta) // 2
+
+
+def test_prefill_inputs_store_every_context_token():
+    """Whole prompts over gqa_bf16's pool: the held-back newest tokens are
+    back in their slots, every other slot past a context is still NaN."""
+    w = wl.make_workload("gqa_bf16", seed=1, batch=6)
+    pw = wl.prefill_workload(w, seed=1)
+    base = pw.base
+    assert base.slot_mapping is None and base.k_new is None
+    assert pw.chunk_lens.tolist() == w.context_lens.tolist()
+    assert pw.query_start[0] == 0 and np.all(np.diff(pw.query_start) == pw.chunk_lens)
+    assert pw.q.shape == (pw.num_tokens, w.num_q_heads, w.head_dim) and pw.q.dtype == np.uint16
+    live = np.zeros((base.num_blocks, base.block_size), dtype=bool)
+    for b in range(base.batch):
+        for t in range(int(base.context_lens[b])):
+            live[base.block_tables[b, t // base.block_size], t % base.block_size] = True
+    nan = np.uint16(0x7FC0)
+    assert not np.any(base.key_cache[live] == nan) and not np.any(base.value_cache[live] == nan)
+    assert np.all(base.key_cache[~live] == nan) and np.all(base.value_cache[~live] == nan)
+    # the slots the decode step held back now hold exactly its new rows
+    for i, s in enumerate(w.slot_mapping.tolist()):
+        pb, off = divmod(s, w.block_size)
+        assert np.array_equal(base.key_cache[pb, off], w.k_new[i])
+        assert np.array_equal(base.value_cache[pb, off], w.v_new[i])
+    # the decode workload itself is untouched
+    assert np.all(w.key_cache[w.slot_mapping // w.block_size, w.slot_mapping % w.block_size] == nan)
+
+
+def test_prefill_flops_and_bytes_by_brute_force():
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=4, num_q_heads=8, num_kv_heads=2,
+                           head_dim=64, block_size=4, context_lens=[1, 7, 12, 0], seed=3,
+                           new_tokens=True)
+    for chunk in (None, 5):
+        pw = wl.prefill_workload(w, chunk=chunk, seed=2)
+        pairs = 0
+        for b in range(w.batch):
+            ctx, n = int(w.context_lens[b]), int(pw.chunk_lens[b])
+            assert n == (ctx if chunk is None else min(ctx, chunk))
+            for j in range(n):
+                pairs += sum(1 for t in range(ctx) if t <= ctx - n + j)
+        assert wl.prefill_flops(pw) == 4 * 64 * 8 * pairs
+        kv = 2 * int(w.context_lens.sum()) * 2 * 64 * 2  # no page shared
+        qo = 2 * pw.num_tokens * 8 * 64 * 2
+        meta = w.block_tables.size * 4 + w.context_lens.size * 4 + pw.query_start.nbytes
+        assert wl.prefill_roofline_bytes(pw) == kv + qo + meta
+    assert wl.prefill_workload(w, chunk=5).max_query_len == 5
