@@ -426,6 +426,34 @@ def test_e4m3_encode_is_the_nearest_code():
     assert oracle.e4m3_encode(np.array([np.nan]))[0] == 0x7F
 
 
+def test_decode_fp8_matches_sdpa_on_torch_float8_values():
+    """decode over FP8 pages == torch's float64 SDPA on K/V that torch's own
+    float8_e4m3fn conversion decodes, times the per-tensor scales, gathered
+    here by plain indexing through the table (pins the dequantisation, the
+    scales' roles and the bf16 query path of decode_fp8)."""
+    lens = [1, 6, 11]
+    w = wl.custom_workload(dtype=wl.DTYPE_FP8, batch=3, num_q_heads=8, num_kv_heads=2,
+                           head_dim=32, block_size=4, context_lens=lens, seed=9,
+                           k_scale=0.25, v_scale=0.5)
+    out, fl = oracle.decode_fp8(w.q, w.key_cache, w.value_cache, w.k_scale, w.v_scale,
+                                w.block_tables, w.context_lens)
+    assert not fl.any()
+    as_f8 = lambda a: torch.from_numpy(a).view(torch.float8_e4m3fn).to(torch.float64)
+    for b, n in enumerate(lens):
+        rows = [(w.block_tables[b, t // 4], t % 4) for t in range(n)]
+        K = torch.stack([as_f8(w.key_cache[pb, off]) for pb, off in rows]) * 0.25
+        V = torch.stack([as_f8(w.value_cache[pb, off]) for pb, off in rows]) * 0.5
+        qb = torch.from_numpy(w.q[b].copy()).view(torch.bfloat16).to(torch.float64)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qb.reshape(1, 8, 1, 32), K.permute(1, 0, 2)[None], V.permute(1, 0, 2)[None],
+            scale=1.0 / math.sqrt(32), enable_gqa=True).reshape(8, 32).numpy()
+        np.testing.assert_allclose(out[b], ref, rtol=0, atol=1e-12)
+    # swapping the scales changes the result: each scale belongs to its tensor
+    swapped, _ = oracle.decode_fp8(w.q, w.key_cache, w.value_cache, w.v_scale, w.k_scale,
+                                   w.block_tables, w.context_lens)
+    assert np.abs(swapped[1:] - out[1:]).max() > 1e-3
+
+
 def test_write_kv_cache_fp8_worked_example():
     """Two tokens into a 2-block pool of 2-token pages, 1 KV head, head_dim 4:
     bf16 1.0, -3.0, 0.25, 1000.0 divided by k_scale 0.5 are 2, -6, 0.5 and
