@@ -313,8 +313,41 @@ def time_oracle(w, target_seconds: float, max_reps: int = 1000):
         total += _oracle_step(sample)
         reps += 1
     per_step = total / reps
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return per_step, sample, cores, f"{desc}, {reps} repetition(s)"
+    return per_step, sample, oracle.max_threads(), f"{desc}, {reps} repetition(s)"
+
+
+def cpu_baseline(w, cpu_seconds: float) -> dict:
+    """The oracle timed on the host cores (as many threads as its OpenMP
+    loops get) on a bounded sample of the batch, and on one thread on the
+    first 1/threads of that sample; GB/s on each sample's algorithmic
+    bytes."""
+    import oracle
+    per_step, sample, threads, desc = time_oracle(w, cpu_seconds)
+    line = {"value": wl.roofline_bytes(sample) / per_step / 1e9, "unit": "GB/s",
+            "cores": threads, "kind": "oracle", "sample": desc,
+            "ms_per_step": per_step * 1e3}
+    nb1 = max(1, sample.batch // max(1, threads))
+    one = _prefix(sample, nb1) if nb1 < sample.batch else sample
+    oracle.set_num_threads(1)
+    try:
+        total, reps = _oracle_step(one), 1
+        while total < cpu_seconds / 2 and reps < 1000:
+            total += _oracle_step(one)
+            reps += 1
+    finally:
+        oracle.set_num_threads(threads)
+    line["single_thread"] = {
+        "value": wl.roofline_bytes(one) / (total / reps) / 1e9, "unit": "GB/s", "cores": 1,
+        "sample": f"first {nb1} of the {sample.batch} sequences above, {reps} repetition(s)",
+        "ms_per_step": total / reps * 1e3}
+    return line
+
+
+def timing_stats(ms) -> dict:
+    """Mean, median, minimum and maximum of per-step times (ms)."""
+    ms = list(ms)
+    return {"mean": statistics.mean(ms), "median": statistics.median(ms), "min": min(ms),
+            "max": max(ms)}
 
 
 def _oracle_step(w) -> float:
@@ -556,10 +589,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_step, sample, cores, desc = time_oracle(w, args.cpu_seconds)
-        cpu = {"value": wl.roofline_bytes(sample) / per_step / 1e9, "unit": "GB/s",
-               "cores": cores, "kind": "oracle", "sample": desc,
-               "ms_per_step": per_step * 1e3}
+        cpu = cpu_baseline(w, args.cpu_seconds)
 
     peak, peak_src = hbm_peak()
     achieved = dec_bytes / (t_dec * 1e-3) / 1e9
@@ -586,6 +616,7 @@ def run_ours(args):
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": t_step_max,
+        "step_ms": timing_stats(step_ms),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -787,6 +818,7 @@ def run_prefill(args):
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": t_max,
+        "step_ms": timing_stats(e[0].elapsed_time(e[1]) for e in ev),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,

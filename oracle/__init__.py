@@ -47,6 +47,10 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         P = ctypes.c_void_p
         i32, i64, dbl = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        lib.orc_set_num_threads.argtypes = [ctypes.c_int]
+        lib.orc_set_num_threads.restype = None
+        lib.orc_max_threads.argtypes = []
+        lib.orc_max_threads.restype = ctypes.c_int
         lib.orc_map_token.argtypes = [P, i32, i32, i32, i64, P, P]
         lib.orc_map_token.restype = ctypes.c_int
         lib.orc_widen.argtypes = [P, ctypes.c_int, i64, P]
@@ -93,6 +97,16 @@ def _dtype_code(a: np.ndarray) -> int:
         return 3
     raise TypeError("storage dtype must be float32, uint16 (bf16 bits), uint8 (E4M3 codes) "
                     f"or float64, got {a.dtype}")
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops from now on (timing runs)."""
+    _load().orc_set_num_threads(int(n))
+
+
+def max_threads() -> int:
+    """Threads the oracle's OpenMP loops use."""
+    return int(_load().orc_max_threads())
 
 
 def e4m3_value(codes: np.ndarray) -> np.ndarray:

@@ -505,3 +505,25 @@ int orc_write_kv_cache(void *key_cache, void *value_cache, const void *k_new,
   }
   return flags;
 }
+
+/* Threads of the OpenMP loops (query heads of a sequence, partitions):
+ * set for timing runs, read back to report what a run used.  Without OpenMP
+ * everything runs on one thread. */
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+int orc_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -91,3 +91,22 @@ def test_prefill_step_arguments_and_oracle_sample():
     part, _ = oracle.prefill(s.q, s.base.key_cache, s.base.value_cache, s.base.block_tables,
                              s.base.context_lens, s.query_start)
     assert np.isfinite(full).all() and np.array_equal(part, full[2:6])
+
+
+def test_cpu_baseline_reports_threads_and_a_single_thread_run():
+    """The oracle baseline states the threads its OpenMP loops used, adds a
+    one-thread run on a smaller sample, and leaves the thread count as it
+    was; the step statistics are mean / median / min / max."""
+    import bench
+    import oracle
+    from paged_kv_cache_334_b200 import workloads as wl
+
+    w = wl.make_workload("gqa_bf16", seed=0, batch=3)
+    before = oracle.max_threads()
+    line = bench.cpu_baseline(w, 0.2)
+    assert oracle.max_threads() == before
+    assert line["cores"] == before and line["kind"] == "oracle" and line["value"] > 0
+    st = line["single_thread"]
+    assert st["cores"] == 1 and st["value"] > 0 and st["ms_per_step"] > 0
+    s = bench.timing_stats([3.0, 1.0, 2.0, 10.0])
+    assert s == {"mean": 4.0, "median": 2.5, "min": 1.0, "max": 10.0}
