@@ -343,6 +343,32 @@ def cpu_baseline(w, cpu_seconds: float) -> dict:
     return line
 
 
+SM_COUNT = 148
+EX2_PER_SM_CLK = 16  # fp32 ex2 results per SM per clock (multi-function unit, nominal)
+
+
+def ceilings(w, flops: float, nbytes: float, launch_us: float, sm_mhz: float) -> dict:
+    """Lower bounds on one call's time from its three candidate limits --
+    HBM bytes at the measured copy bandwidth, flops at the measured bf16
+    peak, and one ex2 per (visible token, query head) score at the
+    multi-function unit's nominal rate at the sampled SM clock -- and the
+    call's time as a multiple of each."""
+    hbm, _ = hbm_peak()
+    tensor, _ = tensor_peak()
+    exps = float(w.context_lens.sum()) * w.num_q_heads
+    ex2_per_s = SM_COUNT * EX2_PER_SM_CLK * sm_mhz * 1e6
+    out = {"hbm_us": nbytes / (hbm * 1e9) * 1e6,
+           "tensor_us": flops / (tensor * 1e12) * 1e6,
+           "ex2_us": exps / ex2_per_s * 1e6,
+           "ex2_per_launch": exps, "ex2_peak_per_s": ex2_per_s,
+           "ex2_peak": f"{SM_COUNT} SMs x {EX2_PER_SM_CLK} ex2/clock x {sm_mhz:.0f} MHz "
+                       "(nominal unit count, sampled clock)",
+           "launch_us": launch_us}
+    for k in ("hbm", "tensor", "ex2"):
+        out[k + "_frac"] = out[k + "_us"] / launch_us
+    return out
+
+
 def timing_stats(ms) -> dict:
     """Mean, median, minimum and maximum of per-step times (ms)."""
     ms = list(ms)
@@ -607,6 +633,8 @@ def run_ours(args):
                        "pa_forward_decode" if fused else "pa_decode"),
             "flops_per_launch": attention_flops(w), "launch_us": t_dec * 1e3,
             "peak_source": tpeak_src, "hbm_gbs": achieved, "hbm_frac": achieved / peak,
+            "ceilings": ceilings(w, attention_flops(w), dec_bytes, t_dec * 1e3,
+                                 (clk or {}).get("sm_mhz") or 1965.0),
         }
     line = {
         "metric": METRIC,

@@ -110,3 +110,24 @@ def test_cpu_baseline_reports_threads_and_a_single_thread_run():
     assert st["cores"] == 1 and st["value"] > 0 and st["ms_per_step"] > 0
     s = bench.timing_stats([3.0, 1.0, 2.0, 10.0])
     assert s == {"mean": 4.0, "median": 2.5, "min": 1.0, "max": 10.0}
+
+
+def test_ceilings_of_a_tensor_path_call():
+    """The three lower bounds of one call (HBM bytes, tensor flops, one ex2
+    per score) and the call's time as a fraction of each."""
+    import bench
+    from paged_kv_cache_334_b200 import workloads as wl
+
+    w = wl.make_workload("mqa_prefix_bf16", seed=0, batch=4)
+    flops = bench.attention_flops(w)
+    nbytes = wl.roofline_bytes(w, include_write=False)
+    c = bench.ceilings(w, flops, nbytes, 50.0, 1965.0)
+    exps = float(w.context_lens.sum()) * 64
+    assert c["ex2_per_launch"] == exps
+    assert abs(c["ex2_us"] - exps / (148 * 16 * 1965e6) * 1e6) < 1e-9
+    hbm, _ = bench.hbm_peak()
+    tp, _ = bench.tensor_peak()
+    assert abs(c["hbm_us"] - nbytes / hbm / 1e3) < 1e-9
+    assert abs(c["tensor_us"] - flops / tp / 1e6) < 1e-9
+    for k in ("hbm", "tensor", "ex2"):
+        assert abs(c[k + "_frac"] - c[k + "_us"] / 50.0) < 1e-12
