@@ -369,6 +369,36 @@ def ceilings(w, flops: float, nbytes: float, launch_us: float, sm_mhz: float) ->
     return out
 
 
+def parity_sample(w, out_rows: np.ndarray, nb: int) -> dict:
+    """Max / mean absolute difference between the timed call's output rows of
+    the first nb sequences (out_rows, float64) and the oracle's write then
+    decode of those sequences, with the tolerance of the workload's dtype.
+    The write is idempotent, so the workload's host pool may already hold
+    it."""
+    import oracle
+    nb = max(1, min(nb, w.batch))
+    s = _prefix(w, nb)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    kc, vc = s.key_cache, s.value_cache
+    if w.dtype == wl.DTYPE_FP8:
+        if s.slot_mapping is not None:
+            oracle.write_kv_cache_fp8(kc, vc, s.k_new, s.v_new, s.slot_mapping, w.k_scale,
+                                      w.v_scale)
+        ref, flags = oracle.decode_fp8(s.q, kc, vc, w.k_scale, w.v_scale, s.block_tables,
+                                       s.context_lens, scale)
+    else:
+        if s.slot_mapping is not None:
+            oracle.write_kv_cache(kc, vc, s.k_new, s.v_new, s.slot_mapping)
+        ref, flags = oracle.decode(s.q, kc, vc, s.block_tables, s.context_lens, scale)
+    err = np.abs(np.asarray(out_rows[:nb], dtype=np.float64) - ref)
+    tol_max, tol_mean = (1e-5, None) if w.dtype == wl.DTYPE_F32 else (2e-2, 1e-2)
+    finite = bool(np.isfinite(err).all())
+    ok = finite and not flags.any() and err.max() <= tol_max and (
+        tol_mean is None or err.mean() <= tol_mean)
+    return {"max_abs": float(err.max()), "mean_abs": float(err.mean()), "sequences": nb,
+            "tolerance": {"max_abs": tol_max, "mean_abs": tol_mean}, "within": bool(ok)}
+
+
 def timing_stats(ms) -> dict:
     """Mean, median, minimum and maximum of per-step times (ms)."""
     ms = list(ms)
@@ -613,9 +643,11 @@ def run_ours(args):
                     "h2d_bytes_per_step": int(e2e[1]), "d2h_bytes_per_step": int(e2e[2]),
                     "ms_per_step": t_e2e_max}
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
+        # the timed call's output rows of the first sequences against the oracle
+        parity = parity_sample(w, out[:8].double().cpu().numpy(), 8)
 
     peak, peak_src = hbm_peak()
     achieved = dec_bytes / (t_dec * 1e-3) / 1e9
@@ -665,6 +697,7 @@ def run_ours(args):
         },
         "e2e": e2e_line,
         "cpu_baseline": cpu,
+        "parity": parity,
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }

@@ -131,3 +131,33 @@ def test_ceilings_of_a_tensor_path_call():
     assert abs(c["tensor_us"] - flops / tp / 1e6) < 1e-9
     for k in ("hbm", "tensor", "ex2"):
         assert abs(c[k + "_frac"] - c[k + "_us"] / 50.0) < 1e-12
+
+
+def test_parity_sample_against_the_oracle():
+    """bench's parity record: zero against the oracle's own rows, the size
+    of a planted error otherwise, and the dtype's tolerance."""
+    import math
+
+    import bench
+    import oracle
+    from paged_kv_cache_334_b200 import workloads as wl
+
+    for name in ("gqa_bf16", "gqa_fp8"):
+        w = wl.make_workload(name, seed=2, batch=3)
+        kc, vc = w.key_cache.copy(), w.value_cache.copy()
+        if name == "gqa_fp8":
+            oracle.write_kv_cache_fp8(kc, vc, w.k_new, w.v_new, w.slot_mapping, w.k_scale,
+                                      w.v_scale)
+            ref, _ = oracle.decode_fp8(w.q, kc, vc, w.k_scale, w.v_scale, w.block_tables,
+                                       w.context_lens, 1.0 / math.sqrt(w.head_dim))
+        else:
+            oracle.write_kv_cache(kc, vc, w.k_new, w.v_new, w.slot_mapping)
+            ref, _ = oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens,
+                                   1.0 / math.sqrt(w.head_dim))
+        rec = bench.parity_sample(w, ref, 2)
+        assert rec["max_abs"] == 0.0 and rec["within"] and rec["sequences"] == 2
+        bad = ref.copy()
+        bad[1, 3, 5] += 0.05
+        rec = bench.parity_sample(w, bad, 2)
+        assert abs(rec["max_abs"] - 0.05) < 1e-12 and not rec["within"]
+        assert rec["tolerance"] == {"max_abs": 2e-2, "mean_abs": 1e-2}
