@@ -761,6 +761,22 @@ def time_oracle_prefill(pw, target_seconds: float):
     return total / reps, sample, 1, f"{sample.description}, {reps} repetition(s)"
 
 
+def prefill_parity(pw, sample, out_rows: np.ndarray) -> dict:
+    """Max / mean absolute difference between the call's output rows of the
+    oracle's sample (sequence 0's last m chunk rows; out_rows holds the
+    whole call's rows as float64) and the oracle's prefill of that sample."""
+    import oracle
+    b = sample.base
+    ref, flags = oracle.prefill(sample.q, b.key_cache, b.value_cache, b.block_tables,
+                                b.context_lens, sample.query_start, 1.0 / math.sqrt(b.head_dim))
+    n0, m = int(pw.chunk_lens[0]), int(sample.chunk_lens[0])
+    err = np.abs(np.asarray(out_rows[n0 - m:n0], dtype=np.float64) - ref)
+    ok = bool(np.isfinite(err).all()) and not flags.any() and err.max() <= 2e-2 and \
+        err.mean() <= 1e-2
+    return {"max_abs": float(err.max()), "mean_abs": float(err.mean()), "rows": m,
+            "tolerance": {"max_abs": 2e-2, "mean_abs": 1e-2}, "within": bool(ok)}
+
+
 def run_prefill(args):
     import torch
     from paged_kv_cache_334_b200 import pa
@@ -861,12 +877,13 @@ def run_prefill(args):
         e2e_line = {"value": flops_all / (t_e2e_max * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(e2e[1]), "d2h_bytes_per_step": int(e2e[2]),
                     "ms_per_step": t_e2e_max}
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         per_step, sample, cores, desc = time_oracle_prefill(pw, args.cpu_seconds)
         cpu = {"value": wl.prefill_flops(sample) / per_step / 1e12, "unit": "TFLOP/s",
                "cores": cores, "kind": "oracle", "sample": desc,
                "ms_per_step": per_step * 1e3}
+        parity = prefill_parity(pw, sample, out[:int(pw.chunk_lens[0])].double().cpu().numpy())
     tpeak, tpeak_src = tensor_peak()
     hpeak, _ = hbm_peak()
     achieved = flops / (t_call * 1e-3) / 1e12
@@ -906,6 +923,7 @@ def run_prefill(args):
         },
         "e2e": e2e_line,
         "cpu_baseline": cpu,
+        "parity": parity,
         "gpu_launches": K,
         "clocks": clk,
     }

@@ -161,3 +161,26 @@ def test_parity_sample_against_the_oracle():
         rec = bench.parity_sample(w, bad, 2)
         assert abs(rec["max_abs"] - 0.05) < 1e-12 and not rec["within"]
         assert rec["tolerance"] == {"max_abs": 2e-2, "mean_abs": 1e-2}
+
+
+def test_prefill_parity_record():
+    import bench
+    import oracle
+    from paged_kv_cache_334_b200 import workloads as wl
+
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=2, num_q_heads=8, num_kv_heads=2,
+                           head_dim=64, block_size=4, context_lens=[9, 5], seed=4,
+                           new_tokens=True)
+    pw = wl.prefill_workload(w, seed=4)
+    b = pw.base
+    full, _ = oracle.prefill(pw.q, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
+                             pw.query_start)
+    s = bench.prefill_sample(pw, 3)
+    rec = bench.prefill_parity(pw, s, full)
+    assert rec["max_abs"] == 0.0 and rec["within"] and rec["rows"] == 3
+    bad = full.copy()
+    bad[7, 0, 0] += 0.5  # a row of the sample (sequence 0's rows 6..8)
+    assert not bench.prefill_parity(pw, s, bad)["within"]
+    bad = full.copy()
+    bad[2, 0, 0] += 0.5  # outside the sample
+    assert bench.prefill_parity(pw, s, bad)["within"]
