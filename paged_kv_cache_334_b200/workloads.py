@@ -49,6 +49,11 @@ token of the current decode step: its K/V rows are returned in
 its place in the cache is filled with NaN until the cache write runs.  Slots
 of unreferenced blocks and slots past each context length are NaN too, so a
 kernel that reads outside the visible history produces NaN.
+
+Prefill inputs (``prefill_workload``) reuse a bf16 workload's pool, tables
+and lengths with the held-back newest tokens put into their slots, and draw
+a fresh q (N(0, 1), bf16) with one row per chunk token: whole prompts, or
+the last tokens of each context as the chunk of a chunked prefill.
 """
 from __future__ import annotations
 
