@@ -70,7 +70,14 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="gqa_bf16", choices=wl.WORKLOADS)
+    ap.add_argument("--workload", default=None, choices=wl.WORKLOADS,
+                    help="default: the mixed-length continuous batch (decode steps), the "
+                         "long-context batch (--step splitk), the bf16 GQA batch as prompts "
+                         "(--step prefill)")
+    ap.add_argument("--companion", default="gqa_bf16", choices=wl.WORKLOADS + ("none",),
+                    help="a second workload measured in the same run and reported under its "
+                         "own key of the same JSON line (default: the bf16 GQA batch, the "
+                         "other configuration the target names); 'none' skips it")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--block-size", type=int, default=None,
                     help="page size override for gqa_bf16 / mixed_bf16 / long_bf16 (a sweep)")
@@ -78,17 +85,25 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--step", choices=("fused", "separate", "prefix", "prefill"),
+    ap.add_argument("--step", choices=("fused", "separate", "prefix", "splitk", "prefill"),
                     default="fused",
                     help="fused: one pa_forward_decode call per step (cache write inside the "
                          "decode kernel); separate: pa_write_kv_cache then pa_decode; prefix: "
                          "pa_write_kv_cache then pa_decode_shared_prefix (workloads with a "
-                         "shared prefix); prefill: one pa_prefill call over the workload's "
-                         "sequences as whole prompts (bf16 workloads), reported in TFLOP/s")
+                         "shared prefix); splitk: pa_write_kv_cache then pa_decode_splitk "
+                         "(--partition-tokens partitions) and pa_reduce; prefill: one "
+                         "pa_prefill call over the workload's sequences as whole prompts "
+                         "(bf16 workloads), reported in TFLOP/s")
+    ap.add_argument("--partition-tokens", type=int, default=512,
+                    help="--step splitk: tokens per partition")
     ap.add_argument("--chunk", type=int, default=None,
                     help="--step prefill: the last CHUNK tokens of each context are the "
                          "chunk (a later chunk of a chunked prefill) instead of whole prompts")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    if args.workload is None:
+        args.workload = {"prefill": "gqa_bf16", "splitk": "long_bf16",
+                         "prefix": "mqa_prefix_bf16"}.get(args.step, "mixed_bf16")
+    return args
 
 
 # ---------------------------------------------------------------------------
@@ -444,7 +459,10 @@ def workload_config(w, args):
                           "decode kernel, then decode)",
                  "separate": "pa_write_kv_cache(newest token of every sequence) + pa_decode",
                  "prefix": "pa_write_kv_cache(newest token of every sequence) + "
-                           "pa_decode_shared_prefix"}[args.step],
+                           "pa_decode_shared_prefix",
+                 "splitk": f"pa_write_kv_cache(newest token of every sequence) + "
+                           f"pa_decode_splitk({args.partition_tokens}-token partitions) + "
+                           f"pa_reduce"}[args.step],
         "l2": "flushed before every timed step (zero-fill then read of 2x L2, outside the events)",
         "parallelism": f"replicas: one independent batch per GPU x{args.gpus}",
     }
@@ -483,19 +501,14 @@ def run_reference(args):
 # our arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args):
+def measure_decode(args, name, dev, dist, rank, world, baseline=True):
+    """Time K decode steps of workload `name` (the step --step selects) and
+    return the fields of its JSON record (device-timed value and roofline,
+    e2e, and on rank 0 of a one-GPU run the CPU baseline and parity)."""
     import torch
     from paged_kv_cache_334_b200 import pa
 
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = init_dist(world, local)
-    pa.load()
-
-    w = wl.make_workload(args.workload, seed=rank_seed(args.seed, rank),
-                         block_size=args.block_size)
-    tdt = torch.float32 if w.dtype == wl.DTYPE_F32 else torch.bfloat16
+    w = wl.make_workload(name, seed=rank_seed(args.seed, rank), block_size=args.block_size)
 
     def dev_t(a):
         t = torch.from_numpy(np.ascontiguousarray(a))
@@ -525,15 +538,24 @@ def run_ours(args):
     flush_sink = torch.empty((), dtype=torch.float32, device=dev)
     fused = has_new and args.step == "fused"
     prefix = args.step == "prefix"
+    splitk = args.step == "splitk"
     if prefix and not w.shared_prefix_blocks:
         raise SystemExit(f"--step prefix needs a workload with a shared prefix, not {w.name}")
+    if splitk:
+        P = args.partition_tokens
+        maxp = -(-w.max_blocks * w.block_size // P)
+        pm = torch.empty(w.batch, w.num_q_heads, maxp, dtype=torch.float32, device=dev)
+        ps = torch.empty_like(pm)
+        po = torch.empty(w.batch, w.num_q_heads, maxp, w.head_dim, dtype=torch.float32,
+                         device=dev)
     # libpa kernels per step.  Groups of 64 or 128 query heads (tensor-core
     # path): the write (inside pa_forward_decode or as its own call), the
     # tile kernel, and its finishing pass or, with a shared prefix, the
-    # prefix kernel.  Other groups: the persistent decode
-    # kernel and its merge kernel, plus the write kernel when the write is a
-    # separate call, plus the prefix kernel of the shared-prefix path.
-    tensor = tensor_path(w)
+    # prefix kernel.  Other groups: the persistent decode kernel and its
+    # merge kernel (split-K: pa_reduce's kernel instead), plus the write
+    # kernel when the write is a separate call, plus the prefix kernel of
+    # the shared-prefix path.
+    tensor = tensor_path(w) and not splitk
     if tensor:
         launches_per_step = 2 + (1 if has_new else 0)
     else:
@@ -554,6 +576,10 @@ def run_ours(args):
         if prefix:
             pa.pa_decode_shared_prefix(out, q, kc, vc, bt, cl, w.shared_prefix_blocks, scale=scale,
                                        err_word=err, stream=stream, **sc)
+        elif splitk:
+            pa.pa_decode_splitk(q, kc, vc, bt, cl, P, pm, ps, po, scale=scale, err_word=err,
+                                stream=stream, **sc)
+            pa.pa_reduce(out, pm, ps, po, cl, P, err_word=err, stream=stream)
         elif fused:
             pa.pa_forward_decode(out, q, kc, vc, kn, vn, sm, bt, cl, scale=scale, workspace=ws,
                                  err_word=err, stream=stream, **sc)
@@ -571,7 +597,7 @@ def run_ours(args):
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index)
     clocks.start()
     if dist is not None:
         dist.barrier()
@@ -591,7 +617,8 @@ def run_ours(args):
         dist.barrier()
     clk = clocks.stop()
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    # the timed kernel call: pa_forward_decode (the whole step) or pa_decode
+    # the timed kernel call: pa_forward_decode (the whole step) or the decode
+    # call(s) after the write
     dec_ms = step_ms if fused else [e[1].elapsed_time(e[2]) for e in ev]
     t_step = statistics.mean(step_ms)
     t_dec = statistics.mean(dec_ms)
@@ -630,7 +657,7 @@ def run_ours(args):
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word {int(err.item())}")
 
-    step_bytes = wl.roofline_bytes(w)
+    step_bytes = wl.roofline_bytes(w, include_write=has_new)
     dec_bytes = step_bytes if fused else wl.roofline_bytes(w, include_write=False)
     t_step_max = reduce_scalar(t_step, "max", dist, dev)
     bytes_all = reduce_scalar(step_bytes, "sum", dist, dev)
@@ -644,13 +671,17 @@ def run_ours(args):
                     "ms_per_step": t_e2e_max}
 
     cpu = parity = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0 and world == 1:
+        if baseline and not args.no_cpu_baseline:
+            cpu = cpu_baseline(w, args.cpu_seconds)
         # the timed call's output rows of the first sequences against the oracle
         parity = parity_sample(w, out[:8].double().cpu().numpy(), 8)
 
     peak, peak_src = hbm_peak()
     achieved = dec_bytes / (t_dec * 1e-3) / 1e9
+    kernel = ("pa_decode_shared_prefix" if prefix else
+              "pa_decode_splitk + pa_reduce" if splitk else
+              "pa_forward_decode" if fused else "pa_decode")
     roofline_tensor = None
     if prefix or tensor:
         # 64 or 128 query heads per KV head (32 or 64 flop per byte of KV),
@@ -660,15 +691,20 @@ def run_ours(args):
         tach = attention_flops(w) / (t_dec * 1e-3) / 1e12
         roofline_tensor = {
             "bound": "tensor", "achieved": tach, "peak": tpeak, "unit": "TFLOP/s",
-            "frac": tach / tpeak, "traffic": None,
-            "kernel": ("pa_decode_shared_prefix" if prefix else
-                       "pa_forward_decode" if fused else "pa_decode"),
+            "frac": tach / tpeak, "traffic": None, "kernel": kernel,
             "flops_per_launch": attention_flops(w), "launch_us": t_dec * 1e3,
             "peak_source": tpeak_src, "hbm_gbs": achieved, "hbm_frac": achieved / peak,
             "ceilings": ceilings(w, attention_flops(w), dec_bytes, t_dec * 1e3,
                                  (clk or {}).get("sm_mhz") or 1965.0),
         }
-    line = {
+    traffic = None
+    if args.block_size is None and not splitk and not prefix:
+        traffic = recorded_traffic(name)
+    config = workload_config(w, args)
+    if splitk:
+        config["partitions"] = {"tokens": P, "max_partitions": maxp,
+                                "partials_bytes": int(pm.numel() * 8 + po.numel() * 4)}
+    return {
         "metric": METRIC,
         "value": bytes_all / (t_step_max * 1e-3) / 1e9,
         "unit": "GB/s",
@@ -682,16 +718,13 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic",
-        "config": workload_config(w, args),
+        "config": config,
         "seq_tokens_per_s": seqs_all / (t_step_max * 1e-3),
         "context_tokens_per_s": ctx_all / (t_step_max * 1e-3),
         "hbm_frac_step": (bytes_all / (t_step_max * 1e-3) / 1e9) / (peak * world),
         "roofline": roofline_tensor if roofline_tensor is not None else {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak,
-            "traffic": recorded_traffic(args.workload) if args.block_size is None else None,
-            "kernel": ("pa_forward_decode" if fused else
-                       "pa_decode_shared_prefix" if prefix else "pa_decode"),
+            "frac": achieved / peak, "traffic": traffic, "kernel": kernel,
             "algorithmic_bytes_per_launch": dec_bytes,
             "launch_us": t_dec * 1e3, "peak_source": peak_src,
         },
@@ -701,6 +734,30 @@ def run_ours(args):
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
+
+
+def run_ours(args):
+    import torch
+    from paged_kv_cache_334_b200 import pa
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, local)
+    pa.load()
+
+    line = measure_decode(args, args.workload, dev, dist, rank, world)
+    if (args.companion != "none" and args.companion != args.workload
+            and args.step in ("fused", "separate")):
+        # the second configuration the target names, timed the same way in
+        # the same run (its own warm-up, K steps, L2 flushes and clocks)
+        torch.cuda.empty_cache()
+        sub = measure_decode(args, args.companion, dev, dist, rank, world, baseline=False)
+        line["gpu_launches"] += sub["gpu_launches"]
+        line[args.companion] = {k: sub[k] for k in (
+            "value", "unit", "ms_per_step", "step_ms", "hbm_frac_step", "seq_tokens_per_s",
+            "context_tokens_per_s", "roofline", "e2e", "parity", "gpu_launches", "clocks",
+            "config", "dtype")}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -78,9 +78,9 @@ typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1, PA_DTYPE_FP8_E4M3 =
  * pa_write_kv_cache stores the code nearest to x / scale (the division in
  * IEEE single precision, ties to the even mantissa, magnitudes at or above
  * 448 saturating to 448).  Served by pa_write_kv_cache, pa_decode,
- * pa_forward_decode and pa_decode_noalloc for head_dim 128, block_size >=
- * 16, 4 or 8 KV heads and at most 8 query heads per KV head; other calls
- * and shapes return PA_ERR_UNSUPPORTED.  Decode converts the codes exactly
+ * pa_forward_decode, pa_decode_noalloc and pa_decode_splitk for head_dim
+ * 128, block_size >= 16, 4 or 8 KV heads and at most 8 query heads per KV
+ * head; other calls and shapes return PA_ERR_UNSUPPORTED.  Decode converts the codes exactly
  * and multiplies them in fp16 tiles (fp32 accumulation), so q must lie
  * within fp16's range (|q| < 65504).
  */
@@ -372,7 +372,12 @@ pa_status pa_decode_noalloc(const pa_cache_desc *cache, void *out,
  * part_out [batch, num_q_heads, max_partitions, head_dim]; all fp32.
  * partition_tokens must be a positive multiple of block_size;
  * max_partitions must be >= ceil(max_blocks_per_seq * block_size /
- * partition_tokens).
+ * partition_tokens).  No workspace: on the shapes of pa_decode's persistent
+ * page-stream kernel the partitions of all sequences form one stream cut
+ * into one range per SM at partition boundaries, so each partition is
+ * computed whole by one CTA and written once; other shapes run one CTA per
+ * (partition, KV head, head tile) and allow at most 1024 blocks per
+ * partition.
  */
 pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
                            const void *key_cache, const void *value_cache,

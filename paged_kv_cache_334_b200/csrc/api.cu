@@ -418,6 +418,84 @@ namespace pa {
 void set_last_error_message(const char *msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
 }  // namespace pa
 
+// Arguments of the persistent page-stream kernel common to pa_decode (and its
+// variants) and pa_decode_splitk: shapes, the tensor maps of the caches (or a
+// row-copy plan when they cannot be described), the stage layout and the
+// scales.  The caller fills in the outputs and the workspace pointers.
+static pa_status stream_params(const pa_cache_desc *cache, const void *q, const void *key_cache,
+                               const void *value_cache, const int32_t *block_tables,
+                               const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+                               int32_t max_blocks_per_seq, int32_t prefix_blocks, float scale,
+                               int32_t *err_word, pa::stream::Params *pp, StreamPlan *plan) {
+  const bool fp8 = cache->dtype == PA_DTYPE_FP8_E4M3;
+  StreamPlan sp = plan_stream(cache, num_q_heads);
+  const int sms = device_sm_count();
+  if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
+  pa::stream::Params &p = *pp;
+  if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, sp.vbs) &&
+                   encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs))) {
+    if (fp8) return fail(PA_ERR_CUDA, "cannot describe the FP8 caches for the tensor copies%s");
+    sp = plan_stream(cache, num_q_heads, /*allow_tile=*/false);
+  }
+  if (!sp.ok) return fail(PA_ERR_UNSUPPORTED, "no page-stream plan for these shapes%s");
+  p.q = q;
+  p.key_cache = const_cast<void *>(key_cache);
+  p.value_cache = const_cast<void *>(value_cache);
+  p.block_tables = block_tables + prefix_blocks;
+  p.context_lens = context_lens;
+  p.err_word = err_word;
+  p.num_blocks = cache->num_blocks;
+  p.block_size = cache->block_size;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.num_q_heads = num_q_heads;
+  p.max_blocks = max_blocks_per_seq - prefix_blocks;
+  p.table_stride = max_blocks_per_seq;
+  p.tok_offset = prefix_blocks * cache->block_size;
+  p.batch = batch;
+  p.vbs = sp.vbs;
+  p.log2_vbs = sp.log2_vbs;
+  p.log2_vpp = sp.log2_vpp;
+  p.row_bytes = sp.row_bytes;
+  p.row_pitch = sp.row_pitch;
+  p.vpage_stride = sp.vpage_stride;
+  p.q_bytes = sp.q_bytes;
+  p.pps = sp.pps;
+  p.stages = sp.stages;
+  p.stage_bytes = sp.stage_bytes;
+  p.hdr_bytes = pa::stream::kHdrBytes;
+  p.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.fp8 = fp8 ? 1 : 0;
+  p.out_scale = 1.f;
+  p.k_scale = cache->k_scale;
+  p.v_scale = cache->v_scale;
+  if (fp8) {
+    // the consumers see code value * 2^-8 (exact in fp16): 256 k_scale
+    // goes into the score scale, 256 v_scale into the output
+    p.scale_log2 *= 256.f * cache->k_scale;
+    p.out_scale = 256.f * cache->v_scale;
+  }
+  p.group = num_q_heads / cache->num_kv_heads;
+  p.heads_per_warp = sp.heads_per_warp;
+  p.warps_per_kv = sp.warps_per_kv;
+  p.tile = sp.tile ? 1 : 0;
+  p.box_bytes = sp.box_bytes;
+  p.n_dhalf = sp.n_dhalf;
+  *plan = sp;
+  return PA_OK;
+}
+
+static cudaError_t launch_stream(const pa::stream::Params &p, const pa_cache_desc *cache,
+                                 const StreamPlan &sp, cudaStream_t stream) {
+  if (cache->dtype == PA_DTYPE_FP8_E4M3)
+    return pa::stream::launch_fp8(p, cache->num_kv_heads, sp.smem, stream);
+  if (cache->dtype == PA_DTYPE_F32)
+    return pa::stream::launch_f32(p, cache->head_dim, p.group, cache->num_kv_heads, sp.smem,
+                                  stream);
+  return pa::stream::launch_bf16(p, cache->head_dim, p.group, cache->num_kv_heads, sp.smem,
+                                 stream);
+}
+
 // pa_decode, and pa_forward_decode when k_new / v_new / slot_mapping are set.
 // With prefix_blocks > 0 (pa_decode_shared_prefix, persistent kernel only):
 // the first prefix_blocks pages of every sequence are left out and each
@@ -484,79 +562,25 @@ static pa_status decode_impl(const pa_cache_desc *cache, void *out, const void *
                 "FP8 pages: head_dim 128, block_size >= 16, 4 or 8 KV heads and at most 8 "
                 "query heads per KV head%s");
   if (w.stream) {
-    StreamPlan sp = plan_stream(cache, num_q_heads);
-    const int sms = device_sm_count();
-    if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
     pa::stream::Params p{};
-    if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, sp.vbs) &&
-                     encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs))) {
-      if (fp8) return fail(PA_ERR_CUDA, "cannot describe the FP8 caches for the tensor copies%s");
-      sp = plan_stream(cache, num_q_heads, /*allow_tile=*/false);
-    }
-    p.q = q;
+    StreamPlan sp{};
+    s = stream_params(cache, q, key_cache, value_cache, block_tables, context_lens, batch,
+                      num_q_heads, max_blocks_per_seq, prefix_blocks, scale, err_word, &p, &sp);
+    if (s != PA_OK) return s;
     p.out = out;
-    p.key_cache = key_cache;
-    p.value_cache = value_cache;
     p.k_new = k_new;
     p.v_new = v_new;
     p.slot_mapping = slot_mapping;
-    p.block_tables = block_tables + prefix_blocks;
-    p.context_lens = context_lens;
     p.seq_ml = seq_ml;
     p.seq_o = seq_o;
     p.part_ml = reinterpret_cast<float *>(ws + w.part_max);
     p.part_o = reinterpret_cast<float *>(ws + w.part_out);
     p.seq_merge = reinterpret_cast<int32_t *>(ws + w.counters);
-    p.err_word = err_word;
-    p.num_blocks = cache->num_blocks;
-    p.block_size = cache->block_size;
-    p.num_kv_heads = cache->num_kv_heads;
-    p.num_q_heads = num_q_heads;
-    p.max_blocks = max_blocks_per_seq - prefix_blocks;
-    p.table_stride = max_blocks_per_seq;
-    p.tok_offset = prefix_blocks * cache->block_size;
-    p.batch = batch;
-    p.vbs = sp.vbs;
-    p.log2_vbs = sp.log2_vbs;
-    p.log2_vpp = sp.log2_vpp;
-    p.row_bytes = sp.row_bytes;
-    p.row_pitch = sp.row_pitch;
-    p.vpage_stride = sp.vpage_stride;
-    p.q_bytes = sp.q_bytes;
-    p.pps = sp.pps;
-    p.stages = sp.stages;
-    p.stage_bytes = sp.stage_bytes;
-    p.hdr_bytes = pa::stream::kHdrBytes;
-    p.grid = sms < pa::stream::kMaxGrid ? sms : pa::stream::kMaxGrid;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.fp8 = fp8 ? 1 : 0;
-    p.out_scale = 1.f;
-    p.k_scale = cache->k_scale;
-    p.v_scale = cache->v_scale;
-    if (fp8) {
-      // the consumers see code value * 2^-8 (exact in fp16): 256 k_scale
-      // goes into the score scale, 256 v_scale into the output
-      p.scale_log2 *= 256.f * cache->k_scale;
-      p.out_scale = 256.f * cache->v_scale;
-    }
-    const int group = num_q_heads / cache->num_kv_heads;
-    p.group = group;
-    p.heads_per_warp = sp.heads_per_warp;
-    p.warps_per_kv = sp.warps_per_kv;
-    p.tile = sp.tile ? 1 : 0;
-    p.box_bytes = sp.box_bytes;
-    p.n_dhalf = sp.n_dhalf;
-    const bool mma = cache->dtype != PA_DTYPE_F32;
-    cudaError_t e = fp8 ? pa::stream::launch_fp8(p, cache->num_kv_heads, sp.smem,
-                                                 static_cast<cudaStream_t>(stream))
-                    : mma
-                        ? pa::stream::launch_bf16(p, cache->head_dim, group, cache->num_kv_heads,
-                                                  sp.smem, static_cast<cudaStream_t>(stream))
-                        : pa::stream::launch_f32(p, cache->head_dim, group, cache->num_kv_heads,
-                                                 sp.smem, static_cast<cudaStream_t>(stream));
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_stream(p, cache, sp, st);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    e = mma ? pa::stream::launch_merge_bf16(p, cache->head_dim, static_cast<cudaStream_t>(stream))
-            : pa::stream::launch_merge_f32(p, cache->head_dim, static_cast<cudaStream_t>(stream));
+    e = cache->dtype == PA_DTYPE_F32 ? pa::stream::launch_merge_f32(p, cache->head_dim, st)
+                                     : pa::stream::launch_merge_bf16(p, cache->head_dim, st);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
     return PA_OK;
   }
@@ -960,13 +984,16 @@ pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
                                     context_lens, batch, num_q_heads,
                                     max_blocks_per_seq, scale);
   if (s != PA_OK) return s;
-  if (cache->dtype == PA_DTYPE_FP8_E4M3)
-    return fail(PA_ERR_UNSUPPORTED, "pa_decode_splitk takes F32 or BF16 pages, not FP8%s");
+  const bool streamed = plan_stream(cache, num_q_heads).ok;
+  if (cache->dtype == PA_DTYPE_FP8_E4M3 && !streamed)
+    return fail(PA_ERR_UNSUPPORTED,
+                "FP8 pages: head_dim 128, block_size >= 16, 4 or 8 KV heads and at most 8 "
+                "query heads per KV head%s");
   if (partition_tokens <= 0 || partition_tokens % cache->block_size != 0)
     return fail(PA_ERR_INVALID_ARG,
                 "partition_tokens must be a positive multiple of block_size%s (got %lld)", "",
                 partition_tokens);
-  if (partition_tokens / cache->block_size > kMaxPartitionPages)
+  if (!streamed && partition_tokens / cache->block_size > kMaxPartitionPages)
     return fail(PA_ERR_UNSUPPORTED, "more than 1024 blocks per partition%s (%lld)", "",
                 partition_tokens / cache->block_size);
   const int64_t need =
@@ -980,6 +1007,25 @@ pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
   if ((s = check_ptr(part_max, "part_max")) != PA_OK) return s;
   if ((s = check_ptr(part_sum, "part_sum")) != PA_OK) return s;
   if ((s = check_ptr(part_out, "part_out")) != PA_OK) return s;
+  if (streamed) {
+    // the persistent page-stream kernel in split-K mode: CTA ranges end on
+    // partition boundaries, so every partition is written by one CTA and
+    // no workspace is needed
+    pa::stream::Params p{};
+    StreamPlan sp{};
+    s = stream_params(cache, q, key_cache, value_cache, block_tables, context_lens, batch,
+                      num_q_heads, max_blocks_per_seq, 0, scale, err_word, &p, &sp);
+    if (s != PA_OK) return s;
+    p.sk_max = part_max;
+    p.sk_sum = part_sum;
+    p.sk_o = part_out;
+    p.part_pages = partition_tokens / sp.vbs;
+    p.max_parts = max_partitions;
+    const cudaError_t e = launch_stream(p, cache, sp, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+      return fail(PA_ERR_CUDA, "decode_splitk launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+  }
   pa::DecodeArgs a{};
   a.q = q;
   a.out = nullptr;

@@ -43,6 +43,11 @@
 //   and the CTA that owns its last page records where they are; a small merge
 //   kernel (launched right behind, programmatically) folds them together with
 //   the running-max rescaling once the stream of pages is done.
+// * Split-K mode (pa_decode_splitk): the units are (sequence, partition)
+//   pairs of partition_tokens tokens; CTA ranges are snapped to unit
+//   boundaries (a unit goes to the CTA whose share of the stream holds its
+//   midpoint), so no unit is cut and each CTA writes its units' (max, sum,
+//   normalised output) straight into the caller's partial arrays.
 //
 // Every mbarrier wait is bounded; on expiry the kernel sets PA_DEVERR_TIMEOUT,
 // drains its own copies (bounded) and returns.
@@ -56,10 +61,15 @@
 #include "pa_launch.h"
 #include "sm100_ptx.cuh"
 
+
 namespace pa {
 namespace stream {
 
-constexpr int kFirst = 1, kLast = 2, kBad = 4;
+// Page descriptor flags: first page of a sequence in this CTA (reset, load
+// q), last page of a unit (a sequence, or a split-K partition) in this CTA
+// (flush, then reset), a bad block id, the sequence is cut between CTAs
+// (flush a partial), the partial goes to this CTA's second slot.
+constexpr int kFirst = 1, kLast = 2, kBad = 4, kCut = 8, kSlot1 = 16;
 // Block tables up to this size are prefetched into L2 at kernel start.
 constexpr uint64_t kTablePrefetchMax = 16ull << 20;
 constexpr int kSeqCache = 256;
@@ -69,8 +79,8 @@ constexpr int kSeqCache = 256;
 struct Fp8E4M3 {};
 
 struct alignas(16) PageDesc {
-  int32_t seq, ntok, flags, n_contrib;
-  int32_t c_first, slot_bits, pb, toff;
+  int32_t seq, ntok, flags, unit;  // unit: split-K partition index
+  int32_t pb, toff, pad0, pad1;
 };
 
 // Tokens of sequence s this call attends to (all of them, or the suffix
@@ -129,11 +139,22 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t *s_re
   return base + inc - v;
 }
 
+// Start of the first unit whose midpoint lies at or after stream page x,
+// where [P, P + v) are the pages of the sequence holding x and pp the pages
+// of a full partition (split-K mode).
+__device__ __forceinline__ int64_t unit_bound(int64_t x, int64_t P, int64_t v, int64_t pp) {
+  const int64_t u = (x - P) / pp;
+  const int64_t us = P + u * pp;
+  const int64_t ue = P + ((u + 1) * pp < v ? (u + 1) * pp : v);
+  return (us + ue >= 2 * x) ? us : ue;
+}
+
 struct alignas(16) Shared {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   int64_t red[32];
   int64_t P_begin;
+  int64_t range[2];  // split-K: this CTA's pages [range[0], range[1]) of the stream
   int32_t s_begin, vlb_begin, abort_flag, pad;
   // Batches of up to kSeqCache sequences: context lengths and new-token
   // slots read once by the prologue, so that the producer never waits on a
@@ -375,7 +396,29 @@ struct MmaConsumer {
       v[k] = q < 2 ? make_float4(lo0 * inv, lo1 * inv, r0 * inv, r1 * inv)
                    : make_float4(r0 * inv, r1 * inv, hi0 * inv, hi1 * inv);
     }
-    if (d.n_contrib == 1) {
+    if (p.sk_o != nullptr) {
+      // split-K: this partition's (max, normaliser, normalised output), the
+      // max back in natural units
+      const int64_t row = ((int64_t)d.seq * p.num_q_heads + hq0) * p.max_parts + d.unit;
+      const int64_t mp = p.max_parts;
+      if (g == 0) {
+        if (2 * t < nh) {
+          p.sk_max[row + 2 * t * mp] = m0_ * kLn2;
+          p.sk_sum[row + 2 * t * mp] = seg_bad ? -1.f : L0;
+        }
+        if (2 * t + 1 < nh) {
+          p.sk_max[row + (2 * t + 1) * mp] = m1_ * kLn2;
+          p.sk_sum[row + (2 * t + 1) * mp] = seg_bad ? -1.f : L1;
+        }
+      }
+      if (hh < nh) {
+#pragma unroll
+        for (int k = 0; k < KS; ++k)
+          *reinterpret_cast<float4 *>(p.sk_o + (row + hh * mp) * D + k * 16 + dcol) = v[k];
+      }
+      return;
+    }
+    if (!(d.flags & kCut)) {
       if (p.seq_o != nullptr) {
         // suffix mode: the sequence's result as a partial for the prefix pass
         const int64_t row = (int64_t)d.seq * p.num_q_heads + hq0;
@@ -400,7 +443,7 @@ struct MmaConsumer {
       }
       return;
     }
-    const int64_t prow = ((int64_t)c * 2 + (d.slot_bits & 1)) * p.num_q_heads + hq0;
+    const int64_t prow = ((int64_t)c * 2 + ((d.flags & kSlot1) ? 1 : 0)) * p.num_q_heads + hq0;
     if (g == 0) {
       if (2 * t < nh)
         *reinterpret_cast<float2 *>(p.part_ml + (prow + 2 * t) * 2) =
@@ -414,7 +457,7 @@ struct MmaConsumer {
 #pragma unroll
       for (int k = 0; k < KS; ++k) *reinterpret_cast<float4 *>(row + k * 16 + dcol) = v[k];
     }
-    // merged later by the merge kernel
+    // merged by the last contributing CTA at its end
   }
 };
 
@@ -602,7 +645,27 @@ struct HeadRowConsumer {
       L1 += __shfl_xor_sync(0xffffffffu, L1, mask);
     }
     const float i0 = seg_bad ? 0.f : p.out_scale / L0, i1 = seg_bad ? 0.f : p.out_scale / L1;
-    if (d.n_contrib == 1 && p.seq_o != nullptr) {
+    if (p.sk_o != nullptr) {
+      // split-K: this partition's (max, normaliser, normalised output)
+      const int64_t mp = p.max_parts;
+      const int64_t ix0 = ((int64_t)d.seq * p.num_q_heads + hq0 + r) * mp + d.unit;
+      const int64_t ix1 = ix0 + 8 * mp;
+      if (c == 0) {
+        p.sk_max[ix0] = m0_ * kLn2;
+        p.sk_sum[ix0] = seg_bad ? -1.f : L0;
+        p.sk_max[ix1] = m1_ * kLn2;
+        p.sk_sum[ix1] = seg_bad ? -1.f : L1;
+      }
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        *reinterpret_cast<float2 *>(p.sk_o + ix0 * D + 8 * j + 2 * c) =
+            make_float2(o[j][0] * i0, o[j][1] * i0);
+        *reinterpret_cast<float2 *>(p.sk_o + ix1 * D + 8 * j + 2 * c) =
+            make_float2(o[j][2] * i1, o[j][3] * i1);
+      }
+      return;
+    }
+    if (!(d.flags & kCut) && p.seq_o != nullptr) {
       // suffix mode: the sequence's result as a partial for the prefix pass
       const int64_t row = (int64_t)d.seq * p.num_q_heads + hq0 + r;
       if (c == 0) {
@@ -618,7 +681,7 @@ struct HeadRowConsumer {
       }
       return;
     }
-    if (d.n_contrib == 1) {
+    if (!(d.flags & kCut)) {
       const int64_t row0 = ((int64_t)d.seq * p.num_q_heads + hq0 + r) * D;
       const int64_t row1 = row0 + 8 * D;
 #pragma unroll
@@ -628,7 +691,8 @@ struct HeadRowConsumer {
       }
       return;
     }
-    const int64_t prow = ((int64_t)c_idx * 2 + (d.slot_bits & 1)) * p.num_q_heads + hq0;
+    const int64_t prow =
+        ((int64_t)c_idx * 2 + ((d.flags & kSlot1) ? 1 : 0)) * p.num_q_heads + hq0;
     if (c == 0) {
       *reinterpret_cast<float2 *>(p.part_ml + (prow + r) * 2) =
           make_float2(m0_, seg_bad ? -1.f : L0);
@@ -642,7 +706,7 @@ struct HeadRowConsumer {
       *reinterpret_cast<float2 *>(orow0 + 8 * j + 2 * c) = make_float2(o[j][0] * i0, o[j][1] * i0);
       *reinterpret_cast<float2 *>(orow1 + 8 * j + 2 * c) = make_float2(o[j][2] * i1, o[j][3] * i1);
     }
-    // merged later by the merge kernel
+    // merged by the last contributing CTA at its end
   }
 };
 
@@ -809,7 +873,25 @@ struct FmaConsumer {
 #pragma unroll
     for (int g = 0; g < G; ++g) lg[g] = __shfl_sync(0xffffffffu, lsum, g);
     const int64_t orow = (int64_t)d.seq * p.num_q_heads + hq0;
-    if (d.n_contrib == 1) {
+    if (p.sk_o != nullptr) {
+      // split-K: this partition's (max, normaliser, normalised output)
+      const int64_t mp = p.max_parts;
+      if (lane < G) {
+        const int64_t ix = (orow + lane) * mp + d.unit;
+        p.sk_max[ix] = m_run * kLn2;
+        p.sk_sum[ix] = seg_bad ? -1.f : lsum;
+      }
+      if (tg == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int e = 0; e < EPV; ++e)
+            p.sk_o[((orow + g) * mp + d.unit) * D + j * EPV + e] =
+                seg_bad ? 0.f : ac[g][e] / lg[g];
+      }
+      return;
+    }
+    if (!(d.flags & kCut)) {
       if (tg == 0) {
 #pragma unroll
         for (int g = 0; g < G; ++g)
@@ -820,7 +902,7 @@ struct FmaConsumer {
       }
       return;
     }
-    const int64_t prow = ((int64_t)c * 2 + (d.slot_bits & 1)) * p.num_q_heads + hq0;
+    const int64_t prow = ((int64_t)c * 2 + ((d.flags & kSlot1) ? 1 : 0)) * p.num_q_heads + hq0;
     if (lane < G) {
       p.part_ml[(prow + lane) * 2 + 0] = m_run;
       p.part_ml[(prow + lane) * 2 + 1] = seg_bad ? -1.f : lsum;
@@ -832,7 +914,7 @@ struct FmaConsumer {
         for (int e = 0; e < EPV; ++e)
           p.part_o[(prow + g) * D + j * EPV + e] = seg_bad ? 0.f : ac[g][e] / lg[g];
     }
-    // merged later by the merge kernel
+    // merged by the last contributing CTA at its end
   }
 };
 
@@ -1136,11 +1218,18 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       mbar_init(&sh.empty[i], NCW);
     }
     sh.abort_flag = 0;
+    sh.range[0] = sh.range[1] = 0;
     // make the initialised barriers visible to the bulk-copy (async) proxy
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
 
-  // ---- Prologue: total virtual pages T, this CTA's range and first page.
+  // ---- Prologue: pages per sequence, the stream's total T, this CTA's
+  // range [start, end) of it and the sequence / page it starts at.
+  //   pa_decode: ranges of equal page counts; units (sequences) may be cut.
+  //   split-K: unit boundaries nearest to the equal cuts (a unit goes to the
+  //   CTA whose share holds its midpoint); no unit is cut.
+  const bool splitk = p.sk_o != nullptr;
+  const int32_t pp = splitk ? p.part_pages : 0;  // pages per split-K partition
   int64_t Tp, start = 0, end = 0;
   int32_t g_eff;
   const bool cached = p.batch <= kSeqCache;
@@ -1156,15 +1245,26 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     }
     const int64_t v = (tid < p.batch) ? vpages_of(ctx, p) : 0;
     const int64_t P = block_exclusive_scan(v, sh.red, &Tp);
-    g_eff = (int32_t)((Tp < p.grid) ? Tp : p.grid);
-    if (c < g_eff) {
-      start = (int64_t)c * Tp / g_eff;
-      end = (int64_t)(c + 1) * Tp / g_eff;
-      if (v > 0 && P <= start && start < P + v) {
-        sh.s_begin = tid;
-        sh.vlb_begin = (int32_t)(start - P);
-        sh.P_begin = P;
+    if (splitk) {
+      g_eff = p.grid;
+      const int64_t x0 = (int64_t)c * Tp / g_eff, x1 = (int64_t)(c + 1) * Tp / g_eff;
+      if (v > 0 && P <= x0 && x0 < P + v) sh.range[0] = unit_bound(x0, P, v, pp);
+      if (v > 0 && P <= x1 && x1 < P + v) sh.range[1] = unit_bound(x1, P, v, pp);
+      if (tid == 0 && x1 >= Tp) sh.range[1] = Tp;
+      __syncthreads();
+      start = sh.range[0];
+      end = sh.range[1];
+    } else {
+      g_eff = (int32_t)((Tp < p.grid) ? Tp : p.grid);
+      if (c < g_eff) {
+        start = (int64_t)c * Tp / g_eff;
+        end = (int64_t)(c + 1) * Tp / g_eff;
       }
+    }
+    if (start < end && v > 0 && P <= start && start < P + v) {
+      sh.s_begin = tid;
+      sh.vlb_begin = (int32_t)(start - P);
+      sh.P_begin = P;
     }
   } else {
     int64_t T_loc = 0;
@@ -1182,10 +1282,32 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       T_loc += block_sum(v, sh.red);
     }
     Tp = T_loc;
-    g_eff = (int32_t)((Tp < p.grid) ? Tp : p.grid);
-    if (c < g_eff) {
-      start = (int64_t)c * Tp / g_eff;
-      end = (int64_t)(c + 1) * Tp / g_eff;
+    if (splitk) {
+      g_eff = p.grid;
+      const int64_t x0 = (int64_t)c * Tp / g_eff, x1 = (int64_t)(c + 1) * Tp / g_eff;
+      int64_t run = 0;
+      for (int base = 0; base < p.batch; base += blockDim.x) {
+        const int s = base + tid;
+        const int64_t v = (s < p.batch) ? vpages_of(visible_len(p, s), p) : 0;
+        int64_t tot;
+        const int64_t P = run + block_exclusive_scan(v, sh.red, &tot);
+        if (v > 0 && P <= x0 && x0 < P + v) sh.range[0] = unit_bound(x0, P, v, pp);
+        if (v > 0 && P <= x1 && x1 < P + v) sh.range[1] = unit_bound(x1, P, v, pp);
+        run += tot;
+        if (run > x1) break;  // uniform: every thread sees the same `run`
+      }
+      if (tid == 0 && x1 >= Tp) sh.range[1] = Tp;
+      __syncthreads();
+      start = sh.range[0];
+      end = sh.range[1];
+    } else {
+      g_eff = (int32_t)((Tp < p.grid) ? Tp : p.grid);
+      if (c < g_eff) {
+        start = (int64_t)c * Tp / g_eff;
+        end = (int64_t)(c + 1) * Tp / g_eff;
+      }
+    }
+    if (start < end) {
       int64_t run = 0;
       for (int base = 0; base < p.batch; base += blockDim.x) {
         const int s = base + tid;
@@ -1202,7 +1324,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       }
     }
   }
-  const bool active = c < g_eff;
+  const bool active = start < end;
   __syncthreads();
 
   const bool per_row = p.row_pitch != p.row_bytes;
@@ -1231,7 +1353,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           const int32_t ntok = wk.ntok(p);
           const bool first = (wk.vlb == 0) || (wk.cursor == start);
           const bool seq_last = wk.vlb == wk.pages_s - 1;
-          const bool last = seq_last || (wk.cursor == end - 1);
+          // split-K: a partition ends every pp pages (ranges end on unit ends)
+          const bool last = seq_last || (wk.cursor == end - 1) ||
+                            (pp > 0 && (wk.vlb + 1) % pp == 0);
           const bool bad_block = pb < 0 || pb >= p.num_blocks;
           bool bad = bad_block;
           if (bad_block && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
@@ -1256,26 +1380,27 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             PageDesc d;
             d.seq = wk.s;
             d.ntok = ntok;
-            d.flags = (first ? kFirst : 0) | (last ? kLast : 0) | (bad ? kBad : 0);
+            d.unit = pp > 0 ? wk.vlb / (int32_t)pp : 0;
             d.pb = pb;
             d.toff = (wk.vlb & ((1 << p.log2_vpp) - 1)) * p.vbs;
-            d.n_contrib = 1;
-            d.c_first = c;
-            d.slot_bits = 0;
-            if (last) {
+            d.pad0 = d.pad1 = 0;
+            int32_t flags = (first ? kFirst : 0) | (last ? kLast : 0) | (bad ? kBad : 0);
+            if (last && pp == 0) {
+              // is the sequence cut between CTAs?  Then this CTA leaves a
+              // partial in its slot 0 (the sequence holds the CTA's first
+              // page) or 1 (it starts inside the range and runs past it).
               const int32_t c_first = owner_of(wk.P_s, Tp, g_eff);
               const int32_t c_last = owner_of(wk.P_s + wk.pages_s - 1, Tp, g_eff);
-              d.n_contrib = c_last - c_first + 1;
-              d.c_first = c_first;
               const int64_t st_first = (int64_t)c_first * Tp / g_eff;
-              d.slot_bits = ((start < wk.P_s) ? 1 : 0) | ((st_first < wk.P_s) ? 2 : 0);
+              if (c_last > c_first) flags |= kCut | ((start < wk.P_s) ? kSlot1 : 0);
               if (c == c_last) {
                 // the owner of the sequence's last page tells the merge kernel
                 // where the partials are (or that there is nothing to merge)
-                reinterpret_cast<int4 *>(p.seq_merge)[wk.s] =
-                    make_int4(c_first, d.n_contrib, (st_first < wk.P_s) ? 1 : 0, 0);
+                reinterpret_cast<int4 *>(p.seq_merge)[wk.s] = make_int4(
+                    c_first, c_last - c_first + 1, (st_first < wk.P_s) ? 1 : 0, 0);
               }
             }
+            d.flags = flags;
             descs[slot * kMaxPPS + k] = d;
           }
           if (!bad)
@@ -1431,20 +1556,41 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     }
   }
 
-  // ---- Sequences with no visible page: zero output (and flag bad lengths).
   __syncthreads();
 
+  // ---- Sequences with no visible page: zero output, or empty partials
+  // (split-K: also every partition past a sequence's context); flag bad
+  // lengths.
   for (int s = c; s < p.batch; s += p.grid) {
-    if (vpages_of(visible_len(p, s), p) > 0) continue;
-    const int32_t ctx = p.context_lens[s];
-    if (tid == 0) {
-      reinterpret_cast<int4 *>(p.seq_merge)[s] = make_int4(0, 0, 0, 0);
+    const int32_t vis = cached ? sh.ctx_c[s] : visible_len(p, s);
+    const bool has = vpages_of(vis, p) > 0;
+    const int32_t ctx = vis + p.tok_offset;
+    if (!has && tid == 0) {
+      if (!splitk) reinterpret_cast<int4 *>(p.seq_merge)[s] = make_int4(0, 0, 0, 0);
       if (ctx < 0 || (int64_t)ctx > (int64_t)p.table_stride * p.block_size)
         set_error(p.err_word, PA_DEVERR_CONTEXT_LEN);
       // fused write: no visible position for the new token
-      if (p.slot_mapping != nullptr && p.slot_mapping[s] >= 0)
+      if (p.slot_mapping != nullptr && (cached ? sh.slot_c[s] : p.slot_mapping[s]) >= 0)
         set_error(p.err_word, PA_DEVERR_SLOT);
     }
+    if (splitk) {
+      const int32_t pt = (int32_t)pp << p.log2_vbs;  // tokens per partition
+      const int32_t used = has ? (vis + pt - 1) / pt : 0;
+      const int32_t left = p.max_parts - used;
+      if (left <= 0) continue;
+      const int64_t n4 = (int64_t)p.num_q_heads * left * (D / 4);
+      for (int64_t x = tid; x < n4; x += blockDim.x) {
+        const int32_t r = (int32_t)(x / (D / 4)), dq = (int32_t)(x % (D / 4));
+        const int64_t ix = ((int64_t)s * p.num_q_heads + r / left) * p.max_parts + used + r % left;
+        *reinterpret_cast<float4 *>(p.sk_o + ix * D + dq * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (dq == 0) {
+          p.sk_max[ix] = -INFINITY;
+          p.sk_sum[ix] = 0.f;
+        }
+      }
+      continue;
+    }
+    if (has) continue;
     const int64_t n = (int64_t)p.num_q_heads * D;
     if (p.seq_o != nullptr) {
       // empty suffix: a partial that weighs nothing
@@ -1505,7 +1651,6 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Para
   const int hq0 = (blockIdx.x % slices) * p.heads_per_warp;
   const int4 md = __ldcg(reinterpret_cast<const int4 *>(p.seq_merge) + seq);
   const int n = md.y;
-  if (n <= 1) return;  // empty, or written directly by its only CTA
   const int first_slot = md.z;
   const int64_t orow = (int64_t)seq * p.num_q_heads + hq0;
   // thread -> 4 consecutive outputs (head, d .. d+3) of this slice

@@ -63,6 +63,12 @@ struct Params {
   float *part_o;      // [kMaxGrid * 2][Hq][D]: normalised partial output
   int32_t *seq_merge;  // [batch][4]: first contributing CTA, contributors, slot of the first
   int32_t *err_word;
+  // Split-K mode (pa_decode_splitk) when sk_o is set: sequence b's
+  // partition u (part_pages virtual pages) writes sk_max / sk_sum [b][hq][u]
+  // (max in natural units, normaliser) and sk_o [b][hq][u][D] (normalised
+  // output), max_parts partitions per row; out, part_* and seq_merge unused.
+  float *sk_max, *sk_sum, *sk_o;
+  int32_t part_pages, max_parts;
   // Suffix mode (shared-prefix decode): the first tok_offset tokens of every
   // sequence are left out (block_tables then points tok_offset / block_size
   // entries into each row, rows table_stride entries apart, max_blocks of

@@ -20,7 +20,8 @@ static int failures = 0;
 int main(void) {
   pa_cache_desc bf16 = {1000, 16, 8, 128, PA_DTYPE_BF16, 1.0f, 1.0f};
   pa_cache_desc f32 = {1000, 16, 8, 128, PA_DTYPE_F32, 1.0f, 1.0f};
-  pa_cache_desc fp8 = {1000, 16, 8, 128, PA_DTYPE_FP8_E4M3, 0.25f, 0.5f};
+  /* FP8 pages with head_dim 64: no compiled kernel */
+  pa_cache_desc fp8_d64 = {1000, 16, 8, 64, PA_DTYPE_FP8_E4M3, 0.25f, 0.5f};
   void *fake = (void *)(size_t)0x10000; /* aligned, never dereferenced */
   int32_t *ifake = (int32_t *)fake;
   size_t ws;
@@ -39,7 +40,7 @@ int main(void) {
   CHECK(pa_decode(NULL, fake, fake, fake, fake, ifake, ifake, 2, 32, 4, 0.1f, fake, ws, NULL,
                   NULL) == PA_ERR_INVALID_ARG);
   CHECK(strlen(pa_last_error_message()) > 0);
-  CHECK(pa_decode_splitk(&fp8, fake, fake, fake, ifake, ifake, 2, 32, 4, 0.1f, 512, 1,
+  CHECK(pa_decode_splitk(&fp8_d64, fake, fake, fake, ifake, ifake, 2, 32, 4, 0.1f, 512, 1,
                          (float *)fake, (float *)fake, (float *)fake, NULL,
                          NULL) == PA_ERR_UNSUPPORTED);
   CHECK(pa_prefill(&f32, fake, fake, fake, fake, ifake, ifake, ifake, 2, 64, 32, 16, 32, 0.1f,

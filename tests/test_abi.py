@@ -98,9 +98,11 @@ def test_splitk_and_reduce_argument_checks(lib):
     # too few partitions for max_blocks * block_size tokens
     assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 64, 0.1, 256, 3, FAKE, FAKE,
              FAKE, None, None) == pa.PA_ERR_INVALID_ARG
-    # more than 1024 blocks in one partition
-    assert f(ctypes.byref(_desc(bs=1)), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4096, 0.1, 2048, 2,
-             FAKE, FAKE, FAKE, None, None) == pa.PA_ERR_UNSUPPORTED
+    # more than 1024 blocks in one partition, on a shape only the partition
+    # kernel serves (fp32 pages with 2 KV heads; the page-stream kernel has no
+    # such limit)
+    assert f(ctypes.byref(_desc(bs=1, hkv=2, dtype=0)), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4096,
+             0.1, 2048, 2, FAKE, FAKE, FAKE, None, None) == pa.PA_ERR_UNSUPPORTED
     r = lib.pa_reduce
     assert r(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 128, 512, 4, 9, None, None) == pa.PA_ERR_INVALID_ARG
     assert r(MISALIGNED, FAKE, FAKE, FAKE, FAKE, 2, 32, 128, 512, 4, 1, None, None) == \
@@ -185,10 +187,12 @@ def test_fp8_argument_checks_need_no_device(lib):
     assert _decode(lib, _fp8(hkv=2), Hq=4) == pa.PA_ERR_UNSUPPORTED
     assert _decode(lib, _fp8(hkv=4), Hq=64) == pa.PA_ERR_UNSUPPORTED
     assert b"FP8" in lib.pa_last_error_message()
-    # split-K partials and the shared-prefix call take bf16 / fp32 pages only
+    # split-K partials of FP8 pages: the page-stream shapes only; the
+    # shared-prefix call takes bf16 pages only
     P = 8
-    assert lib.pa_decode_splitk(ctypes.byref(_fp8()), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4,
+    assert lib.pa_decode_splitk(ctypes.byref(_fp8(hkv=2)), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 4,
                                 0.1, 16, P, FAKE, FAKE, FAKE, None, None) == pa.PA_ERR_UNSUPPORTED
+    assert b"FP8" in lib.pa_last_error_message()
     assert lib.pa_decode_shared_prefix(ctypes.byref(_fp8()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                                        2, 32, 4, 1, 0.1, FAKE, 1 << 30, None,
                                        None) == pa.PA_ERR_UNSUPPORTED
@@ -243,8 +247,11 @@ def test_noalloc_refuses_what_its_scratch_cannot_hold(lib):
     assert f(ctypes.byref(desc), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 128, 4096, 0.1,
              None, None) == pa.PA_ERR_UNSUPPORTED
     assert b"scratch" in lib.pa_last_error_message()
-    # 64 query heads fit, but not with a million sequences' counters
-    assert f(ctypes.byref(desc), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, 64, 4096, 0.1,
+    # the partition kernel's workspace grows with batch x partitions: fp32
+    # pages with 2 KV heads (a shape the page-stream kernel does not serve),
+    # 8 sequences of up to 131072 tokens need 512 partials per row
+    fp32 = _desc(nb=1000, bs=32, hkv=2, d=128, dtype=0)
+    assert f(ctypes.byref(fp32), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 32, 4096, 0.1,
              None, None) == pa.PA_ERR_UNSUPPORTED
     assert b"scratch" in lib.pa_last_error_message()
 
