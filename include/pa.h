@@ -400,7 +400,8 @@ pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
  * partition is non-empty or when any of them has part_sum < 0 (a bad
  * block id upstream).  A context length < 0 or past max_partitions *
  * partition_tokens sets PA_DEVERR_CONTEXT_LEN and gives zeros.  out has
- * dtype `out_dtype`.
+ * dtype `out_dtype`.  head_dim a multiple of 4, at most 1024; up to about
+ * 56000 partitions (else PA_ERR_UNSUPPORTED).
  */
 pa_status pa_reduce(void *out, const float *part_max, const float *part_sum,
                     const float *part_out, const int32_t *context_lens,
