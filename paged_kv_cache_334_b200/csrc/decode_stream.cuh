@@ -156,6 +156,10 @@ struct alignas(16) Shared {
   int64_t P_begin;
   int64_t range[2];  // split-K: this CTA's pages [range[0], range[1]) of the stream
   int32_t s_begin, vlb_begin, abort_flag, pad;
+  // pa_decode mode, when the CTA's first sequence began in an earlier CTA:
+  // the CTA holding its first page and that CTA's partial slot for it
+  // (worked out in the prologue, so the producer divides nothing)
+  int32_t first_cfirst, first_fslot, pad3[2];
   // Batches of up to kSeqCache sequences: context lengths and new-token
   // slots read once by the prologue, so that the producer never waits on a
   // global load of them behind its own bulk copies.
@@ -986,7 +990,7 @@ struct PageWalker {
   // cached context lengths (nothing is prefetched without the cache).
   __device__ __forceinline__ void prefetch_next_window(const Params &p, int64_t end,
                                                        int lane) {
-    const int32_t blocks = (ctx_s + p.block_size - 1) / p.block_size;
+    const int32_t blocks = (ctx_s + p.block_size - 1) >> (p.log2_vbs + p.log2_vpp);
     if (tw_lb + 32 < blocks) {
       tn_seq = s;
       tn_lb = tw_lb + 32;
@@ -1265,6 +1269,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       sh.s_begin = tid;
       sh.vlb_begin = (int32_t)(start - P);
       sh.P_begin = P;
+      if (!splitk && P < start) {
+        const int32_t cf = owner_of(P, Tp, g_eff);
+        sh.first_cfirst = cf;
+        sh.first_fslot = ((int64_t)cf * Tp / g_eff < P) ? 1 : 0;
+      }
     }
   } else {
     int64_t T_loc = 0;
@@ -1318,6 +1327,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           sh.s_begin = s;
           sh.vlb_begin = (int32_t)(start - P);
           sh.P_begin = P;
+          if (!splitk && P < start) {
+            const int32_t cf = owner_of(P, Tp, g_eff);
+            sh.first_cfirst = cf;
+            sh.first_fslot = ((int64_t)cf * Tp / g_eff < P) ? 1 : 0;
+          }
         }
         run += tot;
         if (run > start) break;  // uniform: every thread sees the same `run`
@@ -1338,11 +1352,19 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
               lane);
       bool ok = true;
       int issued = 0;
+      // split-K: the partition of the current page and the pages left in it
+      // (CTA ranges start on partition boundaries), kept without a division
+      int32_t u_cur = pp > 0 ? sh.vlb_begin / pp : 0, u_left = pp;
+      // stage slot and how many times the ring went round (no divisions)
+      int slot = -1, round = 0;
       for (int i = 0; i < n_stages && ok; ++i) {
-        const int slot = i % p.stages;
-        if (i >= p.stages) {
+        if (++slot == p.stages) {
+          slot = 0;
+          ++round;
+        }
+        if (round > 0) {
           ok = __all_sync(0xffffffffu,
-                          mbar_wait(&sh.empty[slot], ((i / p.stages) - 1) & 1, &sh.abort_flag));
+                          mbar_wait(&sh.empty[slot], (round - 1) & 1, &sh.abort_flag));
           if (!ok) break;
         }
         const int npg = (int)min((int64_t)p.pps, end - wk.cursor);
@@ -1354,8 +1376,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           const bool first = (wk.vlb == 0) || (wk.cursor == start);
           const bool seq_last = wk.vlb == wk.pages_s - 1;
           // split-K: a partition ends every pp pages (ranges end on unit ends)
-          const bool last = seq_last || (wk.cursor == end - 1) ||
-                            (pp > 0 && (wk.vlb + 1) % pp == 0);
+          const bool last = seq_last || (wk.cursor == end - 1) || u_left == 1;
           const bool bad_block = pb < 0 || pb >= p.num_blocks;
           bool bad = bad_block;
           if (bad_block && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
@@ -1380,24 +1401,25 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             PageDesc d;
             d.seq = wk.s;
             d.ntok = ntok;
-            d.unit = pp > 0 ? wk.vlb / (int32_t)pp : 0;
+            d.unit = u_cur;
             d.pb = pb;
             d.toff = (wk.vlb & ((1 << p.log2_vpp) - 1)) * p.vbs;
             d.pad0 = d.pad1 = 0;
             int32_t flags = (first ? kFirst : 0) | (last ? kLast : 0) | (bad ? kBad : 0);
             if (last && pp == 0) {
-              // is the sequence cut between CTAs?  Then this CTA leaves a
-              // partial in its slot 0 (the sequence holds the CTA's first
-              // page) or 1 (it starts inside the range and runs past it).
-              const int32_t c_first = owner_of(wk.P_s, Tp, g_eff);
-              const int32_t c_last = owner_of(wk.P_s + wk.pages_s - 1, Tp, g_eff);
-              const int64_t st_first = (int64_t)c_first * Tp / g_eff;
-              if (c_last > c_first) flags |= kCut | ((start < wk.P_s) ? kSlot1 : 0);
-              if (c == c_last) {
+              // is the sequence cut between CTAs (it began before this CTA's
+              // range or runs past it)?  Then this CTA leaves a partial in
+              // its slot 0 (the sequence holds the CTA's first page) or 1
+              // (it starts inside the range and runs past it).
+              const bool before = wk.P_s < start;
+              if (before || !seq_last) flags |= kCut | ((start < wk.P_s) ? kSlot1 : 0);
+              if (seq_last) {
                 // the owner of the sequence's last page tells the merge kernel
-                // where the partials are (or that there is nothing to merge)
-                reinterpret_cast<int4 *>(p.seq_merge)[wk.s] = make_int4(
-                    c_first, c_last - c_first + 1, (st_first < wk.P_s) ? 1 : 0, 0);
+                // where the partials are (or that there is nothing to merge);
+                // only the CTA's first sequence can have begun earlier
+                reinterpret_cast<int4 *>(p.seq_merge)[wk.s] =
+                    before ? make_int4(sh.first_cfirst, c - sh.first_cfirst + 1, sh.first_fslot, 0)
+                           : make_int4(c, 1, 0, 0);
               }
             }
             d.flags = flags;
@@ -1407,7 +1429,17 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             bytes += p.tile ? 2u * (uint32_t)nbox * (uint32_t)p.box_bytes
                             : 2u * (uint32_t)ntok * (uint32_t)p.row_bytes;
           if (first) bytes += (uint32_t)p.q_bytes;
+          const int32_t s_before = wk.s;
           wk.advance(p, end, lane);
+          if (pp > 0) {
+            if (wk.s != s_before) {
+              u_cur = 0;
+              u_left = pp;
+            } else if (--u_left == 0) {
+              ++u_cur;
+              u_left = pp;
+            }
+          }
         }
         __syncwarp();
         // the rows written above are read back by this stage's copies
@@ -1477,10 +1509,13 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
       if constexpr (kMma) cs.scale_log2_ = p.scale_log2;
       float *sc_buf = s_scores + (size_t)cw_idx * kScoreFloats;
       int64_t cursor = start;
+      int slot = -1, round = 0;  // stage slot and ring round, as the producer's
       for (int i = 0; i < n_stages; ++i) {
-        const int slot = i % p.stages;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sh.full[slot], (i / p.stages) & 1,
-                                               &sh.abort_flag))) {
+        if (++slot == p.stages) {
+          slot = 0;
+          ++round;
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&sh.full[slot], round & 1, &sh.abort_flag))) {
           if (lane == 0) {
             sh.abort_flag = 1;
             set_error(p.err_word, PA_DEVERR_TIMEOUT);
@@ -1651,6 +1686,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Para
   const int hq0 = (blockIdx.x % slices) * p.heads_per_warp;
   const int4 md = __ldcg(reinterpret_cast<const int4 *>(p.seq_merge) + seq);
   const int n = md.y;
+  if (n <= 1) return;  // empty, or written directly by its only CTA
   const int first_slot = md.z;
   const int64_t orow = (int64_t)seq * p.num_q_heads + hq0;
   // thread -> 4 consecutive outputs (head, d .. d+3) of this slice
