@@ -384,15 +384,14 @@ def ceilings(w, flops: float, nbytes: float, launch_us: float, sm_mhz: float) ->
     return out
 
 
-def parity_sample(w, out_rows: np.ndarray, nb: int) -> dict:
+def parity_sample(w, out_rows: np.ndarray, idx) -> dict:
     """Max / mean absolute difference between the timed call's output rows of
-    the first nb sequences (out_rows, float64) and the oracle's write then
-    decode of those sequences, with the tolerance of the workload's dtype.
-    The write is idempotent, so the workload's host pool may already hold
-    it."""
+    the sequences `idx` (out_rows, float64, in that order) and the oracle's
+    write then decode of those sequences, with the tolerance of the
+    workload's dtype.  The write is idempotent, so the workload's host pool
+    may already hold it."""
     import oracle
-    nb = max(1, min(nb, w.batch))
-    s = _prefix(w, nb)
+    s = _subset(w, idx)
     scale = 1.0 / math.sqrt(w.head_dim)
     kc, vc = s.key_cache, s.value_cache
     if w.dtype == wl.DTYPE_FP8:
@@ -405,13 +404,21 @@ def parity_sample(w, out_rows: np.ndarray, nb: int) -> dict:
         if s.slot_mapping is not None:
             oracle.write_kv_cache(kc, vc, s.k_new, s.v_new, s.slot_mapping)
         ref, flags = oracle.decode(s.q, kc, vc, s.block_tables, s.context_lens, scale)
-    err = np.abs(np.asarray(out_rows[:nb], dtype=np.float64) - ref)
+    err = np.abs(np.asarray(out_rows, dtype=np.float64) - ref)
     tol_max, tol_mean = (1e-5, None) if w.dtype == wl.DTYPE_F32 else (2e-2, 1e-2)
     finite = bool(np.isfinite(err).all())
     ok = finite and not flags.any() and err.max() <= tol_max and (
         tol_mean is None or err.mean() <= tol_mean)
-    return {"max_abs": float(err.max()), "mean_abs": float(err.mean()), "sequences": nb,
+    return {"max_abs": float(err.max()), "mean_abs": float(err.mean()),
+            "sequences": [int(i) for i in idx],
             "tolerance": {"max_abs": tol_max, "mean_abs": tol_mean}, "within": bool(ok)}
+
+
+def parity_indices(batch: int, n: int = 12):
+    """n sequences spread over the batch (its first and last included), so
+    that sequences cut between CTAs and sequences kept whole are both
+    checked."""
+    return sorted(set(int(round(x)) for x in np.linspace(0, batch - 1, min(n, batch))))
 
 
 def timing_stats(ms) -> dict:
@@ -437,6 +444,20 @@ def _oracle_step(w) -> float:
         oracle.write_kv_cache(kc, vc, w.k_new, w.v_new, w.slot_mapping)
     oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens, scale)
     return time.perf_counter() - t0
+
+
+def _subset(w, idx):
+    """The workload restricted to sequences idx (same pool)."""
+    import dataclasses
+    idx = np.asarray(idx, dtype=np.int64)
+    keep = w.slot_mapping is not None
+    # the bench workloads have a new token in every sequence: row b is b's
+    assert not keep or w.slot_mapping.shape[0] == w.batch
+    return dataclasses.replace(
+        w, batch=len(idx), q=w.q[idx].copy(), block_tables=w.block_tables[idx].copy(),
+        context_lens=w.context_lens[idx].copy(),
+        k_new=w.k_new[idx].copy() if keep else None, v_new=w.v_new[idx].copy() if keep else None,
+        slot_mapping=w.slot_mapping[idx].copy() if keep else None)
 
 
 def _prefix(w, nb):
@@ -675,7 +696,8 @@ def measure_decode(args, name, dev, dist, rank, world, baseline=True):
         if baseline and not args.no_cpu_baseline:
             cpu = cpu_baseline(w, args.cpu_seconds)
         # the timed call's output rows of the first sequences against the oracle
-        parity = parity_sample(w, out[:8].double().cpu().numpy(), 8)
+        pidx = parity_indices(w.batch)
+        parity = parity_sample(w, out[pidx].double().cpu().numpy(), pidx)
 
     peak, peak_src = hbm_peak()
     achieved = dec_bytes / (t_dec * 1e-3) / 1e9

@@ -327,10 +327,19 @@ pa_status pa_prefill(const pa_cache_desc *cache, void *out, const void *q,
  * GPU that loads the library holds it until the process exits.  This call
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  *
- * - Limit: when pa_decode_workspace_bytes(cache, batch, num_q_heads,
- *   max_blocks_per_seq) exceeds PA_DECODE_NOALLOC_SCRATCH_BYTES the call
- *   returns PA_ERR_UNSUPPORTED (see pa_last_error_message) and enqueues no
- *   work; use pa_decode with a workspace for such sizes.
+ * - Kernels: those of pa_decode, except that bf16 caches with 64 or 128
+ *   query heads per KV head run on the page-stream kernel (16 query heads
+ *   per consumer warp) instead of the tensor-core tile kernel, whose scratch
+ *   (per-row results of the whole batch) would not fit.
+ * - Limit: the call needs the scratch pa_decode needs on those kernels.
+ *   That is pa_decode_workspace_bytes(cache, batch, num_q_heads,
+ *   max_blocks_per_seq) for every shape except the 64 / 128 query-head
+ *   groups above, where it is the page-stream kernel's fixed per-SM
+ *   partials, 2 * 192 * num_q_heads * (head_dim + 2) * 4 bytes plus 16
+ *   bytes per sequence (about 12.8 MB at 64 heads of head_dim 128).  When it
+ *   exceeds PA_DECODE_NOALLOC_SCRATCH_BYTES the call returns
+ *   PA_ERR_UNSUPPORTED (see pa_last_error_message) and enqueues no work; use
+ *   pa_decode with a workspace for such sizes.
  * - Set-up: the first call on a device looks up the array's device address
  *   for that device (the calling thread's current device) and remembers it.
  *   Make that first call on each device before any stream capture.

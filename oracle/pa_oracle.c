@@ -129,8 +129,13 @@ void orc_widen(const void *src, int dtype, int64_t n, double *dst) {
   for (int64_t i = 0; i < n; ++i) dst[i] = orc_load(src, i, dtype);
 }
 
-/* The address mapping of one logical token.  Returns 0, or a flag if the
- * logical block is past max_blocks or the physical id is out of range. */
+/* The address mapping of one logical token.  This is the definition the
+ * teaching page gives (section "From logical token to physical block": the
+ * logical block is the token index divided by the block size, the offset
+ * its remainder, the physical block the table's entry), written out from
+ * that statement in this file's own terms; the gather below applies it per
+ * token in logical order.  Returns 0, or a flag if the logical block is
+ * past max_blocks or the physical id is out of range. */
 int orc_map_token(const int32_t *block_table, int32_t max_blocks,
                   int32_t num_blocks, int32_t block_size, int64_t token_index,
                   int32_t *physical_block_id, int32_t *block_offset) {

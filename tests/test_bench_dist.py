@@ -154,13 +154,21 @@ def test_parity_sample_against_the_oracle():
             oracle.write_kv_cache(kc, vc, w.k_new, w.v_new, w.slot_mapping)
             ref, _ = oracle.decode(w.q, kc, vc, w.block_tables, w.context_lens,
                                    1.0 / math.sqrt(w.head_dim))
-        rec = bench.parity_sample(w, ref, 2)
-        assert rec["max_abs"] == 0.0 and rec["within"] and rec["sequences"] == 2
+        idx = bench.parity_indices(w.batch)
+        assert idx == [0, 1, 2]
+        rec = bench.parity_sample(w, ref[idx], idx)
+        assert rec["max_abs"] == 0.0 and rec["within"] and rec["sequences"] == idx
+        # rows of any subset, in the subset's order
+        rec = bench.parity_sample(w, ref[[2, 0]], [2, 0])
+        assert rec["max_abs"] == 0.0 and rec["within"]
         bad = ref.copy()
         bad[1, 3, 5] += 0.05
-        rec = bench.parity_sample(w, bad, 2)
+        rec = bench.parity_sample(w, bad[idx], idx)
         assert abs(rec["max_abs"] - 0.05) < 1e-12 and not rec["within"]
         assert rec["tolerance"] == {"max_abs": 2e-2, "mean_abs": 1e-2}
+    # spread over a large batch, ends included
+    idx = bench.parity_indices(128)
+    assert idx[0] == 0 and idx[-1] == 127 and len(idx) == 12
 
 
 def test_prefill_parity_record():

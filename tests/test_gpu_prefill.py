@@ -3,7 +3,7 @@ against the fp64 oracle's prefill of the same inputs: whole prompts and later
 chunks of ragged lengths across the 128-row and 128-token tiles, every GQA
 group width the kernel serves, head_dim 64 and 128, pages of 8 to 128
 tokens, NaN in every slot past a context, sampled rows of 2048-token
-prompts, and each flagged case.  Named to run after the other GPU tests.
+prompts, and each flagged case.
 
 Tolerance: bf16, <= 2e-2 max-abs and <= 1e-2 mean-abs (as for pa_decode).
 """
