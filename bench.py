@@ -79,6 +79,9 @@ def parse_args(argv=None):
                          "own key of the same JSON line (default: the bf16 GQA batch, the "
                          "other configuration the target names); 'none' skips it")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="the workload's first BATCH sequences only (smaller captures for "
+                         "profiling; not a headline configuration)")
     ap.add_argument("--block-size", type=int, default=None,
                     help="page size override for gqa_bf16 / mixed_bf16 / long_bf16 (a sweep)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -493,7 +496,8 @@ def run_reference(args):
     world, rank, local = dist_env()
     if rank != 0:
         return 0
-    w = wl.make_workload(args.workload, seed=args.seed, block_size=args.block_size)
+    w = wl.make_workload(args.workload, seed=args.seed, batch=args.batch,
+                         block_size=args.block_size)
     nbytes_full = wl.roofline_bytes(w)
     budget = max(2.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     per_step, sample, cores, desc = time_oracle(w, budget, max_reps=1)
@@ -529,7 +533,8 @@ def measure_decode(args, name, dev, dist, rank, world, baseline=True):
     import torch
     from paged_kv_cache_334_b200 import pa
 
-    w = wl.make_workload(name, seed=rank_seed(args.seed, rank), block_size=args.block_size)
+    w = wl.make_workload(name, seed=rank_seed(args.seed, rank), batch=args.batch,
+                         block_size=args.block_size)
 
     def dev_t(a):
         t = torch.from_numpy(np.ascontiguousarray(a))
