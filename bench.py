@@ -59,8 +59,9 @@ METRIC = "decode-attention KV GB/s & fraction of B200 HBM peak; seq-tokens/s per
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "paged_kv_cache_334_b200", "csrc")
 # sources that define the decode kernel's code and launch shape
-DECODE_SOURCES = ("decode_stream.cuh", "decode_stream_bf16.cu", "decode_stream_f32.cu", "sm100_ptx.cuh",
-                  "pa_common.cuh", "pa_launch.h", "api.cu")
+DECODE_SOURCES = ("decode_stream.cuh", "decode_stream_bf16.cu", "decode_stream_f32.cu",
+                  "decode_stream_fp8.cu", "reduce.cu", "sm100_ptx.cuh", "pa_common.cuh",
+                  "pa_launch.h", "api.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.md")
 
 
@@ -290,8 +291,9 @@ def decode_source_hash() -> str:
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel sources for this workload; else None."""
+    """DRAM bytes per decode call (all its kernels) from the committed ncu
+    summary, if it was taken on the current kernel sources for this workload
+    (`<workload>/splitk` for the split-K step); else None."""
     try:
         text = open(TRAFFIC_FILE).read()
     except OSError:
@@ -725,8 +727,8 @@ def measure_decode(args, name, dev, dist, rank, world, baseline=True):
                                  (clk or {}).get("sm_mhz") or 1965.0),
         }
     traffic = None
-    if args.block_size is None and not splitk and not prefix:
-        traffic = recorded_traffic(name)
+    if args.block_size is None and args.batch is None and not prefix:
+        traffic = recorded_traffic(name + ("/splitk" if splitk else ""))
     config = workload_config(w, args)
     if splitk:
         config["partitions"] = {"tokens": P, "max_partitions": maxp,
