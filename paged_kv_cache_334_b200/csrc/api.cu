@@ -112,8 +112,7 @@ struct StreamPlan {
   int32_t vbs, log2_vbs, log2_vpp, row_bytes, row_pitch, vpage_stride, q_bytes, pps, stages,
       stage_bytes, box_bytes, n_dhalf;
   int32_t heads_per_warp, warps_per_kv;
-  bool fp8;               // E4M3 pages, converted to bf16 by the consumers
-  int32_t scratch_bytes;  // fp8: the bf16 page the consumers convert into
+  bool fp8;               // E4M3 pages: fp16 fragments built from the codes
   size_t smem;
 };
 
@@ -129,7 +128,7 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   s.ok = false;
   const int32_t hkv = c->num_kv_heads;
   const int32_t group = num_q_heads / hkv;
-  // fp8 pages take the bf16 tensor-core consumers after a conversion
+  // fp8 pages take the token-row tensor-core consumers (fp16 fragments)
   const bool fp8 = c->dtype == PA_DTYPE_FP8_E4M3;
   const bool bf16 = c->dtype == PA_DTYPE_BF16 || fp8;
   s.fp8 = fp8;
@@ -161,8 +160,7 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   if (s.row_bytes + 16 > st::kVPageBytes) return s;
   int32_t rows = st::kVPageBytes / s.row_bytes;  // power of two
   if (fp8) {
-    // 16-token virtual pages (one MMA tile), each warp alone on its KV
-    // head's rows of the converted page (a warp never shares them)
+    // 16-token virtual pages (one MMA tile), one warp per KV head
     if (c->block_size < 16 || (hkv != 4 && hkv != 8) || s.warps_per_kv != 1 ||
         s.heads_per_warp > 8)
       return s;
@@ -191,10 +189,7 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   if (s.pps > st::kMaxPPS) s.pps = st::kMaxPPS;
   if (s.pps < 1) s.pps = 1;
   if (fp8 && !s.tile) return s;
-  // fp8: a bf16 page (K and V, every 64-wide half of D) to convert into
-  s.scratch_bytes = fp8 ? 2 * s.n_dhalf * s.box_bytes : 0;
-  const int32_t avail =
-      st::kSmemLimit - st::kHdrBytes - 1024 - s.scratch_bytes;  // 1 KB alignment slack
+  const int32_t avail = st::kSmemLimit - st::kHdrBytes - 1024;  // 1 KB alignment slack
   for (;;) {
     s.stage_bytes = (int32_t)(((size_t)2 * s.pps * s.vpage_stride + (size_t)s.pps * s.q_bytes +
                                1023) / 1024 * 1024);
@@ -204,7 +199,7 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
     --s.pps;
   }
   if (s.stages < 2) return s;
-  s.smem = (size_t)st::kHdrBytes + 1024 + (size_t)s.stages * s.stage_bytes + s.scratch_bytes;
+  s.smem = (size_t)st::kHdrBytes + 1024 + (size_t)s.stages * s.stage_bytes;
   s.ok = true;
   return s;
 }

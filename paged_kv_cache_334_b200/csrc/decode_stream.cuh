@@ -167,14 +167,30 @@ struct alignas(16) Shared {
   int32_t ctx_c[kSeqCache];
 };
 
+// E4M3 codes to fp16 holding code value * 2^-8: the code's sign bit becomes
+// bit 15 and its 7 other bits bits 7..13 -- exact for every code, subnormals
+// included, by integer operations only (no conversion instructions).  Four
+// codes (bytes 0..3 of x) give two fp16 pairs: codes 0, 1 in lo, 2, 3 in hi.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t &lo, uint32_t &hi) {
+  const uint32_t a = __byte_perm(x, 0u, 0x1404);  // codes 0, 1 in the high byte of each half
+  const uint32_t b = __byte_perm(x, 0u, 0x3424);  // codes 2, 3
+  lo = (a & 0x80008000u) | ((a >> 1) & 0x3f803f80u);
+  hi = (b & 0x80008000u) | ((b >> 1) & 0x3f803f80u);
+}
+
 // ===========================================================================
 // bf16 consumer: tensor-core tiles of 16 tokens x 8 query heads.
 // Lane (g = lane / 4, t = lane % 4) holds, for each 16-token tile, the scores
 // of tokens g and g + 8 for query heads 2t and 2t + 1, and for each 16-wide
 // d tile the output accumulator of d = 16 dt + g (+8) for the same two heads.
 // ===========================================================================
-// F16: fp16 tiles (FP8 pages, converted to fp16 by the consumers), with q
-// and P in fp16; else bf16.
+// F16: FP8 pages.  The tensor-core fragments are built in registers from the
+// staged codes (fp16 values holding code * 2^-8, see e4m3x4_to_f16x4), with q
+// and P in fp16.  Inside the products head_dim is taken in another order, so
+// that each lane reads whole 16-byte chunks of codes: in S = q K^T quad lane t
+// owns d = 32t .. 32t + 31 (k step ks: d = 32t + 4ks + 0..3, q taken in the
+// same order); in O^T the rows g and g + 8 of d tile k are d = 16g + 2k and
+// 16g + 2k + 1.  The flush stores natural order.  Else bf16 tiles.
 template <int D, bool F16 = false>
 struct MmaConsumer {
   static constexpr int KS = D / 16;  // k steps of QK, d tiles of PV
@@ -218,8 +234,13 @@ struct MmaConsumer {
     for (int k = 0; k < KS; ++k) {
       if (g < nh) {
         const uint32_t *row = reinterpret_cast<const uint32_t *>(qs + (size_t)(hq0 + g) * D);
-        qb[k][0] = q_pair(row[(k * 16 + t * 2) >> 1]);
-        qb[k][1] = q_pair(row[(k * 16 + t * 2 + 8) >> 1]);
+        if constexpr (F16) {
+          qb[k][0] = q_pair(row[(t * (D / 4) + 4 * k) >> 1]);
+          qb[k][1] = q_pair(row[(t * (D / 4) + 4 * k + 2) >> 1]);
+        } else {
+          qb[k][0] = q_pair(row[(k * 16 + t * 2) >> 1]);
+          qb[k][1] = q_pair(row[(k * 16 + t * 2 + 8) >> 1]);
+        }
       } else {
         qb[k][0] = qb[k][1] = 0u;
       }
@@ -364,6 +385,92 @@ struct MmaConsumer {
       page_t<false>(kp, vp, ntok, p, h, col_bytes, lane);
   }
 
+  // FP8 pages (F16, head_dim 128): one 16-token page of E4M3 codes, K and V
+  // each one box of [KV head][16 tokens][128 codes] with the 128-byte swizzle
+  // (16-byte chunk c of row r at chunk c ^ (r % 8)).  The fragments come
+  // straight from the codes: for S a lane reads d chunks 2t, 2t + 1 of tokens
+  // g and g + 8; for O^T d chunk g of tokens 2t, 2t + 1, 2t + 8, 2t + 9,
+  // pairing the two tokens of each fragment register with a byte permute.
+  __device__ __forceinline__ void page_codes(const unsigned char *kp, const unsigned char *vp,
+                                             int ntok, int h, int lane) {
+    static_assert(D == 128, "FP8 pages: head_dim 128");
+    const int g = lane >> 2, t = lane & 3;
+    const unsigned char *kr = kp + (h * 16 + g) * 128;  // token g; token g + 8 is 1 KB on
+    const int c0 = ((2 * t) ^ g) << 4, c1 = ((2 * t + 1) ^ g) << 4;
+    const uint4 ka0 = *reinterpret_cast<const uint4 *>(kr + c0);
+    const uint4 ka1 = *reinterpret_cast<const uint4 *>(kr + c1);
+    const uint4 kb0 = *reinterpret_cast<const uint4 *>(kr + 1024 + c0);
+    const uint4 kb1 = *reinterpret_cast<const uint4 *>(kr + 1024 + c1);
+    const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
+    const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      uint32_t a[4];
+      e4m3x4_to_f16x4(wa[k], a[0], a[2]);
+      e4m3x4_to_f16x4(wb[k], a[1], a[3]);
+      mma((k & 1) ? sb : sa, a, qb[k][0], qb[k][1]);
+    }
+    const bool v0 = g < ntok, v1 = g + 8 < ntok;
+    const float s0 = v0 ? (sa[0] + sb[0]) * scale_log2_ : -INFINITY;
+    const float s1 = v0 ? (sa[1] + sb[1]) * scale_log2_ : -INFINITY;
+    const float s2 = v1 ? (sa[2] + sb[2]) * scale_log2_ : -INFINITY;
+    const float s3 = v1 ? (sa[3] + sb[3]) * scale_log2_ : -INFINITY;
+    float x0 = fmaxf(s0, s2), x1 = fmaxf(s1, s3);
+#pragma unroll
+    for (int mask = 4; mask < 32; mask <<= 1) {
+      x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, mask));
+      x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, mask));
+    }
+    const float n0 = fmaxf(m0_, x0), n1 = fmaxf(m1_, x1);
+    const float a0 = ex2(m0_ - n0), a1 = ex2(m1_ - n1);
+    m0_ = n0;
+    m1_ = n1;
+    const float p0 = ex2(s0 - n0), p1 = ex2(s1 - n1);
+    const float p2 = ex2(s2 - n0), p3 = ex2(s3 - n1);
+    l0 = l0 * a0 + (p0 + p2);
+    l1 = l1 * a1 + (p1 + p3);
+    // P^T (16 tokens x 8 heads) as the B operand
+    const uint32_t pb0 = movmatrix_trans(pack(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(pack(p2, p3));
+    if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        o[k][0] *= a0;
+        o[k][1] *= a1;
+        o[k][2] *= a0;
+        o[k][3] *= a1;
+      }
+    }
+    // tokens past ntok may hold anything: their V codes are zeroed (P is 0)
+    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+    if (ntok < 16) {
+      mlo = (2 * t < ntok ? 0x0000ffffu : 0u) | (2 * t + 1 < ntok ? 0xffff0000u : 0u);
+      mhi = (2 * t + 8 < ntok ? 0x0000ffffu : 0u) | (2 * t + 9 < ntok ? 0xffff0000u : 0u);
+    }
+    const unsigned char *vr = vp + (h * 16 + 2 * t) * 128;
+    const int e0 = (g ^ (2 * t)) << 4, e1 = (g ^ (2 * t + 1)) << 4;
+    const uint4 vx = *reinterpret_cast<const uint4 *>(vr + e0);          // token 2t
+    const uint4 vy = *reinterpret_cast<const uint4 *>(vr + 128 + e1);    // 2t + 1
+    const uint4 vz = *reinterpret_cast<const uint4 *>(vr + 1024 + e0);   // 2t + 8
+    const uint4 vw = *reinterpret_cast<const uint4 *>(vr + 1152 + e1);   // 2t + 9
+    const uint32_t xs[4] = {vx.x, vx.y, vx.z, vx.w}, ys[4] = {vy.x, vy.y, vy.z, vy.w};
+    const uint32_t zs[4] = {vz.x, vz.y, vz.z, vz.w}, ws[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      // codes 2k, 2k + 1 of the chunk (d = 16g + 2k, + 1) of two tokens
+      const uint32_t sel = (k & 1) ? 0x7362u : 0x5140u;
+      uint32_t a[4];
+      e4m3x4_to_f16x4(__byte_perm(xs[k >> 1], ys[k >> 1], sel), a[0], a[1]);
+      e4m3x4_to_f16x4(__byte_perm(zs[k >> 1], ws[k >> 1], sel), a[2], a[3]);
+      a[0] &= mlo;
+      a[1] &= mlo;
+      a[2] &= mhi;
+      a[3] &= mhi;
+      mma(o[k], a, pb0, pb1);
+    }
+  }
+
   // End of a segment: write out[...] directly (n_contrib == 1) or this CTA's
   // normalised partial for the merge kernel.  Two rounds of lane swaps turn
   // the MMA layout into four consecutive d per lane, so that every store
@@ -385,20 +492,48 @@ struct MmaConsumer {
     const int hh = 2 * t + (odd ? 1 : 0);  // head of this lane's values
     // out_scale: 1, or V's scale for FP8 pages (the products saw the codes)
     const float inv = seg_bad ? 0.f : p.out_scale / (odd ? L1 : L0);
-    const int dcol = (g - q) + (q < 2 ? 0 : 8);
+    // this lane's float4 k holds d = dcol + k * dstep .. + 3
+    int dcol, dstep;
     float4 v[KS];
+    if constexpr (F16) {
+      // O^T row pairs: lane g holds d = 16g + 2k, + 1 of heads 2t, 2t + 1;
+      // one exchange (lanes g, g ^ 1) leaves an even-g lane head 2t and an
+      // odd-g lane head 2t + 1, each for d = 16 (g & ~1) .. + 31
+      dcol = 16 * (g & ~1);
+      dstep = 4;
+      float lo[KS][2], hi[KS][2];
 #pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      // first exchange (lanes g, g ^ 1): pairs (d, d + 1) of one head, at +0 and +8
-      const float s0 = __shfl_xor_sync(0xffffffffu, odd ? o[k][0] : o[k][1], 4);
-      const float s2 = __shfl_xor_sync(0xffffffffu, odd ? o[k][2] : o[k][3], 4);
-      const float lo0 = odd ? s0 : o[k][0], lo1 = odd ? o[k][1] : s0;
-      const float hi0 = odd ? s2 : o[k][2], hi1 = odd ? o[k][3] : s2;
-      // second exchange (lanes g, g ^ 2): q < 2 keeps the +0 pairs, q >= 2 the +8 pairs
-      const float r0 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi0 : lo0, 8);
-      const float r1 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi1 : lo1, 8);
-      v[k] = q < 2 ? make_float4(lo0 * inv, lo1 * inv, r0 * inv, r1 * inv)
-                   : make_float4(r0 * inv, r1 * inv, hi0 * inv, hi1 * inv);
+      for (int k = 0; k < KS; ++k) {
+        const float s0 = __shfl_xor_sync(0xffffffffu, odd ? o[k][0] : o[k][1], 4);
+        const float s2 = __shfl_xor_sync(0xffffffffu, odd ? o[k][2] : o[k][3], 4);
+        lo[k][0] = odd ? s0 : o[k][0];
+        lo[k][1] = odd ? s2 : o[k][2];
+        hi[k][0] = odd ? o[k][1] : s0;
+        hi[k][1] = odd ? o[k][3] : s2;
+      }
+#pragma unroll
+      for (int j = 0; j < KS / 2; ++j) {
+        v[j] = make_float4(lo[2 * j][0] * inv, lo[2 * j][1] * inv, lo[2 * j + 1][0] * inv,
+                           lo[2 * j + 1][1] * inv);
+        v[KS / 2 + j] = make_float4(hi[2 * j][0] * inv, hi[2 * j][1] * inv,
+                                    hi[2 * j + 1][0] * inv, hi[2 * j + 1][1] * inv);
+      }
+    } else {
+      dcol = (g - q) + (q < 2 ? 0 : 8);
+      dstep = 16;
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        // first exchange (lanes g, g ^ 1): pairs (d, d + 1) of one head, at +0 and +8
+        const float s0 = __shfl_xor_sync(0xffffffffu, odd ? o[k][0] : o[k][1], 4);
+        const float s2 = __shfl_xor_sync(0xffffffffu, odd ? o[k][2] : o[k][3], 4);
+        const float lo0 = odd ? s0 : o[k][0], lo1 = odd ? o[k][1] : s0;
+        const float hi0 = odd ? s2 : o[k][2], hi1 = odd ? o[k][3] : s2;
+        // second exchange (lanes g, g ^ 2): q < 2 keeps the +0 pairs, q >= 2 the +8 pairs
+        const float r0 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi0 : lo0, 8);
+        const float r1 = __shfl_xor_sync(0xffffffffu, q < 2 ? hi1 : lo1, 8);
+        v[k] = q < 2 ? make_float4(lo0 * inv, lo1 * inv, r0 * inv, r1 * inv)
+                     : make_float4(r0 * inv, r1 * inv, hi0 * inv, hi1 * inv);
+      }
     }
     if (p.sk_o != nullptr) {
       // split-K: this partition's (max, normaliser, normalised output), the
@@ -418,7 +553,7 @@ struct MmaConsumer {
       if (hh < nh) {
 #pragma unroll
         for (int k = 0; k < KS; ++k)
-          *reinterpret_cast<float4 *>(p.sk_o + (row + hh * mp) * D + k * 16 + dcol) = v[k];
+          *reinterpret_cast<float4 *>(p.sk_o + (row + hh * mp) * D + k * dstep + dcol) = v[k];
       }
       return;
     }
@@ -436,14 +571,14 @@ struct MmaConsumer {
         if (hh < nh) {
 #pragma unroll
           for (int k = 0; k < KS; ++k)
-            *reinterpret_cast<float4 *>(p.seq_o + (row + hh) * D + k * 16 + dcol) = v[k];
+            *reinterpret_cast<float4 *>(p.seq_o + (row + hh) * D + k * dstep + dcol) = v[k];
         }
         return;
       }
       if (hh < nh) {
         const int64_t row = ((int64_t)d.seq * p.num_q_heads + hq0 + hh) * D;
 #pragma unroll
-        for (int k = 0; k < KS; ++k) Elem<Tout>::store4(p.out, row + k * 16 + dcol, v[k]);
+        for (int k = 0; k < KS; ++k) Elem<Tout>::store4(p.out, row + k * dstep + dcol, v[k]);
       }
       return;
     }
@@ -459,7 +594,7 @@ struct MmaConsumer {
     if (hh < nh) {
       float *row = p.part_o + (prow + hh) * D;
 #pragma unroll
-      for (int k = 0; k < KS; ++k) *reinterpret_cast<float4 *>(row + k * 16 + dcol) = v[k];
+      for (int k = 0; k < KS; ++k) *reinterpret_cast<float4 *>(row + k * dstep + dcol) = v[k];
     }
     // merged by the last contributing CTA at its end
   }
@@ -1118,42 +1253,6 @@ __device__ __forceinline__ void write_new_rows_fp8(const Params &p, int32_t s, i
   fence_proxy_async_global();
 }
 
-// FP8 pages: this warp's KV-head rows (h * 16 .. + 15) of one staged page,
-// stored as one box of 128 codes per row with the 128-byte swizzle (16-byte
-// chunk c of row r at chunk c ^ (r % 8)), converted into the tile layout the
-// tensor-core consumer reads (64-wide halves of head_dim in boxes box_bytes
-// apart, 8 elements per 16-byte chunk, the same swizzle) as fp16 holding
-// code value * 2^-8: the code's sign bit becomes bit 15 and its 7 other bits
-// bits 7..13 -- exact for every code, subnormals included, by integer
-// operations only (no conversion instructions).
-__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t &lo, uint32_t &hi) {
-  const uint32_t a = __byte_perm(x, 0u, 0x1404);  // codes 0, 1 in the high byte of each half
-  const uint32_t b = __byte_perm(x, 0u, 0x3424);  // codes 2, 3
-  lo = (a & 0x80008000u) | ((a >> 1) & 0x3f803f80u);
-  hi = (b & 0x80008000u) | ((b >> 1) & 0x3f803f80u);
-}
-
-__device__ __forceinline__ void fp8_rows_to_f16(const unsigned char *src, unsigned char *dst,
-                                                int h, const Params &p, int lane) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int k = lane + 32 * i;       // 16 rows x 8 chunks
-    const int r = h * 16 + (k & 15);   // row in the page's box
-    const int c = k >> 4;              // chunk of 16 codes: elements 16c .. 16c + 15
-    const uint4 x = *reinterpret_cast<const uint4 *>(src + r * 128 + ((c ^ (r & 7)) << 4));
-    uint32_t y[8];
-    e4m3x4_to_f16x4(x.x, y[0], y[1]);
-    e4m3x4_to_f16x4(x.y, y[2], y[3]);
-    e4m3x4_to_f16x4(x.z, y[4], y[5]);
-    e4m3x4_to_f16x4(x.w, y[6], y[7]);
-    unsigned char *row = dst + (c >> 2) * p.box_bytes + r * 128;
-    const int j0 = 2 * (c & 3);  // first of the two 16-byte chunks in its half
-    *reinterpret_cast<uint4 *>(row + ((j0 ^ (r & 7)) << 4)) = make_uint4(y[0], y[1], y[2], y[3]);
-    *reinterpret_cast<uint4 *>(row + (((j0 + 1) ^ (r & 7)) << 4)) =
-        make_uint4(y[4], y[5], y[6], y[7]);
-  }
-}
-
 // ===========================================================================
 // The kernel.  T = element type; D = head_dim; G = query heads per KV head
 // for the fp32 consumer; for bf16, G = 16 selects the head-row consumer (16
@@ -1185,8 +1284,6 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   // stages start 1024-byte aligned (the 128-byte swizzle repeats every 1 KB)
   unsigned char *stages =
       smem_raw + (((smem_u32(smem_raw) + p.hdr_bytes + 1023u) & ~1023u) - smem_u32(smem_raw));
-  // FP8 pages: the fp16 page the consumers convert into (K, then V)
-  unsigned char *scratch = stages + (size_t)p.stages * p.stage_bytes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
@@ -1545,23 +1642,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           } else {
             const unsigned char *kp = kst + (size_t)k * p.vpage_stride;
             const unsigned char *vp = vst + (size_t)k * p.vpage_stride;
-            if constexpr (kMma) {
-              if constexpr (kFp8) {
-                // one warp per KV head: its rows of the converted page are its own
-                unsigned char *sk = scratch, *sv = scratch + (size_t)p.n_dhalf * p.box_bytes;
-                fp8_rows_to_f16(kp, sk, h, p, lane);
-                fp8_rows_to_f16(vp, sv, h, p, lane);
-                __syncwarp();
-                // the products read the converted copy: the stage can go back
-                // to the producer after its last page is converted (q, read
-                // at the sequence's first page, is in registers already)
-                if (k == npg - 1) {
-                  if (lane == 0) mbar_arrive(&sh.empty[slot]);
-                  released = true;
-                }
-                kp = sk;
-                vp = sv;
-              }
+            if constexpr (kFp8) {
+              cs.page_codes(kp, vp, d.ntok, h, lane);
+            } else if constexpr (kMma) {
               cs.page(kp, vp, d.ntok, p, h, col_bytes, lane);
             } else {
               cs.page(kp, vp, d.ntok, p.row_pitch, col_bytes, sc_buf, lane);
