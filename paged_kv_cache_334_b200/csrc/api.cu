@@ -465,10 +465,10 @@ static pa_status stream_params(const pa_cache_desc *cache, const void *q, const 
   p.k_scale = cache->k_scale;
   p.v_scale = cache->v_scale;
   if (fp8) {
-    // the consumers see code value * 2^-8 (exact in fp16): 256 k_scale
-    // goes into the score scale, 256 v_scale into the output
-    p.scale_log2 *= 256.f * cache->k_scale;
-    p.out_scale = 256.f * cache->v_scale;
+    // the consumers see the code values: k_scale goes into the score scale,
+    // v_scale into the output
+    p.scale_log2 *= cache->k_scale;
+    p.out_scale = cache->v_scale;
   }
   p.group = num_q_heads / cache->num_kv_heads;
   p.heads_per_warp = sp.heads_per_warp;

@@ -167,15 +167,14 @@ struct alignas(16) Shared {
   int32_t ctx_c[kSeqCache];
 };
 
-// E4M3 codes to fp16 holding code value * 2^-8: the code's sign bit becomes
-// bit 15 and its 7 other bits bits 7..13 -- exact for every code, subnormals
-// included, by integer operations only (no conversion instructions).  Four
-// codes (bytes 0..3 of x) give two fp16 pairs: codes 0, 1 in lo, 2, 3 in hi.
+// Four E4M3 codes (bytes 0..3 of x) to two fp16 pairs, exactly (every E4M3
+// value, subnormals included, is an fp16 value): codes 0, 1 in lo, 2, 3 in hi,
+// the lower-addressed code in the lower half.
 __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t &lo, uint32_t &hi) {
-  const uint32_t a = __byte_perm(x, 0u, 0x1404);  // codes 0, 1 in the high byte of each half
-  const uint32_t b = __byte_perm(x, 0u, 0x3424);  // codes 2, 3
-  lo = (a & 0x80008000u) | ((a >> 1) & 0x3f803f80u);
-  hi = (b & 0x80008000u) | ((b >> 1) & 0x3f803f80u);
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
 }
 
 // ===========================================================================
@@ -185,8 +184,8 @@ __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t &lo, uint32
 // d tile the output accumulator of d = 16 dt + g (+8) for the same two heads.
 // ===========================================================================
 // F16: FP8 pages.  The tensor-core fragments are built in registers from the
-// staged codes (fp16 values holding code * 2^-8, see e4m3x4_to_f16x4), with q
-// and P in fp16.  Inside the products head_dim is taken in another order, so
+// staged codes (their exact fp16 values, see e4m3x4_to_f16x4), with q and P
+// in fp16.  Inside the products head_dim is taken in another order, so
 // that each lane reads whole 16-byte chunks of codes: in S = q K^T quad lane t
 // owns d = 32t .. 32t + 31 (k step ks: d = 32t + 4ks + 0..3, q taken in the
 // same order); in O^T the rows g and g + 8 of d tile k are d = 16g + 2k and
@@ -1449,6 +1448,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
               lane);
       bool ok = true;
       int issued = 0;
+      // pages are read once: they go to L2 with evict-first priority, so that
+      // the block tables, the partials and the merge records stay there
+      const uint64_t kv_policy = l2_evict_first_policy();
       // split-K: the partition of the current page and the pages left in it
       // (CTA ranges start on partition boundaries), kept without a division
       int32_t u_cur = pp > 0 ? sh.vlb_begin / pp : 0, u_left = pp;
@@ -1554,9 +1556,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             if (lane < 2 * nbox) {
               const int dh = lane % nbox;
               const bool isv = lane >= nbox;
-              tma_load_3d((isv ? vst : kst) + (size_t)k * p.vpage_stride + (size_t)dh * p.box_bytes,
-                          isv ? &p.tmap_v : &p.tmap_k, dh * 64, d.pb * p.block_size + d.toff, 0,
-                          &sh.full[slot]);
+              tma_load_3d_hint((isv ? vst : kst) + (size_t)k * p.vpage_stride +
+                                   (size_t)dh * p.box_bytes,
+                               isv ? &p.tmap_v : &p.tmap_k, dh * 64, d.pb * p.block_size + d.toff,
+                               0, &sh.full[slot], kv_policy);
             }
           } else if (!(d.flags & kBad)) {
             const int64_t off = ((int64_t)d.pb * p.block_size + d.toff) * (int64_t)p.row_bytes;
@@ -1829,10 +1832,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Para
         reinterpret_cast<float2 *>(p.seq_ml)[orow + h] = make_float2(M, bad ? -1.f : W);
       continue;
     }
-    Elem<Tout>::store1(p.out, e + 0, bad ? 0.f : acc.x * inv);
-    Elem<Tout>::store1(p.out, e + 1, bad ? 0.f : acc.y * inv);
-    Elem<Tout>::store1(p.out, e + 2, bad ? 0.f : acc.z * inv);
-    Elem<Tout>::store1(p.out, e + 3, bad ? 0.f : acc.w * inv);
+    Elem<Tout>::store4(p.out, e,
+                       bad ? make_float4(0.f, 0.f, 0.f, 0.f)
+                           : make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
   }
 }
 

@@ -91,10 +91,9 @@ struct Params {
   int32_t tile;                     // 1: tensor copies of swizzled boxes, else row copies
   int32_t box_bytes;                // bytes of one box (64 x vbs x Hkv bf16)
   int32_t n_dhalf;                  // boxes per page per tensor (head_dim / 64)
-  // FP8 pages: one box of 128 codes x vbs x Hkv per page and tensor, which
-  // the consumers convert into an fp16 page (the tile layout, code value *
-  // 2^-8) after the stages; scale_log2 then includes 256 k_scale and
-  // out_scale is 256 v_scale
+  // FP8 pages: one box of 128 codes x vbs x Hkv per page and tensor, from
+  // which the consumers build fp16 fragments of the code values;
+  // scale_log2 then includes k_scale and out_scale is v_scale
   int32_t fp8;
   float out_scale;
   float k_scale, v_scale;  // FP8 pages: the fused write's quantisation scales
