@@ -964,12 +964,17 @@ def run_prefill(args):
                     "h2d_bytes_per_step": int(e2e[1]), "d2h_bytes_per_step": int(e2e[2]),
                     "ms_per_step": t_e2e_max}
     cpu = parity = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_step, sample, cores, desc = time_oracle_prefill(pw, args.cpu_seconds)
-        cpu = {"value": wl.prefill_flops(sample) / per_step / 1e12, "unit": "TFLOP/s",
-               "cores": cores, "kind": "oracle", "sample": desc,
-               "ms_per_step": per_step * 1e3}
-        parity = prefill_parity(pw, sample, out[:int(pw.chunk_lens[0])].double().cpu().numpy())
+    if rank == 0 and world == 1:
+        rows0 = out[:int(pw.chunk_lens[0])].double().cpu().numpy()
+        if args.no_cpu_baseline:
+            # the call's last rows of sequence 0 against the oracle, untimed
+            sample = prefill_sample(pw, 16)
+        else:
+            per_step, sample, cores, desc = time_oracle_prefill(pw, args.cpu_seconds)
+            cpu = {"value": wl.prefill_flops(sample) / per_step / 1e12, "unit": "TFLOP/s",
+                   "cores": cores, "kind": "oracle", "sample": desc,
+                   "ms_per_step": per_step * 1e3}
+        parity = prefill_parity(pw, sample, rows0)
     tpeak, tpeak_src = tensor_peak()
     hpeak, _ = hbm_peak()
     achieved = flops / (t_call * 1e-3) / 1e12

@@ -19,7 +19,8 @@
 // head), so one K/V read serves the whole GQA group.  It walks the sequence's
 // 128-token K/V tiles up to its last row's position, as a FlashAttention
 // forward pass (online softmax, no score matrix in memory); tiles past a
-// row's position are masked per row.  The later tiles of a sequence do the
+// row's position are masked per row, and the last tile's products stop at
+// the 16-token step that holds the tile's last position.  The later tiles of a sequence do the
 // most work and are launched first.
 //
 //   warp 0     tiled copies (no multicast): the Q tile once, then K and V of
@@ -260,12 +261,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!wait_all(&sh.vfull[vst], (u / kVStages) & 1, sh, p, lane)) return false;
       if (!wait_all(&sh.pfull[x], (u >> 1) & 1, sh, p, lane)) return false;
       const int ntok = tile_tokens(u);
-      if (ntok < kTok) {
-        // V rows past the last position: later slots of the last page (which
-        // may hold anything) and stage memory no page was copied to; their
-        // probabilities are 0, but 0 x NaN is not
+      // K steps of 16 tokens that hold a position <= pos_max; the later ones
+      // (all masked) are skipped
+      const int nks = (ntok + 15) >> 4;
+      if (ntok < 16 * nks) {
+        // V rows past the last position inside the last K step: later slots
+        // of the last page (which may hold anything) or stage memory no page
+        // was copied to; their probabilities are 0, but 0 x NaN is not
         unsigned char *vs = v_stage(vst);
-        const int units = (kTok - ntok) * 8;
+        const int units = (16 * nks - ntok) * 8;
         for (int i = lane; i < units * NH; i += 32) {
           const int dh = i / units, rem = i - dh * units;
           *reinterpret_cast<uint4 *>(vs + dh * kBox + (ntok + (rem >> 3)) * 128 + (rem & 7) * 16) =
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (lane == 0) {
         const uint32_t va = smem_u32(v_stage(vst));
-        for (int ks = 0; ks < kTok / 16; ++ks)
+        for (int ks = 0; ks < nks; ++ks)
           tc_mma_ts(tm + Cols<D>::O, tm + Cols<D>::P + 64 * x + 8 * ks,
                     sw128_desc(va + 2048 * ks, (uint32_t)kBox, 1024), id_o,
                     (u == 0 && ks == 0) ? 0u : 1u);
@@ -300,11 +304,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (lane == 0) {
         const uint32_t qa = smem_u32(qt), ka = smem_u32(k_stage(kst));
+        // the last tile: only its first columns (16 at a time) hold positions
+        // <= pos_max; the rest of S is left as it was and masked by the softmax
+        const int ntok = tile_tokens(t);
+        const uint32_t id_t =
+            ntok < kTok ? idesc_bf16(kRows, (ntok + 15) & ~15, false) : id_s;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32;
           tc_mma_ss(tm + Cols<D>::S + kTok * x, sw128_desc(qa + off, 16, 1024),
-                    sw128_desc(ka + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+                    sw128_desc(ka + off, 16, 1024), id_t, kk > 0 ? 1u : 0u);
         }
         tc_commit(&sh.sfull[x]);
         tc_commit(&sh.kempty[kst]);  // K stage free once S is computed
