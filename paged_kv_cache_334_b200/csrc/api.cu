@@ -113,6 +113,7 @@ struct StreamPlan {
       stage_bytes, box_bytes, n_dhalf;
   int32_t heads_per_warp, warps_per_kv;
   bool fp8;               // E4M3 pages: fp16 fragments built from the codes
+  bool pair;              // 8-token blocks, two per 16-token page (tile path)
   size_t smem;
 };
 
@@ -167,8 +168,15 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
     rows = 16;
   }
   s.vbs = c->block_size < rows ? c->block_size : rows;
+  // 8-token blocks of bf16, head_dim 128, one warp per KV head: pages of two
+  // blocks, so that the tensor-core tiles (16 tokens) and the tiled copies
+  // serve them as they serve 16-token blocks
+  s.pair = allow_tile && !fp8 && bf16 && c->block_size == 8 && rows >= 16 &&
+           c->head_dim == 128 && s.warps_per_kv == 1 && s.heads_per_warp <= 8 &&
+           (hkv == 4 || hkv == 8);
+  if (s.pair) s.vbs = 16;
   s.log2_vbs = ilog2(s.vbs);
-  s.log2_vpp = ilog2(c->block_size / s.vbs);
+  s.log2_vpp = s.pair ? 0 : ilog2(c->block_size / s.vbs);
   s.tile = allow_tile && bf16 && s.vbs >= 16 && hkv <= 256;
   s.n_dhalf = c->head_dim / 64;
   s.box_bytes = 128 * s.vbs * hkv;
@@ -427,8 +435,10 @@ static pa_status stream_params(const pa_cache_desc *cache, const void *q, const 
   const int sms = device_sm_count();
   if (sms <= 0) return fail(PA_ERR_CUDA, "cannot query the device%s");
   pa::stream::Params &p = *pp;
-  if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, sp.vbs) &&
-                   encode_cache_map(&p.tmap_v, value_cache, cache, sp.vbs))) {
+  // boxes of a page's rows of all KV heads (two-block pages: of a block's)
+  const int32_t box_tok = sp.pair ? cache->block_size : sp.vbs;
+  if (sp.tile && !(encode_cache_map(&p.tmap_k, key_cache, cache, box_tok) &&
+                   encode_cache_map(&p.tmap_v, value_cache, cache, box_tok))) {
     if (fp8) return fail(PA_ERR_CUDA, "cannot describe the FP8 caches for the tensor copies%s");
     sp = plan_stream(cache, num_q_heads, /*allow_tile=*/false);
   }
@@ -450,6 +460,8 @@ static pa_status stream_params(const pa_cache_desc *cache, const void *q, const 
   p.vbs = sp.vbs;
   p.log2_vbs = sp.log2_vbs;
   p.log2_vpp = sp.log2_vpp;
+  p.log2_bs = ilog2(cache->block_size);
+  p.pair = sp.pair ? 1 : 0;
   p.row_bytes = sp.row_bytes;
   p.row_pitch = sp.row_pitch;
   p.vpage_stride = sp.vpage_stride;
@@ -979,7 +991,10 @@ pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
                                     context_lens, batch, num_q_heads,
                                     max_blocks_per_seq, scale);
   if (s != PA_OK) return s;
-  const bool streamed = plan_stream(cache, num_q_heads).ok;
+  // the page-stream kernel serves the shape when partitions hold whole
+  // virtual pages (two-block pages of 8-token blocks: 16 tokens)
+  const StreamPlan spl = plan_stream(cache, num_q_heads);
+  const bool streamed = spl.ok && partition_tokens > 0 && partition_tokens % spl.vbs == 0;
   if (cache->dtype == PA_DTYPE_FP8_E4M3 && !streamed)
     return fail(PA_ERR_UNSUPPORTED,
                 "FP8 pages: head_dim 128, block_size >= 16, 4 or 8 KV heads and at most 8 "

@@ -190,7 +190,9 @@ __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t &lo, uint32
 // owns d = 32t .. 32t + 31 (k step ks: d = 32t + 4ks + 0..3, q taken in the
 // same order); in O^T the rows g and g + 8 of d tile k are d = 16g + 2k and
 // 16g + 2k + 1.  The flush stores natural order.  Else bf16 tiles.
-template <int D, bool F16 = false>
+// PAIR: a page is two 8-token blocks, each landed as one box of [KV head][8
+// tokens] rows per d half, the second box after the first.
+template <int D, bool F16 = false, bool PAIR = false>
 struct MmaConsumer {
   static constexpr int KS = D / 16;  // k steps of QK, d tiles of PV
   __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -256,6 +258,14 @@ struct MmaConsumer {
   // Tokens go in groups of NT (1 or 2) 16-token tiles that share one max
   // reduction and one rescale; each tile's QK runs as two independent MMA
   // chains, so the dependent-latency path per token is short.
+  // Row of KV head h's token tk in a staged tile page (one d half).
+  __device__ __forceinline__ static int tile_row(int h, int tk, const Params &p) {
+    if constexpr (PAIR)
+      return ((tk >> 3) * p.num_kv_heads + h) * 8 + (tk & 7);
+    else
+      return h * p.vbs + tk;
+  }
+
   template <int NT, bool TL>
   __device__ __forceinline__ void tiles(const unsigned char *kp, const unsigned char *vp, int m0,
                                         int ntok, const Params &p, int h, int col_bytes,
@@ -274,7 +284,7 @@ struct MmaConsumer {
     for (int u = 0; u < NT; ++u) {
       const int tk = m0 + 16 * u + (lane & 15);
       const unsigned char *kr =
-          TL ? kp + (h * p.vbs + tk) * 128 : kp + tk * p.row_pitch + col_bytes + ck;
+          TL ? kp + tile_row(h, tk, p) * 128 : kp + tk * p.row_pitch + col_bytes + ck;
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < KS; k += 2) {
@@ -349,7 +359,7 @@ struct MmaConsumer {
       }
       const int tv = base + (lane & 7) + ((mi >> 1) << 3);
       const unsigned char *vr =
-          TL ? vp + (h * p.vbs + tv) * 128 : vp + tv * p.row_pitch + col_bytes + cv;
+          TL ? vp + tile_row(h, tv, p) * 128 : vp + tv * p.row_pitch + col_bytes + cv;
 #pragma unroll
       for (int k = 0; k < KS; ++k) {
         uint32_t a[4];
@@ -1124,7 +1134,7 @@ struct PageWalker {
   // cached context lengths (nothing is prefetched without the cache).
   __device__ __forceinline__ void prefetch_next_window(const Params &p, int64_t end,
                                                        int lane) {
-    const int32_t blocks = (ctx_s + p.block_size - 1) >> (p.log2_vbs + p.log2_vpp);
+    const int32_t blocks = (ctx_s + p.block_size - 1) >> p.log2_bs;
     if (tw_lb + 32 < blocks) {
       tn_seq = s;
       tn_lb = tw_lb + 32;
@@ -1155,6 +1165,27 @@ struct PageWalker {
       tn_seq = -1;
       prefetch_next_window(p, end, lane);
     }
+    return __shfl_sync(0xffffffffu, tw_val, lb - tw_lb);
+  }
+  // Two-block pages: the physical blocks of the current 16-token page
+  // (entries 2 vlb and 2 vlb + 1; windows start at even entries, so both sit
+  // in one window).
+  __device__ __forceinline__ int32_t block_pair(const Params &p, int64_t end, int lane,
+                                                int32_t &pb2) {
+    const int32_t lb = vlb << 1;
+    if (s != tw_seq || lb >= tw_lb + 32) {
+      if (s == tn_seq && lb >= tn_lb && lb < tn_lb + 32) {
+        tw_val = tn_val;  // prefetched
+        tw_lb = tn_lb;
+      } else {
+        tw_lb = lb;
+        tw_val = load_table(p, s, lb, lane);
+      }
+      tw_seq = s;
+      tn_seq = -1;
+      prefetch_next_window(p, end, lane);
+    }
+    pb2 = __shfl_sync(0xffffffffu, tw_val, lb + 1 - tw_lb);
     return __shfl_sync(0xffffffffu, tw_val, lb - tw_lb);
   }
   __device__ __forceinline__ int32_t ntok(const Params &p) const {
@@ -1258,7 +1289,7 @@ __device__ __forceinline__ void write_new_rows_fp8(const Params &p, int32_t s, i
 // heads per warp) and G = 0 the token-row one (up to 8 heads per warp);
 // NCW = consumer warps.
 // ===========================================================================
-template <typename T, int D, int G, int NCW>
+template <typename T, int D, int G, int NCW, bool PAIR = false>
 __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     decode_stream_kernel(const __grid_constant__ Params p) {
   // T: __nv_bfloat16, float, or Fp8E4M3 (FP8 pages; q and out bf16)
@@ -1273,7 +1304,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   static_assert(sizeof(Shared) % 16 == 0 && sizeof(PageDesc) % 16 == 0,
                 "descriptors and score buffers need 16-byte alignment");
   using MmaCons =
-      typename std::conditional<G == 16, HeadRowConsumer<D>, MmaConsumer<D, kFp8>>::type;
+      typename std::conditional<G == 16, HeadRowConsumer<D>, MmaConsumer<D, kFp8, PAIR>>::type;
   using Cons = typename std::conditional<kMma, MmaCons, FmaConsumer<TA, D, kFmaG>>::type;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Shared &sh = *reinterpret_cast<Shared *>(smem_raw);
@@ -1470,13 +1501,16 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         uint32_t bytes = 0;
         bool wrote = false;
         for (int k = 0; k < npg; ++k) {
-          const int32_t pb = wk.block(p, end, lane);
+          int32_t pb2 = -1;  // two-block pages: the second block, if the page reaches it
+          const int32_t pb = PAIR ? wk.block_pair(p, end, lane, pb2) : wk.block(p, end, lane);
           const int32_t ntok = wk.ntok(p);
+          if (PAIR && ntok <= 8) pb2 = -1;
           const bool first = (wk.vlb == 0) || (wk.cursor == start);
           const bool seq_last = wk.vlb == wk.pages_s - 1;
           // split-K: a partition ends every pp pages (ranges end on unit ends)
           const bool last = seq_last || (wk.cursor == end - 1) || u_left == 1;
-          const bool bad_block = pb < 0 || pb >= p.num_blocks;
+          const bool bad_block =
+              pb < 0 || pb >= p.num_blocks || (PAIR && ntok > 8 && (pb2 < 0 || pb2 >= p.num_blocks));
           bool bad = bad_block;
           if (bad_block && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
           if (p.slot_mapping != nullptr && seq_last && wk.slot_s >= 0) {
@@ -1484,7 +1518,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             // this page; its slot must be the one the table gives it, else
             // nothing is stored and the sequence's output is zeroed.
             const int32_t pos = wk.ctx_s - 1;
-            const int64_t want = (int64_t)pb * p.block_size + (pos & (p.block_size - 1));
+            const int32_t pbw = (PAIR && (pos & 8)) ? pb2 : pb;  // the block holding pos
+            const int64_t want = (int64_t)pbw * p.block_size + (pos & (p.block_size - 1));
             if (!bad_block && wk.slot_s == want) {
               if constexpr (kFp8)
                 write_new_rows_fp8(p, wk.s, want, lane);
@@ -1502,8 +1537,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             d.ntok = ntok;
             d.unit = u_cur;
             d.pb = pb;
-            d.toff = (wk.vlb & ((1 << p.log2_vpp) - 1)) * p.vbs;
-            d.pad0 = d.pad1 = 0;
+            d.toff = PAIR ? 0 : (wk.vlb & ((1 << p.log2_vpp) - 1)) * p.vbs;
+            d.pad0 = pb2;
+            d.pad1 = 0;
             int32_t flags = (first ? kFirst : 0) | (last ? kLast : 0) | (bad ? kBad : 0);
             if (last && pp == 0) {
               // is the sequence cut between CTAs (it began before this CTA's
@@ -1525,8 +1561,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             descs[slot * kMaxPPS + k] = d;
           }
           if (!bad)
-            bytes += p.tile ? 2u * (uint32_t)nbox * (uint32_t)p.box_bytes
-                            : 2u * (uint32_t)ntok * (uint32_t)p.row_bytes;
+            bytes += PAIR     ? (pb2 >= 0 ? 2u : 1u) * (uint32_t)nbox * (uint32_t)p.box_bytes
+                     : p.tile ? 2u * (uint32_t)nbox * (uint32_t)p.box_bytes
+                              : 2u * (uint32_t)ntok * (uint32_t)p.row_bytes;
           if (first) bytes += (uint32_t)p.q_bytes;
           const int32_t s_before = wk.s;
           wk.advance(p, end, lane);
@@ -1551,7 +1588,25 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         unsigned char *qst = st + (size_t)2 * p.pps * p.vpage_stride;
         for (int k = 0; k < npg; ++k) {
           const PageDesc d = descs[slot * kMaxPPS + k];
-          if (!(d.flags & kBad) && p.tile) {
+          if constexpr (PAIR) {
+            if (!(d.flags & kBad)) {
+              // one box of the block's 8 token rows of every KV head per
+              // (block, tensor, d half); the second block's box lands after
+              // the first's
+              constexpr int kHalves = D / 64;
+              const int nblk = d.pad0 >= 0 ? 2 : 1;
+              if (lane < nblk * 2 * kHalves) {
+                const int dh = lane % kHalves;
+                const bool isv = (lane / kHalves) & 1;
+                const int blk = lane / (2 * kHalves);
+                tma_load_3d_hint((isv ? vst : kst) + (size_t)k * p.vpage_stride +
+                                     (size_t)dh * p.box_bytes + (size_t)blk * (p.box_bytes / 2),
+                                 isv ? &p.tmap_v : &p.tmap_k, dh * 64,
+                                 (blk ? d.pad0 : d.pb) * p.block_size, 0, &sh.full[slot],
+                                 kv_policy);
+              }
+            }
+          } else if (!(d.flags & kBad) && p.tile) {
             // one box per (tensor, 64-wide d half), one lane each
             if (lane < 2 * nbox) {
               const int dh = lane % nbox;
@@ -1730,9 +1785,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 // Host side: launch one instantiation.  Explicitly instantiated per dtype in
 // its own translation unit.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int G, int NCW>
+template <typename T, int D, int G, int NCW, bool PAIR = false>
 cudaError_t launch_one(const Params &p, size_t smem, cudaStream_t stream) {
-  auto kern = decode_stream_kernel<T, D, G, NCW>;
+  auto kern = decode_stream_kernel<T, D, G, NCW, PAIR>;
   static size_t configured[64] = {};  // per device: largest dynamic smem already allowed
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

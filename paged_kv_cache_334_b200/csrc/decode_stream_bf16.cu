@@ -22,6 +22,16 @@ cudaError_t launch_bf16(const Params &p, int head_dim, int group, int hkv, size_
   (void)group;
   const int ncw = hkv * p.warps_per_kv;
   const bool rows = p.heads_per_warp == 16;
+  if (p.pair) {
+    // 8-token blocks, two per page: head_dim 128, one warp per KV head, 4
+    // or 8 KV heads
+    if (head_dim != 128 || rows || p.warps_per_kv != 1) return cudaErrorInvalidValue;
+    switch (ncw) {
+      case 4: return launch_one<__nv_bfloat16, 128, 0, 4, true>(p, smem, stream);
+      case 8: return launch_one<__nv_bfloat16, 128, 0, 8, true>(p, smem, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   if (head_dim == 64)
     return rows ? launch_ncw<64, 16>(p, ncw, smem, stream) : launch_ncw<64, 0>(p, ncw, smem, stream);
   if (head_dim == 128)

@@ -79,6 +79,10 @@ struct Params {
   int32_t tok_offset, table_stride;
   int32_t num_blocks, block_size, num_kv_heads, num_q_heads, max_blocks, batch;
   int32_t vbs, log2_vbs, log2_vpp;  // virtual page tokens; log2 of pages per block
+  int32_t log2_bs;                  // log2 of block_size
+  // 8-token blocks on the tile path: a virtual page of 16 tokens is two
+  // blocks, copied as one box per (block, tensor, 64-wide d half)
+  int32_t pair;
   int32_t row_bytes;                // one token row, all KV heads (global layout)
   int32_t row_pitch;                // bytes between token rows in a shared-memory stage
   int32_t vpage_stride;             // vbs * row_pitch
