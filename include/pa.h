@@ -382,11 +382,13 @@ pa_status pa_decode_noalloc(const pa_cache_desc *cache, void *out,
  * partition_tokens must be a positive multiple of block_size;
  * max_partitions must be >= ceil(max_blocks_per_seq * block_size /
  * partition_tokens).  No workspace: on the shapes of pa_decode's persistent
- * page-stream kernel the partitions of all sequences form one stream cut
- * into one range per SM at partition boundaries, so each partition is
- * computed whole by one CTA and written once; other shapes run one CTA per
- * (partition, KV head, head tile) and allow at most 1024 blocks per
- * partition.
+ * page-stream kernel, when partition_tokens is a multiple of its page (16
+ * tokens for bf16 caches of 8-token blocks, 32 for FP8 caches, else at most
+ * block_size), the partitions of all sequences form one stream cut into one
+ * range per SM at partition boundaries, so each partition is computed whole
+ * by one CTA and written once; other shapes and partition sizes run one CTA
+ * per (partition, KV head, head tile) and allow at most 1024 blocks per
+ * partition; FP8 caches need the page stream (PA_ERR_UNSUPPORTED otherwise).
  */
 pa_status pa_decode_splitk(const pa_cache_desc *cache, const void *q,
                            const void *key_cache, const void *value_cache,

@@ -161,11 +161,11 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
   if (s.row_bytes + 16 > st::kVPageBytes) return s;
   int32_t rows = st::kVPageBytes / s.row_bytes;  // power of two
   if (fp8) {
-    // 16-token virtual pages (one MMA tile), one warp per KV head
+    // 32-token virtual pages (two MMA tiles), one warp per KV head
     if (c->block_size < 16 || (hkv != 4 && hkv != 8) || s.warps_per_kv != 1 ||
         s.heads_per_warp > 8)
       return s;
-    rows = 16;
+    rows = 32;
   }
   s.vbs = c->block_size < rows ? c->block_size : rows;
   // 8-token blocks of bf16, head_dim 128, one warp per KV head: pages of two
@@ -175,6 +175,11 @@ StreamPlan plan_stream(const pa_cache_desc *c, int32_t num_q_heads, bool allow_t
            c->head_dim == 128 && s.warps_per_kv == 1 && s.heads_per_warp <= 8 &&
            (hkv == 4 || hkv == 8);
   if (s.pair) s.vbs = 16;
+  // FP8 pages of 16-token blocks: two blocks per 32-token page
+  if (allow_tile && fp8 && c->block_size == 16) {
+    s.pair = true;
+    s.vbs = 32;
+  }
   s.log2_vbs = ilog2(s.vbs);
   s.log2_vpp = s.pair ? 0 : ilog2(c->block_size / s.vbs);
   s.tile = allow_tile && bf16 && s.vbs >= 16 && hkv <= 256;

@@ -394,38 +394,67 @@ struct MmaConsumer {
       page_t<false>(kp, vp, ntok, p, h, col_bytes, lane);
   }
 
-  // FP8 pages (F16, head_dim 128): one 16-token page of E4M3 codes, K and V
-  // each one box of [KV head][16 tokens][128 codes] with the 128-byte swizzle
-  // (16-byte chunk c of row r at chunk c ^ (r % 8)).  The fragments come
-  // straight from the codes: for S a lane reads d chunks 2t, 2t + 1 of tokens
-  // g and g + 8; for O^T d chunk g of tokens 2t, 2t + 1, 2t + 8, 2t + 9,
-  // pairing the two tokens of each fragment register with a byte permute.
+  // FP8 pages (F16, head_dim 128): a page of up to 32 tokens of E4M3 codes,
+  // in 16-token tiles; tile u of KV head h starts at row code_row(h, u) of
+  // its tensor's staged rows (128 codes each, 16-byte chunk c of row r at
+  // chunk c ^ (r % 8)): one box of [KV head][32 tokens], or (PAIR: two
+  // 16-token blocks per page) one box of [KV head][16 tokens] per block.
+  // The fragments come straight from the codes: for S a lane reads d chunks
+  // 2t, 2t + 1 of tokens g and g + 8; for O^T d chunk g of tokens 2t, 2t + 1,
+  // 2t + 8, 2t + 9, pairing the two tokens of each fragment register with a
+  // byte permute.  The tiles of a page share one max and one rescale.
+  __device__ __forceinline__ static int code_row(int h, int u, const Params &p) {
+    if constexpr (PAIR)
+      return (u * p.num_kv_heads + h) * 16;
+    else
+      return h * 32 + 16 * u;
+  }
+
   __device__ __forceinline__ void page_codes(const unsigned char *kp, const unsigned char *vp,
-                                             int ntok, int h, int lane) {
+                                             int ntok, const Params &p, int h, int lane) {
+    if (ntok > 16)
+      page_codes_t<2>(kp, vp, ntok, p, h, lane);
+    else
+      page_codes_t<1>(kp, vp, ntok, p, h, lane);
+  }
+
+  template <int NT>
+  __device__ __forceinline__ void page_codes_t(const unsigned char *kp, const unsigned char *vp,
+                                               int ntok, const Params &p, int h, int lane) {
     static_assert(D == 128, "FP8 pages: head_dim 128");
     const int g = lane >> 2, t = lane & 3;
-    const unsigned char *kr = kp + (h * 16 + g) * 128;  // token g; token g + 8 is 1 KB on
     const int c0 = ((2 * t) ^ g) << 4, c1 = ((2 * t + 1) ^ g) << 4;
-    const uint4 ka0 = *reinterpret_cast<const uint4 *>(kr + c0);
-    const uint4 ka1 = *reinterpret_cast<const uint4 *>(kr + c1);
-    const uint4 kb0 = *reinterpret_cast<const uint4 *>(kr + 1024 + c0);
-    const uint4 kb1 = *reinterpret_cast<const uint4 *>(kr + 1024 + c1);
-    const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
-    const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    float s[NT][4];
 #pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      uint32_t a[4];
-      e4m3x4_to_f16x4(wa[k], a[0], a[2]);
-      e4m3x4_to_f16x4(wb[k], a[1], a[3]);
-      mma((k & 1) ? sb : sa, a, qb[k][0], qb[k][1]);
+    for (int u = 0; u < NT; ++u) {
+      const unsigned char *kr = kp + (code_row(h, u, p) + g) * 128;  // token g; g + 8 is 1 KB on
+      const uint4 ka0 = *reinterpret_cast<const uint4 *>(kr + c0);
+      const uint4 ka1 = *reinterpret_cast<const uint4 *>(kr + c1);
+      const uint4 kb0 = *reinterpret_cast<const uint4 *>(kr + 1024 + c0);
+      const uint4 kb1 = *reinterpret_cast<const uint4 *>(kr + 1024 + c1);
+      const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
+      const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        uint32_t a[4];
+        e4m3x4_to_f16x4(wa[k], a[0], a[2]);
+        e4m3x4_to_f16x4(wb[k], a[1], a[3]);
+        mma((k & 1) ? sb : sa, a, qb[k][0], qb[k][1]);
+      }
+      const int r0 = 16 * u + g;
+      const bool v0 = r0 < ntok, v1 = r0 + 8 < ntok;
+      s[u][0] = v0 ? (sa[0] + sb[0]) * scale_log2_ : -INFINITY;
+      s[u][1] = v0 ? (sa[1] + sb[1]) * scale_log2_ : -INFINITY;
+      s[u][2] = v1 ? (sa[2] + sb[2]) * scale_log2_ : -INFINITY;
+      s[u][3] = v1 ? (sa[3] + sb[3]) * scale_log2_ : -INFINITY;
     }
-    const bool v0 = g < ntok, v1 = g + 8 < ntok;
-    const float s0 = v0 ? (sa[0] + sb[0]) * scale_log2_ : -INFINITY;
-    const float s1 = v0 ? (sa[1] + sb[1]) * scale_log2_ : -INFINITY;
-    const float s2 = v1 ? (sa[2] + sb[2]) * scale_log2_ : -INFINITY;
-    const float s3 = v1 ? (sa[3] + sb[3]) * scale_log2_ : -INFINITY;
-    float x0 = fmaxf(s0, s2), x1 = fmaxf(s1, s3);
+    float x0 = -INFINITY, x1 = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      x0 = fmaxf(x0, fmaxf(s[u][0], s[u][2]));
+      x1 = fmaxf(x1, fmaxf(s[u][1], s[u][3]));
+    }
 #pragma unroll
     for (int mask = 4; mask < 32; mask <<= 1) {
       x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, mask));
@@ -435,13 +464,20 @@ struct MmaConsumer {
     const float a0 = ex2(m0_ - n0), a1 = ex2(m1_ - n1);
     m0_ = n0;
     m1_ = n1;
-    const float p0 = ex2(s0 - n0), p1 = ex2(s1 - n1);
-    const float p2 = ex2(s2 - n0), p3 = ex2(s3 - n1);
-    l0 = l0 * a0 + (p0 + p2);
-    l1 = l1 * a1 + (p1 + p3);
-    // P^T (16 tokens x 8 heads) as the B operand
-    const uint32_t pb0 = movmatrix_trans(pack(p0, p1));
-    const uint32_t pb1 = movmatrix_trans(pack(p2, p3));
+    uint32_t pb[NT][2];
+    float add0 = 0.f, add1 = 0.f;
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      const float p0 = ex2(s[u][0] - n0), p1 = ex2(s[u][1] - n1);
+      const float p2 = ex2(s[u][2] - n0), p3 = ex2(s[u][3] - n1);
+      add0 += p0 + p2;
+      add1 += p1 + p3;
+      // P^T (16 tokens x 8 heads) as the B operand
+      pb[u][0] = movmatrix_trans(pack(p0, p1));
+      pb[u][1] = movmatrix_trans(pack(p2, p3));
+    }
+    l0 = l0 * a0 + add0;
+    l1 = l1 * a1 + add1;
     if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
 #pragma unroll
       for (int k = 0; k < KS; ++k) {
@@ -451,32 +487,38 @@ struct MmaConsumer {
         o[k][3] *= a1;
       }
     }
-    // tokens past ntok may hold anything: their V codes are zeroed (P is 0)
-    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-    if (ntok < 16) {
-      mlo = (2 * t < ntok ? 0x0000ffffu : 0u) | (2 * t + 1 < ntok ? 0xffff0000u : 0u);
-      mhi = (2 * t + 8 < ntok ? 0x0000ffffu : 0u) | (2 * t + 9 < ntok ? 0xffff0000u : 0u);
-    }
-    const unsigned char *vr = vp + (h * 16 + 2 * t) * 128;
-    const int e0 = (g ^ (2 * t)) << 4, e1 = (g ^ (2 * t + 1)) << 4;
-    const uint4 vx = *reinterpret_cast<const uint4 *>(vr + e0);          // token 2t
-    const uint4 vy = *reinterpret_cast<const uint4 *>(vr + 128 + e1);    // 2t + 1
-    const uint4 vz = *reinterpret_cast<const uint4 *>(vr + 1024 + e0);   // 2t + 8
-    const uint4 vw = *reinterpret_cast<const uint4 *>(vr + 1152 + e1);   // 2t + 9
-    const uint32_t xs[4] = {vx.x, vx.y, vx.z, vx.w}, ys[4] = {vy.x, vy.y, vy.z, vy.w};
-    const uint32_t zs[4] = {vz.x, vz.y, vz.z, vz.w}, ws[4] = {vw.x, vw.y, vw.z, vw.w};
 #pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      // codes 2k, 2k + 1 of the chunk (d = 16g + 2k, + 1) of two tokens
-      const uint32_t sel = (k & 1) ? 0x7362u : 0x5140u;
-      uint32_t a[4];
-      e4m3x4_to_f16x4(__byte_perm(xs[k >> 1], ys[k >> 1], sel), a[0], a[1]);
-      e4m3x4_to_f16x4(__byte_perm(zs[k >> 1], ws[k >> 1], sel), a[2], a[3]);
-      a[0] &= mlo;
-      a[1] &= mlo;
-      a[2] &= mhi;
-      a[3] &= mhi;
-      mma(o[k], a, pb0, pb1);
+    for (int u = 0; u < NT; ++u) {
+      // tokens past ntok may hold anything: their V codes are zeroed (P is 0)
+      const int base = 16 * u;
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (base + 16 > ntok) {
+        mlo = (base + 2 * t < ntok ? 0x0000ffffu : 0u) |
+              (base + 2 * t + 1 < ntok ? 0xffff0000u : 0u);
+        mhi = (base + 2 * t + 8 < ntok ? 0x0000ffffu : 0u) |
+              (base + 2 * t + 9 < ntok ? 0xffff0000u : 0u);
+      }
+      const unsigned char *vr = vp + (code_row(h, u, p) + 2 * t) * 128;
+      const int e0 = (g ^ (2 * t)) << 4, e1 = (g ^ (2 * t + 1)) << 4;
+      const uint4 vx = *reinterpret_cast<const uint4 *>(vr + e0);         // token 2t
+      const uint4 vy = *reinterpret_cast<const uint4 *>(vr + 128 + e1);   // 2t + 1
+      const uint4 vz = *reinterpret_cast<const uint4 *>(vr + 1024 + e0);  // 2t + 8
+      const uint4 vw = *reinterpret_cast<const uint4 *>(vr + 1152 + e1);  // 2t + 9
+      const uint32_t xs[4] = {vx.x, vx.y, vx.z, vx.w}, ys[4] = {vy.x, vy.y, vy.z, vy.w};
+      const uint32_t zs[4] = {vz.x, vz.y, vz.z, vz.w}, ws[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        // codes 2k, 2k + 1 of the chunk (d = 16g + 2k, + 1) of two tokens
+        const uint32_t sel = (k & 1) ? 0x7362u : 0x5140u;
+        uint32_t a[4];
+        e4m3x4_to_f16x4(__byte_perm(xs[k >> 1], ys[k >> 1], sel), a[0], a[1]);
+        e4m3x4_to_f16x4(__byte_perm(zs[k >> 1], ws[k >> 1], sel), a[2], a[3]);
+        a[0] &= mlo;
+        a[1] &= mlo;
+        a[2] &= mhi;
+        a[3] &= mhi;
+        mma(o[k], a, pb[u][0], pb[u][1]);
+      }
     }
   }
 
@@ -1504,13 +1546,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           int32_t pb2 = -1;  // two-block pages: the second block, if the page reaches it
           const int32_t pb = PAIR ? wk.block_pair(p, end, lane, pb2) : wk.block(p, end, lane);
           const int32_t ntok = wk.ntok(p);
-          if (PAIR && ntok <= 8) pb2 = -1;
+          if (PAIR && ntok <= p.block_size) pb2 = -1;
           const bool first = (wk.vlb == 0) || (wk.cursor == start);
           const bool seq_last = wk.vlb == wk.pages_s - 1;
           // split-K: a partition ends every pp pages (ranges end on unit ends)
           const bool last = seq_last || (wk.cursor == end - 1) || u_left == 1;
           const bool bad_block =
-              pb < 0 || pb >= p.num_blocks || (PAIR && ntok > 8 && (pb2 < 0 || pb2 >= p.num_blocks));
+              pb < 0 || pb >= p.num_blocks ||
+              (PAIR && ntok > p.block_size && (pb2 < 0 || pb2 >= p.num_blocks));
           bool bad = bad_block;
           if (bad_block && lane == 0) set_error(p.err_word, PA_DEVERR_BLOCK_ID);
           if (p.slot_mapping != nullptr && seq_last && wk.slot_s >= 0) {
@@ -1518,7 +1561,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             // this page; its slot must be the one the table gives it, else
             // nothing is stored and the sequence's output is zeroed.
             const int32_t pos = wk.ctx_s - 1;
-            const int32_t pbw = (PAIR && (pos & 8)) ? pb2 : pb;  // the block holding pos
+            // the block holding pos
+            const int32_t pbw = (PAIR && ((pos >> p.log2_bs) & 1)) ? pb2 : pb;
             const int64_t want = (int64_t)pbw * p.block_size + (pos & (p.block_size - 1));
             if (!bad_block && wk.slot_s == want) {
               if constexpr (kFp8)
@@ -1590,10 +1634,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
           const PageDesc d = descs[slot * kMaxPPS + k];
           if constexpr (PAIR) {
             if (!(d.flags & kBad)) {
-              // one box of the block's 8 token rows of every KV head per
-              // (block, tensor, d half); the second block's box lands after
-              // the first's
-              constexpr int kHalves = D / 64;
+              // one box of the block's token rows of every KV head per
+              // (block, tensor, box of the row); the second block's box lands
+              // after the first's
+              constexpr int kHalves = kFp8 ? 1 : D / 64;
               const int nblk = d.pad0 >= 0 ? 2 : 1;
               if (lane < nblk * 2 * kHalves) {
                 const int dh = lane % kHalves;
@@ -1701,7 +1745,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             const unsigned char *kp = kst + (size_t)k * p.vpage_stride;
             const unsigned char *vp = vst + (size_t)k * p.vpage_stride;
             if constexpr (kFp8) {
-              cs.page_codes(kp, vp, d.ntok, h, lane);
+              cs.page_codes(kp, vp, d.ntok, p, h, lane);
             } else if constexpr (kMma) {
               cs.page(kp, vp, d.ntok, p, h, col_bytes, lane);
             } else {

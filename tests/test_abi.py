@@ -193,6 +193,9 @@ def test_fp8_argument_checks_need_no_device(lib):
     assert lib.pa_decode_splitk(ctypes.byref(_fp8(hkv=2)), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 4,
                                 0.1, 16, P, FAKE, FAKE, FAKE, None, None) == pa.PA_ERR_UNSUPPORTED
     assert b"FP8" in lib.pa_last_error_message()
+    # FP8 pages stream 32 tokens at a time: partitions must hold whole pages
+    assert lib.pa_decode_splitk(ctypes.byref(_fp8()), FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 4,
+                                0.1, 16, P, FAKE, FAKE, FAKE, None, None) == pa.PA_ERR_UNSUPPORTED
     assert lib.pa_decode_shared_prefix(ctypes.byref(_fp8()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                                        2, 32, 4, 1, 0.1, FAKE, 1 << 30, None,
                                        None) == pa.PA_ERR_UNSUPPORTED

@@ -122,7 +122,9 @@ FP8_SHAPES = [
 
 @pytest.mark.parametrize("Hq,Hkv,bs", FP8_SHAPES)
 def test_fp8_shapes(Hq, Hkv, bs):
-    lens = [1, 15, 16, 17, 300, 1000, 2049]
+    # around the 16-token tiles and the 32-token pages (the new token in
+    # either block of a two-block page)
+    lens = [1, 15, 16, 17, 31, 32, 33, 48, 49, 300, 1000, 2049]
     w = wl.custom_workload(dtype=wl.DTYPE_FP8, batch=len(lens), num_q_heads=Hq,
                            num_kv_heads=Hkv, head_dim=128, block_size=bs, context_lens=lens,
                            seed=Hq + Hkv + bs, new_tokens=True, k_scale=0.125, v_scale=0.75)
@@ -160,6 +162,34 @@ def test_fp8_forward_bad_slot_is_flagged_and_zeroed():
     got = to_f64(out)
     assert not got[1].any()
     assert_close(got[[0, 2]], ref[[0, 2]], wl.DTYPE_BF16, "unaffected sequences")
+
+
+def test_fp8_bad_ids_in_either_block_of_a_page():
+    """16-token blocks go two to a 32-token page: a bad id in the first or
+    the second block of a visible page zeroes the sequence and sets the flag;
+    the second entry of a page that ends in its first block is never read."""
+    lens = [40, 40, 16, 300]
+    w = wl.custom_workload(dtype=wl.DTYPE_FP8, batch=4, num_q_heads=32, num_kv_heads=8,
+                           head_dim=128, block_size=16, context_lens=lens, seed=41,
+                           max_blocks=24)
+    bt = w.block_tables.copy()
+    bt[0, 1] = w.num_blocks + 2   # second block of page 0 (tokens 16..31)
+    bt[1, 2] = -5                 # first block of page 1 (tokens 32..47)
+    bt[2, 1] = 123456789          # past the 16 visible tokens: never read
+    d = dict(q=up(w.q), kc=up(w.key_cache), vc=up(w.value_cache),
+             bt=torch.from_numpy(bt).cuda(), cl=torch.from_numpy(w.context_lens).cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(d["q"])
+    pa.pa_decode(out, d["q"], d["kc"], d["vc"], d["bt"], d["cl"], err_word=err,
+                 k_scale=w.k_scale, v_scale=w.v_scale)
+    torch.cuda.synchronize()
+    assert int(err.item()) == pa.PA_DEVERR_BLOCK_ID
+    ref, flags = oracle.decode_fp8(w.q, w.key_cache, w.value_cache, w.k_scale, w.v_scale, bt,
+                                   w.context_lens, 1.0 / math.sqrt(w.head_dim))
+    assert list(flags) == [oracle.FLAG_BLOCK_ID, oracle.FLAG_BLOCK_ID, 0, 0]
+    got = to_f64(out)
+    assert not got[0].any() and not got[1].any()
+    assert_close(got, ref, wl.DTYPE_BF16, "fp8 bad ids")
 
 
 def test_fp8_unsupported_shapes_are_refused():
