@@ -10,7 +10,9 @@
 // * Work: the visible pages of all sequences form one stream (sequence 0's
 //   pages, then sequence 1's, ...).  Pages are cut into "virtual pages" of at
 //   most 32 KB (a run of whole token rows of one physical page, all KV heads --
-//   contiguous in the [num_blocks, block_size, Hkv, D] layout).  The grid is one
+//   contiguous in the [num_blocks, block_size, Hkv, D] layout); blocks below
+//   one page's worth (8-token bf16 blocks, 16-token FP8 blocks) are joined two
+//   to a virtual page (two table entries per page).  The grid is one
 //   CTA per SM; CTA c takes the contiguous range [c*T/G, (c+1)*T/G) of the T
 //   virtual pages, so every CTA moves the same number of bytes (+-1 page)
 //   whatever the mix of context lengths.
@@ -22,7 +24,9 @@
 //       (cp.async.bulk.tensor.3d) of boxes [64 d][vbs tokens][Hkv heads] of
 //       K and V with the 128-byte swizzle, one box per 64-wide half of D, so
 //       a whole virtual page takes 2 * D/64 copies and ldmatrix reads it
-//       without bank conflicts;
+//       without bank conflicts (two-block pages: one box per block, the
+//       second after the first); FP8 pages one box of 128 codes per row;
+//       the copies carry an evict-first L2 policy (pages are read once);
 //     - otherwise: 1-D bulk copies (cp.async.bulk) of the valid token rows,
 //       landing at a pitch of row_bytes + 16 for the tensor-core consumers
 //       (eight consecutive tokens in eight different bank groups);
@@ -37,6 +41,9 @@
 //       N = 8 side, tokens are M): S^T = K Q^T and O^T += V^T P^T run on the
 //       tensor cores (mma.sync m16n8k16, fp32 accumulation), P is rounded to
 //       bf16 and turned into the B operand with movmatrix.
+//     - FP8: the same tiles in fp16, the fragments built in registers from
+//       the staged codes (exact conversion), two 16-token tiles of a 32-token
+//       page per pass.
 //     - fp32: CUDA-core FMAs, per-(token, head) dot products reduced with a
 //       transposed butterfly (the 1e-5 tolerance rules out bf16/tf32 MMA).
 // * A sequence split across CTAs leaves one partial per CTA in the workspace,
