@@ -1085,9 +1085,10 @@ pa_status pa_reduce(void *out, const float *part_max, const float *part_sum,
     return fail(PA_ERR_UNSUPPORTED, "batch * num_q_heads too large%s");
   if (head_dim % 4 != 0) return fail(PA_ERR_INVALID_ARG, "head_dim must be a multiple of 4%s");
   // the kernel keeps one weight per partition and head_dim-wide group sums
-  // of 256 threads in shared memory
+  // of its threads in shared memory
   if (head_dim > 1024 ||
-      (size_t)((max_partitions + 3) & ~3) * 4 + (size_t)(256 / (head_dim / 4)) * head_dim * 4 >
+      (size_t)((max_partitions + 3) & ~3) * 4 +
+              (size_t)(pa::kReduceThreads / (head_dim / 4)) * head_dim * 4 >
           (size_t)227 * 1024)
     return fail(PA_ERR_UNSUPPORTED,
                 "head_dim above 1024 or more than about 56000 partitions%s");

@@ -218,6 +218,8 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 // Set the text pa_last_error_message() returns on the calling host thread.
 void set_last_error_message(const char *msg);
 
+// Threads of one pa_reduce CTA (one CTA per sequence and query head).
+constexpr int kReduceThreads = 512;
 cudaError_t launch_reduce(void *out, const float *part_max,
                           const float *part_sum, const float *part_out,
                           const int32_t *context_lens, int32_t batch,

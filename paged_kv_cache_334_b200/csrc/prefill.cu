@@ -165,6 +165,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     sh.abort_flag = 0;
     sh.bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!len_bad) {
+      // the Q tile does not depend on the table: its copy overlaps the
+      // table check below
+      mbar_arrive_expect_tx(&sh.qfull, (uint32_t)(NH * kBox));
+      for (int dh = 0; dh < NH; ++dh)
+        tma_load_3d(qt + dh * kBox, &p.tmap_q, dh * 64, h * p.group, q0 + j0, &sh.qfull);
+    }
+  }
+  // tensor memory is allocated while the table is read
+  if (warp == 1 && !len_bad) {
+    tc_alloc(&sh.tmem_base, kTmemCols);
+    tc_relinquish();
   }
   __syncthreads();
   if (len_bad) {
@@ -183,8 +195,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       sh.ids[i] = pb;
     }
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
   if (sh.bad) {
+    if (!len_bad) {
+      // the Q copy lands before the CTA's shared memory is released, and
+      // the tensor memory goes back
+      if (tid == 0) {
+        volatile int32_t never = 0;
+        if (!mbar_wait(&sh.qfull, 0, &never)) set_error(p.err_word, PA_DEVERR_TIMEOUT);
+      }
+      if (warp == 1) tc_dealloc(sh.tmem_base, kTmemCols);
+    }
     // zero the tile's rows: tokens [j0, j_end) x the group's heads
     const int64_t row_elems = (int64_t)p.group * D;  // one token's heads of this KV head
     const int64_t per_tok = (int64_t)p.num_q_heads * D;
@@ -198,13 +221,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  if (warp == 1) {
-    tc_alloc(&sh.tmem_base, kTmemCols);
-    tc_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
   const uint32_t tm = sh.tmem_base;
 
   const int ppt = kTok / p.block_size;        // pages per K/V tile
@@ -214,12 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tile_tokens = [&](int t) { return min(kTok, pos_max + 1 - t * kTok); };
 
   if (warp == 0) {
-    // ===================== tiled copies =====================
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&sh.qfull, (uint32_t)(NH * kBox));
-      for (int dh = 0; dh < NH; ++dh)
-        tma_load_3d(qt + dh * kBox, &p.tmap_q, dh * 64, h * p.group, q0 + j0, &sh.qfull);
-    }
+    // ===================== tiled copies (Q was issued above) =====================
     const uint32_t page_bytes = (uint32_t)p.block_size * 128u;
     // one K or V tile: its pages' boxes back to back per d half
     auto load = [&](const CUtensorMap *map, unsigned char *dst, uint64_t *bar, int t) {

@@ -23,8 +23,6 @@
 namespace pa {
 namespace {
 
-constexpr int kReduceThreads = 256;
-
 template <typename TO>
 __global__ void __launch_bounds__(kReduceThreads)
 reduce_kernel(void *__restrict__ out, const float *__restrict__ part_max,

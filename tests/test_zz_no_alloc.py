@@ -97,6 +97,24 @@ def test_noalloc_group_of_64_heads_on_the_page_stream():
     assert int(err.item()) == 0
 
 
+def test_noalloc_eight_token_blocks():
+    """8-token blocks, two to a page on the page stream: pa_decode_noalloc
+    against pa_decode and the oracle, two calls in a row."""
+    w = wl.custom_workload(dtype=wl.DTYPE_BF16, batch=7, num_q_heads=32, num_kv_heads=8,
+                           head_dim=128, block_size=8, context_lens=[1, 8, 9, 16, 17, 300, 1025],
+                           seed=13, new_tokens=True)
+    d, ref = _prepare(w)
+    oref, flags, _, _ = oracle_after_write(w)
+    assert not flags.any()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for call in range(2):
+        out = _noalloc(d, err)
+        torch.cuda.synchronize()
+        assert_close(to_f64(out), to_f64(ref), w.dtype, f"bs8 noalloc call {call}")
+        assert_close(to_f64(out), oref, w.dtype, f"bs8 noalloc call {call} vs oracle")
+    assert int(err.item()) == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     # a table long enough for 65536 tokens per sequence: the workspace would
     # exceed the fixed scratch even though the actual contexts are short
