@@ -113,7 +113,9 @@ FP8_SHAPES = [
     # Hq, Hkv, bs
     (32, 8, 16),   # 4 query heads per KV head
     (8, 8, 16),    # 1
-    (16, 8, 256),  # 256-token pages in 16-token virtual pages
+    (16, 4, 16),   # 16-token blocks two to a page at 4 KV heads
+    (32, 4, 16),   # 8
+    (16, 8, 256),  # 256-token pages in 32-token virtual pages
     (16, 4, 32),
     (8, 4, 64),    # 2
     (32, 4, 128),  # 8

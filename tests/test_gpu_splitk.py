@@ -175,6 +175,42 @@ def test_splitk_fp8_pages():
     assert_close(to_f64(out), ref, wl.DTYPE_BF16, "gqa_fp8 split-K reduced")
 
 
+def test_splitk_fp8_two_block_pages_at_four_kv_heads():
+    """FP8 pages of 16-token blocks (two to a 32-token page) at 4 KV heads
+    and 64-token partitions: partials and the reduced output against the
+    oracle on the code values."""
+    ctx = [1, 31, 33, 64, 65, 500, 1000]
+    w = wl.custom_workload(dtype=wl.DTYPE_FP8, batch=len(ctx), num_q_heads=16,
+                           num_kv_heads=4, head_dim=128, block_size=16, context_lens=ctx,
+                           seed=24, k_scale=0.125, v_scale=0.75)
+
+    def up(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        t = t.view(torch.float8_e4m3fn) if a.dtype == np.uint8 else t.view(torch.bfloat16)
+        return t.cuda()
+
+    d = dict(q=up(w.q), key_cache=up(w.key_cache), value_cache=up(w.value_cache),
+             block_tables=torch.from_numpy(w.block_tables).cuda(),
+             context_lens=torch.from_numpy(w.context_lens).cuda())
+    sc = dict(k_scale=w.k_scale, v_scale=w.v_scale)
+    B, Hq, D, P = w.batch, w.num_q_heads, w.head_dim, 64
+    maxp = -(-w.max_blocks * w.block_size // P)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = _splitk(d, P, maxp, B, Hq, D, err, sc)
+    out = torch.empty_like(d["q"])
+    pa.pa_reduce(out, *got, d["context_lens"], P, err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rm, rs, ro, f = oracle.partials(oracle.widen(w.q), oracle.dequantize(w.key_cache, w.k_scale),
+                                    oracle.dequantize(w.value_cache, w.v_scale), w.block_tables,
+                                    w.context_lens, P, maxp)
+    assert f == 0
+    _check_partials(got, (rm, rs, ro), wl.DTYPE_BF16, "fp8 Hkv 4")
+    ref, _ = oracle.decode_fp8(w.q, w.key_cache, w.value_cache, w.k_scale, w.v_scale,
+                               w.block_tables, w.context_lens, 1.0 / math.sqrt(w.head_dim))
+    assert_close(to_f64(out), ref, wl.DTYPE_BF16, "fp8 Hkv 4 split-K reduced")
+
+
 def test_splitk_bad_metadata_on_the_stream_kernel():
     """A bad block id gives that partition sum -1 (the others are intact); a
     bad length gives empty partitions everywhere; both flagged."""
