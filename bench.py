@@ -5,16 +5,21 @@ A step is one pass of the hot path over one batch: the cache write of every
 sequence's newest token via slot_mapping followed by the fused paged decode,
 through the C ABI -- by default as one pa_forward_decode call (the write
 happens inside the decode kernel), with ``--step separate`` as
-pa_write_kv_cache followed by pa_decode.  The default workload
-is the bf16 GQA decode batch (batch 32, 32 query / 8 KV heads, head_dim 128,
-block_size 16, context lengths uniform in [128, 2048]); other workloads are
-selectable with --workload.
+pa_write_kv_cache followed by pa_decode.  The default workload is
+mixed_bf16 (128 sequences of 128 / 4096 / 16000 tokens, 32 query / 8 KV
+heads, head_dim 128, block_size 16, 2.58 GB of pages), and the same line
+carries a second record (``--companion``, default gqa_bf16: batch 32,
+context lengths uniform in [128, 2048]); other workloads are selectable with
+--workload.  ``--step splitk`` times pa_write_kv_cache, pa_decode_splitk and
+pa_reduce (long_bf16 by default), ``--step prefix`` pa_write_kv_cache and
+pa_decode_shared_prefix (mqa_prefix_bf16 by default).
 
 Output: one JSON line on rank 0.  ``value`` is the achieved bandwidth on the
 algorithmic bytes of the step (unique K/V bytes of the visible tokens, block
 tables, context lengths, q, out and the new K/V rows) in GB/s, summed over
 ranks and divided by the slowest rank's time; each timed step is preceded by
-an L2 flush outside its CUDA-event pair.  ``e2e`` is the same metric with the
+an L2 flush outside its CUDA-event pair, and a 20 ms device sleep before the
+first timed step keeps the host's launches ahead of the device.  ``e2e`` is the same metric with the
 per-step inputs copied from pinned host memory and the output read back
 inside the timed region.  ``roofline`` reports the decode call (the whole
 step when fused) against the measured HBM copy bandwidth; ``cpu_baseline`` times the fp64 CPU
