@@ -192,3 +192,21 @@ def test_prefill_parity_record():
     bad = full.copy()
     bad[2, 0, 0] += 0.5  # outside the sample
     assert bench.prefill_parity(pw, s, bad)["within"]
+
+
+def test_staged_inputs_pack_a_step_into_one_copy(monkeypatch):
+    """The e2e loop's staging: every input lands in one buffer, 256-byte
+    aligned, and the device views equal the tensors they stand for."""
+    import torch
+
+    import bench
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)  # no device here
+    a = torch.arange(10, dtype=torch.int32)
+    b = torch.randn(3, 4).to(torch.bfloat16)
+    c = torch.arange(5, dtype=torch.int64)
+    dev_buf, host_buf, views = bench.staged_inputs([a, b, c], torch.device("cpu"))
+    assert torch.equal(views[0], a) and torch.equal(views[2], c)
+    assert torch.equal(views[1].view(torch.int16), b.view(torch.int16))
+    assert torch.equal(dev_buf, host_buf) and dev_buf.numel() == 3 * 256
+    for v in views:
+        assert (v.data_ptr() - dev_buf.data_ptr()) % 256 == 0
