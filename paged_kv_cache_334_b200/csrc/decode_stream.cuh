@@ -85,6 +85,9 @@ constexpr int kSeqCache = 256;
 // codes standing for code * scale.
 struct Fp8E4M3 {};
 
+// One staged page: its sequence, visible tokens, flags, split-K partition;
+// its physical block and first token in it; pad0 is the second block of a
+// two-block page (-1: the page ends in its first block).
 struct alignas(16) PageDesc {
   int32_t seq, ntok, flags, unit;  // unit: split-K partition index
   int32_t pb, toff, pad0, pad1;
