@@ -210,3 +210,22 @@ def test_staged_inputs_pack_a_step_into_one_copy(monkeypatch):
     assert torch.equal(dev_buf, host_buf) and dev_buf.numel() == 3 * 256
     for v in views:
         assert (v.data_ptr() - dev_buf.data_ptr()) % 256 == 0
+
+
+def test_recorded_traffic_follows_the_source_hash(tmp_path, monkeypatch):
+    """roofline.traffic comes from the row of the current kernel sources
+    only: a row under another hash, or no row, gives None."""
+    import bench
+    h = bench.decode_source_hash()
+    f = tmp_path / "traffic.md"
+    f.write_text("| workload | source hash | dram bytes per call |\n|---|---|---|\n"
+                 f"| gqa_bf16 | {h} | 123456 |\n"
+                 "| mixed_bf16 | 0000000000000000 | 999 |\n"
+                 f"| long_bf16/splitk | {h} | 777 |\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.recorded_traffic("gqa_bf16") == 123456.0
+    assert bench.recorded_traffic("long_bf16/splitk") == 777.0
+    assert bench.recorded_traffic("mixed_bf16") is None      # another hash
+    assert bench.recorded_traffic("gqa_fp8") is None         # no row
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "absent.md"))
+    assert bench.recorded_traffic("gqa_bf16") is None
